@@ -1,0 +1,356 @@
+"""Pins for the CPU oracle: checks against what the pages and mathematics fix.
+
+None of these re-types the oracle's formulas: each compares it with a printed
+value, a hand-worked example, an independent routine (scipy's normal quantile,
+torch's bf16 rounding, exact rational arithmetic, Python triple loops), a
+closed form or an invariant.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+from scipy.stats import norm
+
+from oracle import nf4_oracle as O
+from tests.conftest import golden_path, read_golden
+from qlora_linear_layers_nf4_b200 import workloads as WL
+
+
+def _printed_levels():
+    vals = []
+    with open(golden_path("nf4_levels_printed.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                vals.append(float(line))
+    return np.array(vals)
+
+
+# --------------------------------------------------------------------------- levels
+
+def test_levels_match_printed_table():
+    printed = _printed_levels()
+    assert printed.size == 16
+    lv = O.nf4_levels().astype(np.float64)
+    assert np.max(np.abs(lv - printed)) <= 5e-4 + 1e-12
+
+
+def test_levels_invariants():
+    lv = O.nf4_levels()
+    assert lv.dtype == np.float32
+    assert lv[0] == np.float32(-1.0) and lv[15] == np.float32(1.0)
+    assert lv[7] == 0.0 and np.sum(lv == 0.0) == 1
+    assert np.all(np.diff(lv) > 0)
+    assert np.sum(lv < 0) == 7 and np.sum(lv > 0) == 8
+
+
+def test_levels_against_scipy_quantiles():
+    # Independent normal quantile routine (scipy's ndtri) for the same construction.
+    delta = 1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0)
+    pos = norm.ppf(np.linspace(delta, 0.5, 9)[:-1])
+    neg = -norm.ppf(np.linspace(delta, 0.5, 8)[:-1])
+    ref = np.sort(np.concatenate([pos, neg, [0.0]]))
+    ref = ref / np.max(np.abs(ref))
+    assert np.max(np.abs(ref - O.nf4_levels_f64())) < 1e-12
+    # the fp32 table is far from any rounding boundary, so both routines give it bit for bit
+    assert np.array_equal(ref.astype(np.float32).view(np.uint32), O.nf4_levels().view(np.uint32))
+
+
+def test_levels_equally_likely_on_each_side():
+    # Page: levels at quantiles so each is equally likely.  Undo the normalisation
+    # and check the normal CDF of the raw positive / negative levels is evenly spaced.
+    lv = O.nf4_levels_f64()
+    scale = norm.ppf(1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0))
+    p_pos = norm.cdf(lv[7:] * scale)           # 0 and the 8 positive levels
+    p_neg = norm.cdf(-lv[:8] * scale)          # 0 and the 7 negative levels, mirrored
+    assert np.allclose(np.diff(p_pos), np.diff(p_pos)[0], rtol=1e-9, atol=1e-12)
+    assert np.allclose(np.diff(np.sort(p_neg)), np.diff(np.sort(p_neg))[0], rtol=1e-9, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- encode
+
+def _exact_nearest(v32: np.float32) -> int:
+    """Nearest level by exact rational arithmetic, lowest index on a tie."""
+    v = Fraction(float(v32))
+    best, best_d = None, None
+    for i, lev in enumerate(O.nf4_levels()):
+        d = abs(v - Fraction(float(lev)))
+        if best_d is None or d < best_d:
+            best, best_d = i, d
+    return best
+
+
+def _midpoint_neighbourhood():
+    lv = [Fraction(float(x)) for x in O.nf4_levels()]
+    vals = [np.float32(0.0), np.float32(-0.0)]
+    for i in range(15):
+        m = (lv[i] + lv[i + 1]) / 2
+        f = np.float32(float(m))
+        cand = [f]
+        up, dn = f, f
+        for _ in range(3):
+            up = np.nextafter(up, np.float32(2), dtype=np.float32)
+            dn = np.nextafter(dn, np.float32(-2), dtype=np.float32)
+            cand += [up, dn]
+        vals += cand
+    return np.array(vals, dtype=np.float32)
+
+
+def test_encode_matches_exact_arithmetic_at_midpoints():
+    vals = _midpoint_neighbourhood()
+    got = O.nearest_code(vals)
+    want = np.array([_exact_nearest(v) for v in vals], dtype=np.uint8)
+    assert np.array_equal(got, want)
+
+
+def test_exact_ties_go_to_lower_code():
+    lv = [Fraction(float(x)) for x in O.nf4_levels()]
+    ties = 0
+    for i in range(15):
+        m = (lv[i] + lv[i + 1]) / 2
+        f = np.float32(float(m))
+        if Fraction(float(f)) == m:          # midpoint representable in fp32: an exact tie
+            ties += 1
+            assert O.nearest_code(np.array([f]))[0] == i
+    assert ties == 4                         # four of the fifteen midpoints are fp32 numbers
+
+
+def test_levels_round_trip_to_own_code():
+    assert np.array_equal(O.nearest_code(O.nf4_levels()), np.arange(16, dtype=np.uint8))
+
+
+def test_worked_example_block():
+    g = read_golden("nf4_worked_example.txt")
+    w = np.array([float(v) for v in g["w"]], dtype=np.float32)
+    q = O.quantize(w, block_size=8)
+    assert q["absmax"][0] == np.float32(g["absmax"][0])
+    assert np.array_equal(O.unpack_codes(q["codes"]), np.array([int(c) for c in g["codes"]]))
+    assert np.array_equal(q["codes"], np.array([int(c, 16) for c in g["packed"]], dtype=np.uint8))
+
+
+def test_pack_unpack_lossless():
+    rng = np.random.default_rng(11)
+    c = rng.integers(0, 16, size=4096, dtype=np.uint8)
+    assert np.array_equal(O.unpack_codes(O.pack_codes(c)), c)
+    p = rng.integers(0, 256, size=1024, dtype=np.uint8)
+    assert np.array_equal(O.pack_codes(O.unpack_codes(p)), p)
+
+
+def _reciprocal_failures(n=64):
+    """fp32 values a with fp32(a * fp32(1/a)) != 1 (multiplying by a reciprocal is wrong here)."""
+    rng = np.random.default_rng(5)
+    a = (rng.random(200000, dtype=np.float32) * np.float32(0.1) + np.float32(1e-3)).astype(np.float32)
+    bad = a[(a * (np.float32(1.0) / a)).astype(np.float32) != np.float32(1.0)]
+    assert bad.size >= n
+    return bad[:n]
+
+
+def test_absmax_element_maps_to_pm_one_exactly():
+    bad = _reciprocal_failures()
+    rng = np.random.default_rng(3)
+    blocks = rng.standard_normal((bad.size, 64)).astype(np.float32) * np.float32(0.001)
+    idx = rng.integers(0, 64, size=bad.size)
+    sign = np.where(rng.random(bad.size) < 0.5, -1.0, 1.0).astype(np.float32)
+    blocks[np.arange(bad.size), idx] = sign * bad
+    q = O.quantize(blocks, 64)
+    codes = O.unpack_codes(q["codes"]).reshape(bad.size, 64)
+    got = codes[np.arange(bad.size), idx]
+    assert np.array_equal(got, np.where(sign > 0, 15, 0))
+    deq = O.dequantize(q).reshape(bad.size, 64)
+    assert np.array_equal(deq[np.arange(bad.size), idx], sign * bad)
+
+
+def test_all_zero_tensor_quantizes():
+    # export.rs unit tests quantize an all-zeros tensor and expect success.
+    q = O.quantize(np.zeros((32, 32), np.float32), 64, double=True)
+    assert np.all(q["codes"] == 0x77)
+    assert np.all(q["absmax"] == 0) and q["absmax_scale"] == 0 and np.all(q["absmax_q"] == 0)
+    d = O.dequantize(q)
+    assert np.all(d == 0) and not np.any(np.signbit(d))
+
+
+def test_scaled_levels_reproduce_exactly():
+    lv = O.nf4_levels()
+    rng = np.random.default_rng(2)
+    blocks = []
+    for e in range(-8, 4):
+        perm = rng.permutation(np.concatenate([np.arange(16)] * 4))
+        blocks.append((lv[perm] * np.float32(2.0 ** e)).astype(np.float32))
+    w = np.stack(blocks)
+    q = O.quantize(w, 64)
+    assert np.array_equal(O.dequantize(q), w)
+
+
+def test_round_trip_error_bound():
+    w = WL.draw_weight((256, 512), seed=9)
+    for double in (False, True):
+        q = O.quantize(w, 64, double=double)
+        d = O.dequantize(q)
+        lv = O.nf4_levels().astype(np.float64)
+        half_gap = np.max(np.diff(lv)) / 2           # 0.1519, between -1 and -0.696
+        assert abs(half_gap - 0.15190359) < 1e-6
+        absmax = np.repeat(q["absmax"], 64).reshape(w.shape).astype(np.float64)
+        bound = absmax * half_gap * (1 + 1e-6)
+        if double:
+            scale = np.repeat(O.block_scales(q), 64).reshape(w.shape).astype(np.float64)
+            bound = bound + np.abs(scale - absmax) + 1e-12
+        assert np.all(np.abs(w.astype(np.float64) - d) <= bound + 1e-12)
+
+
+def test_refuses_bad_shapes_and_nonfinite():
+    with pytest.raises(ValueError):
+        O.quantize(np.zeros(100, np.float32), 64)
+    with pytest.raises(ValueError):
+        O.quantize(np.zeros(64, np.float32), 63)
+    w = np.zeros(64, np.float32)
+    w[3] = np.inf
+    with pytest.raises(ValueError):
+        O.quantize(w, 64)
+
+
+# --------------------------------------------------------------------------- double quant
+
+def test_double_quant_invariants():
+    w = WL.draw_weight((512, 256), seed=4)
+    q = O.quantize(w, 64, double=True)
+    absmax = q["absmax"].astype(np.float64)
+    s_g = float(q["absmax_scale"])
+    assert q["absmax_q"][np.argmax(absmax)] == 255
+    assert abs(s_g - absmax.max() / 255) <= 1e-7 * s_g
+    dec = O.block_scales(q).astype(np.float64)
+    assert np.all(np.abs(dec - absmax) <= s_g / 2 + 4 * np.spacing(absmax.astype(np.float32)))
+    order = np.argsort(absmax, kind="stable")
+    assert np.all(np.diff(q["absmax_q"][order].astype(int)) >= 0)       # monotone
+
+
+def test_double_quant_half_even_rounding():
+    # absmax values chosen so absmax / s_g lands exactly on k + 0.5 for small k.
+    s_g = np.float32(255.0) / np.float32(255.0)
+    absmax = np.array([255.0, 0.5, 1.5, 2.5, 3.5, 254.5], dtype=np.float32)
+    q, sg = O.double_quant(absmax)
+    assert sg == s_g
+    assert list(q) == [255, 0, 2, 2, 4, 254]
+
+
+# --------------------------------------------------------------------------- dequant rounding
+
+def test_bf16_round_matches_torch():
+    import torch
+    rng = np.random.default_rng(8)
+    x = np.concatenate([
+        rng.standard_normal(100000).astype(np.float32) * np.float32(0.02),
+        np.array([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38, 1e-40], dtype=np.float32),
+    ])
+    u = rng.integers(0, 2 ** 16, size=5000, dtype=np.uint32) << 16 | np.uint32(0x8000)
+    x = np.concatenate([x, u.view(np.float32)[np.isfinite(u.view(np.float32))]])
+    ours = O.bf16_round(x)
+    theirs = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, theirs)
+
+
+def test_dequant_single_product_per_element():
+    lv = O.nf4_levels()
+    rng = np.random.default_rng(1)
+    w = WL.draw_weight((64, 128), seed=21)
+    q = O.quantize(w, 64)
+    d = O.dequantize(q)
+    codes = O.unpack_codes(q["codes"]).reshape(64, 128)
+    # element by element in Python floats rounded once to fp32
+    for _ in range(200):
+        i, j = rng.integers(0, 64), rng.integers(0, 128)
+        s = q["absmax"][(i * 128 + j) // 64]
+        assert d[i, j] == np.float32(float(lv[codes[i, j]]) * float(s))
+
+
+# --------------------------------------------------------------------------- forward / backward
+
+def test_worked_linear_example():
+    g = read_golden("qlora_worked_example.txt")
+    f = lambda k: np.array([float(v) for v in g[k]])
+    x, w, a, b = f("x")[None, :], f("w")[None, :], f("a")[None, :], f("b")[None, :]
+    alpha = float(g["alpha"][0])
+    y, t = O.qlora_forward(x, w, a, b, alpha)
+    assert y[0, 0] == float(g["y"][0]) and t[0, 0] == float(g["t"][0])
+    d_a, d_b, d_x = O.qlora_backward(x, w, a, b, alpha, f("dy")[None, :])
+    assert np.array_equal(d_b.ravel(), f("dB"))
+    assert np.array_equal(d_a.ravel(), f("dA"))
+    assert np.array_equal(d_x.ravel(), f("dx"))
+
+
+def _tiny():
+    inp = WL.draw_linear(WL.TINY)
+    q = O.quantize(inp.w, 64)
+    w_hat = O.bf16_to_f32(O.dequantize(q, "bf16"))
+    f = WL.bf16_bits_to_f32
+    return inp, w_hat, f(inp.x), f(inp.a), f(inp.b), f(inp.dy)
+
+
+def test_forward_matches_bruteforce():
+    inp, w_hat, x, a, b, dy = _tiny()
+    y, t = O.qlora_forward(x, w_hat, a, b, inp.case.alpha)
+    s = inp.case.alpha / inp.case.r
+    t_bf = O.matmul_bruteforce(x, a.T)
+    y_bf = O.matmul_bruteforce(x, w_hat.T) + s * O.matmul_bruteforce(t_bf, b.T)
+    assert np.max(np.abs(y - y_bf)) <= 1e-12 * np.max(np.abs(y_bf))
+    assert np.max(np.abs(t - t_bf)) <= 1e-12 * np.max(np.abs(t_bf))
+
+
+def test_merge_identity():
+    # Equation 6.3.6: x (W' + (alpha/r) B A)^T equals the adapter-on-base forward.
+    inp, w_hat, x, a, b, dy = _tiny()
+    y, _ = O.qlora_forward(x, w_hat, a, b, inp.case.alpha)
+    merged = w_hat.astype(np.float64) + (inp.case.alpha / inp.case.r) * O.matmul_bruteforce(b, a)
+    y2 = O.matmul_bruteforce(x, merged.T)
+    assert np.max(np.abs(y - y2)) <= 1e-11 * np.max(np.abs(y))
+
+
+def test_special_cases():
+    inp, w_hat, x, a, b, dy = _tiny()
+    alpha = inp.case.alpha
+    # B = 0: the base matmul alone
+    y0, _ = O.qlora_forward(x, w_hat, a, np.zeros_like(b), alpha)
+    assert np.array_equal(y0, x.astype(np.float64) @ w_hat.T.astype(np.float64))
+    # zero base weight: only the adapter term remains
+    q0 = O.quantize(np.zeros_like(inp.w), 64)
+    w0 = O.bf16_to_f32(O.dequantize(q0, "bf16"))
+    assert np.all(w0 == 0)
+    ya, t = O.qlora_forward(x, w0, a, b, alpha)
+    assert np.allclose(ya, (alpha / inp.case.r) * O.matmul_bruteforce(O.matmul_bruteforce(x, a.T), b.T),
+                       rtol=1e-12, atol=1e-15)
+    # A = 0: dB vanishes
+    d_a, d_b, d_x = O.qlora_backward(x, w_hat, np.zeros_like(a), b, alpha, dy)
+    assert np.all(d_b == 0)
+
+
+def test_finite_difference_gradients():
+    inp, w_hat, x, a, b, dy = _tiny()
+    alpha = inp.case.alpha
+    x, a, b, dy = (v.astype(np.float64) for v in (x, a, b, dy))
+    d_a, d_b, d_x = O.qlora_backward(x, w_hat, a, b, alpha, dy)
+
+    def loss(xx, aa, bb):
+        return float(np.sum(dy * O.qlora_forward(xx, w_hat, aa, bb, alpha)[0]))
+
+    h = 1e-3
+    rng = np.random.default_rng(0)
+    for i in range(a.shape[0]):
+        for j in range(0, a.shape[1], 7):
+            ap, am = a.copy(), a.copy()
+            ap[i, j] += h
+            am[i, j] -= h
+            fd = (loss(x, ap, b) - loss(x, am, b)) / (2 * h)
+            assert abs(fd - d_a[i, j]) <= 1e-8 * max(1.0, abs(d_a[i, j]))
+    for i in range(0, b.shape[0], 5):
+        for j in range(b.shape[1]):
+            bp, bm = b.copy(), b.copy()
+            bp[i, j] += h
+            bm[i, j] -= h
+            fd = (loss(x, a, bp) - loss(x, a, bm)) / (2 * h)
+            assert abs(fd - d_b[i, j]) <= 1e-8 * max(1.0, abs(d_b[i, j]))
+    for _ in range(256):
+        i, j = rng.integers(0, x.shape[0]), rng.integers(0, x.shape[1])
+        xp, xm = x.copy(), x.copy()
+        xp[i, j] += h
+        xm[i, j] -= h
+        fd = (loss(xp, a, b) - loss(xm, a, b)) / (2 * h)
+        assert abs(fd - d_x[i, j]) <= 1e-8 * max(1.0, abs(d_x[i, j]))
