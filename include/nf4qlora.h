@@ -1,0 +1,225 @@
+/*
+ * nf4qlora.h -- C ABI of the B200 (sm_100a) NF4 quantization and QLoRA
+ * linear-layer library (libnf4qlora.so).
+ *
+ * What it computes (sources are the web pages on the subject):
+ *   - NF4 quantization: qlora-rs README, "Honest capability matrix" (NF4
+ *     pack/unpack + block absmax scales; simplified double quant) and
+ *     "Quick Start" (quantize_nf4(&weights, 64)); "LoRA and QLoRA,
+ *     mathematically", section "NF4: quantizing the frozen base" (sixteen
+ *     levels at normal quantiles).  Storage follows the QuantizedTensor fields
+ *     shown on the qlora-rs src/export.rs page (data, scales,
+ *     scales_quantized, scales_scales, shape).
+ *   - QLoRA linear: y = x W'^T + (alpha/r) (x A^T) B^T with W' the dequantized
+ *     base in the compute dtype ("LoRA and QLoRA, mathematically", sections
+ *     "Rank, alpha, and target modules" and "The merge math", equation 6.3.6;
+ *     rust-ai-core QLoraConfig, scale() = alpha / r and "Compute Dtype").
+ *   - Adapter backward of L = sum(dy * y) with W frozen:
+ *     dB = s dy^T (x A^T), dA = s (dy B)^T x, dx = dy W' + s (dy B) A.
+ *
+ * Conventions shared by every entry point
+ *   Memory     Every pointer argument is DEVICE memory owned by the caller,
+ *              unless stated otherwise.  The library keeps no pointer after a
+ *              call returns and allocates no device memory.
+ *   Streams    `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *              default stream).  All work is enqueued on it; buffers must stay
+ *              alive until it completes.  Nothing synchronizes except
+ *              nf4_read_status.
+ *   Layouts    Row-major, densely packed.  W is [rows = N out, cols = K in].
+ *              x is [M, K], A is [r, K], B is [N, r], y and dy are [M, N].
+ *   Alignment  Device pointers must be 16-byte aligned (NF4_ERR_ALIGNMENT).
+ *   Errors     Arguments are validated on the host before anything is
+ *              launched; a call that returns an error has enqueued nothing.
+ *              Conditions only the GPU can see (non-finite input to quantize,
+ *              an internal wait that exceeded its limit) are recorded in the
+ *              status word at the head of `workspace` and returned by
+ *              nf4_read_status.
+ *   Workspace  Caller-allocated device scratch of at least
+ *              nf4_workspace_bytes(...) bytes, zero-filled once before first
+ *              use (the status word must start at 0).  Calls that share a
+ *              workspace must be ordered on one stream.
+ */
+#ifndef NF4QLORA_H_
+#define NF4QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NF4_API __attribute__((visibility("default")))
+#else
+#define NF4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NF4_OK = 0,
+  NF4_ERR_INVALID_ARG = 1,  /* NULL where a pointer is required, r out of range, ...   */
+  NF4_ERR_SHAPE = 2,        /* sizes the operation does not accept                    */
+  NF4_ERR_ALIGNMENT = 3,    /* a pointer that is not 16-byte aligned                  */
+  NF4_ERR_UNSUPPORTED = 4,  /* a valid request this build does not implement          */
+  NF4_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than nf4_workspace_bytes     */
+  NF4_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed (launch error, ...)  */
+  NF4_ERR_NONFINITE = 7,    /* device-detected: NaN or Inf in the quantize input      */
+  NF4_ERR_TIMEOUT = 8       /* device-detected: an internal wait exceeded its limit   */
+} nf4_status;
+
+typedef enum { NF4_F32 = 0, NF4_BF16 = 1, NF4_F16 = 2 } nf4_dtype;
+
+typedef enum {
+  NF4_OP_QUANTIZE = 0,
+  NF4_OP_DEQUANTIZE = 1,
+  NF4_OP_LINEAR_FWD = 2,
+  NF4_OP_LINEAR_BWD = 3
+} nf4_op;
+
+/*
+ * A quantized weight, mirroring the QuantizedTensor of the qlora-rs
+ * src/export.rs page (data -> codes, scales -> absmax, scales_quantized ->
+ * absmax_q, scales_scales -> absmax_scale, shape -> rows/cols).  Asymmetric
+ * zero-points are not part of NF4 and are not represented.
+ *   codes         rows*cols/2 bytes.  Element e of the row-major flattened
+ *                 tensor has a 4-bit code in byte e/2: the HIGH nibble for
+ *                 even e, the LOW nibble for odd e.
+ *   absmax        fp32 per block (rows*cols/block_size), block b covering
+ *                 elements [b*block_size, (b+1)*block_size).  Used when
+ *                 double_quant == 0.  May be NULL when double_quant != 0.
+ *   absmax_q      u8 per block, used when double_quant != 0.
+ *   absmax_scale  one fp32 (the scale of the scales), used when
+ *                 double_quant != 0.  Block b decodes with
+ *                 scale_b = fp32((float)absmax_q[b] * absmax_scale[0]).
+ */
+typedef struct {
+  const uint8_t* codes;
+  const float* absmax;
+  const uint8_t* absmax_q;
+  const float* absmax_scale;
+  int64_t rows;
+  int64_t cols;
+  int32_t block_size;
+  int32_t double_quant;
+} nf4_weight;
+
+/* Human-readable name of a status code (static string, never NULL). */
+NF4_API const char* nf4_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+NF4_API int nf4_version(void);
+
+/*
+ * Host copy of the device codebook.  levels[i] is the fp32 NF4 level of code
+ * i (ascending, levels[0] = -1, levels[7] = 0, levels[15] = +1).
+ * thresholds[i] is the largest fp32 value not above the exact midpoint of
+ * levels[i] and levels[i+1]; the encoder's code for a normalised value v is
+ * the number of thresholds strictly below v (nearest level, lower code on an
+ * exact tie).  Either pointer may be NULL.  Host memory; needs no GPU.
+ */
+NF4_API void nf4_codebook(float* levels, float* thresholds);
+
+/*
+ * Number of kernel launches the library has made in this process (host-side
+ * counter, incremented once per successful launch).  Needs no GPU.
+ */
+NF4_API int64_t nf4_launch_count(void);
+
+/*
+ * Bytes of workspace an operation needs (0 = none).  M, N, K, r are the
+ * linear-layer sizes (N = W rows, K = W cols); for NF4_OP_QUANTIZE and
+ * NF4_OP_DEQUANTIZE pass N = rows, K = cols and M = r = 0.  Needs no GPU.
+ */
+NF4_API size_t nf4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r, int block_size,
+                           int double_quant);
+
+/*
+ * Synchronizes `stream`, returns the device status recorded in `workspace`
+ * since the last call (NF4_OK if none), and resets it to NF4_OK.  A failing
+ * CUDA call gives NF4_ERR_CUDA.
+ */
+NF4_API nf4_status nf4_read_status(void* workspace, void* stream);
+
+/*
+ * Blockwise NF4 quantization (qlora-rs quantize_nf4; capability matrix
+ * "NF4 pack/unpack + block absmax scales" and "Double quant (simplified
+ * global u8 scales)").
+ *   w            fp32 [rows, cols], read only.
+ *   block_size   positive and even; rows*cols must be a multiple of it.
+ *                Multiples of 8 up to 256 that are powers of two take the
+ *                vectorized path; other even sizes a per-block path.
+ *   For each block: absmax = max |w|; v = w / absmax (IEEE fp32 division);
+ *   code = index of the nearest NF4 level (lower code on an exact tie);
+ *   absmax == 0 gives code 7 for the whole block.
+ *   codes        u8 [rows*cols/2], written (packing as in nf4_weight).
+ *   absmax       fp32 [nblocks]; written when non-NULL.  Required when
+ *                double_quant == 0.
+ *   double_quant 0 or 1.  When 1: G = max absmax, absmax_scale[0] =
+ *                fp32(G / 255) and absmax_q[b] = clamp(rint(absmax_b /
+ *                absmax_scale), 0, 255) with ties to even; G == 0 gives 0
+ *                and 0.  absmax_q (u8 [nblocks]) and absmax_scale (fp32[1])
+ *                are then required.  The codes do not depend on
+ *                double_quant.
+ *   workspace    >= nf4_workspace_bytes(NF4_OP_QUANTIZE, ...).
+ * NaN/Inf in w is outside the contract: the kernels flag NF4_ERR_NONFINITE
+ * in the workspace status word (the outputs are then unspecified).
+ */
+NF4_API nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int block_size,
+                        int double_quant, uint8_t* codes, float* absmax, uint8_t* absmax_q,
+                        float* absmax_scale, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Dequantization (qlora-rs dequantize_nf4; "Honor compute_dtype
+ * (BF16/F16/F32) in forward dequant").  out[e] = fp32(L[code_e] * scale_b)
+ * as one fp32 product; NF4_BF16 / NF4_F16 store its round-to-nearest-even.
+ *   w->block_size must be a positive multiple of 8; out has rows*cols
+ *   elements of out_dtype.
+ */
+NF4_API nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out, void* stream);
+
+/*
+ * QLoRA linear forward (QuantizedLinear::forward of the qlora-rs README;
+ * equation 6.3.6 of "LoRA and QLoRA, mathematically" read as a layer):
+ *   y = x W'^T + s (x A^T) B^T (+ bias),  s = alpha / r,
+ * W' the dequantized base rounded to compute_dtype, operands in
+ * compute_dtype, fp32 accumulation, y rounded to compute_dtype.
+ *   w              N = w->rows (out), K = w->cols (in); block_size 64;
+ *                  K % 64 == 0, N % 8 == 0.
+ *   x              [M, K] compute_dtype; M >= 1.
+ *   A, B           [r, K] and [N, r] compute_dtype; 8 <= r <= 256, r % 8 == 0.
+ *   compute_dtype  NF4_BF16 (NF4_F16 / NF4_F32 give NF4_ERR_UNSUPPORTED).
+ *   bias           [N] compute_dtype, or NULL.
+ *   y              [M, N] compute_dtype, written.
+ *   t_out          [M, r] compute_dtype, or NULL: when given, receives
+ *                  T = s (x A^T) rounded to compute_dtype, which
+ *                  qlora_linear_bwd accepts as `t`.
+ *   workspace      >= nf4_workspace_bytes(NF4_OP_LINEAR_FWD, M, N, K, r, 64, dq).
+ * M <= 32 uses the weight-streaming decode path, larger M the fused
+ * dequantize + tensor-core GEMM; both compute the same function.
+ */
+NF4_API nf4_status qlora_linear_fwd(const nf4_weight* w, const void* x, int64_t M, const void* A,
+                            const void* B, int r, float alpha, int compute_dtype,
+                            const void* bias, void* y, void* t_out, void* workspace,
+                            size_t ws_bytes, void* stream);
+
+/*
+ * QLoRA linear adapter backward for L = sum(dy * y), the base W frozen
+ * (qlora-rs capability matrix: adapters train on a frozen NF4 base):
+ *   U  = s (dy B)                                [M, r]
+ *   dB = s dy^T (x A^T)  = dy^T T                 fp32 [N, r], overwritten
+ *   dA = s (dy B)^T x    = U^T x                  fp32 [r, K], overwritten
+ *   dx = dy W' + s (dy B) A = dy W' + U A         [M, K] compute_dtype, or NULL
+ * Arguments as for qlora_linear_fwd; dy is [M, N] compute_dtype; `t` is the
+ * T written by the forward's t_out, or NULL to recompute it.
+ *   workspace      >= nf4_workspace_bytes(NF4_OP_LINEAR_BWD, M, N, K, r, 64, dq).
+ */
+NF4_API nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const void* A,
+                            const void* B, int r, float alpha, int compute_dtype,
+                            const void* dy, const void* t, float* dA, float* dB, void* dx,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NF4QLORA_H_ */

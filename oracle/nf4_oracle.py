@@ -114,9 +114,15 @@ def nearest_code(v: np.ndarray) -> np.ndarray:
     then returns the first (lowest) index, which is the tie rule of R4.
     """
     levels = nf4_levels().astype(np.float64)
-    v = np.asarray(v, dtype=np.float32).astype(np.float64)
-    dist = np.abs(v[..., None] - levels)
-    return np.argmin(dist, axis=-1).astype(np.uint8)
+    v = np.asarray(v, dtype=np.float32)
+    flat = v.reshape(-1)
+    out = np.empty(flat.size, dtype=np.uint8)
+    step = 1 << 20                      # elementwise; the loop only bounds memory use
+    for lo in range(0, flat.size, step):
+        chunk = flat[lo:lo + step].astype(np.float64)
+        dist = np.abs(chunk[:, None] - levels)
+        out[lo:lo + step] = np.argmin(dist, axis=-1)
+    return out.reshape(v.shape)
 
 
 def pack_codes(codes: np.ndarray) -> np.ndarray:

@@ -1,0 +1,265 @@
+// C-ABI entry points: argument validation on the host, then launches.
+// Every check happens before anything is enqueued, so an error return means
+// the stream was left untouched (the "refuse before writing anything" rule).
+#include <atomic>
+#include <cstring>
+
+#include "nf4_common.cuh"
+#include "kernels.h"
+
+namespace {
+
+std::atomic<int64_t> g_launches{0};
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+nf4_status finish(cudaError_t e, int launches) {
+  g_launches += launches;
+  return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t quantize_ws(int64_t numel, int bs, int dq) {
+  size_t bytes = nf4::kWsHeader;
+  if (dq && bs > 0 && numel > 0) bytes += round_up(size_t(numel / bs) * sizeof(float), 256);
+  return bytes;
+}
+
+// Checks shared by the two linear entry points.
+nf4_status check_linear(const nf4_weight* w, const void* x, int64_t M, const void* A,
+                        const void* B, int r, float alpha, int compute_dtype) {
+  if (w == nullptr || x == nullptr || A == nullptr || B == nullptr || w->codes == nullptr)
+    return NF4_ERR_INVALID_ARG;
+  if (w->double_quant) {
+    if (w->absmax_q == nullptr || w->absmax_scale == nullptr) return NF4_ERR_INVALID_ARG;
+  } else if (w->absmax == nullptr) {
+    return NF4_ERR_INVALID_ARG;
+  }
+  if (!(alpha == alpha) || r < 8 || r > 256 || (r % 8) != 0) return NF4_ERR_INVALID_ARG;
+  if (compute_dtype != NF4_BF16) {
+    if (compute_dtype == NF4_F16 || compute_dtype == NF4_F32) return NF4_ERR_UNSUPPORTED;
+    return NF4_ERR_INVALID_ARG;
+  }
+  if (M < 1 || w->rows < 1 || w->cols < 1) return NF4_ERR_SHAPE;
+  if (w->block_size != 64) return NF4_ERR_UNSUPPORTED;
+  if (w->cols % 64 != 0 || w->rows % 8 != 0) return NF4_ERR_SHAPE;
+  if (M > (int64_t(1) << 31) || w->rows > (int64_t(1) << 31) || w->cols > (int64_t(1) << 31))
+    return NF4_ERR_SHAPE;
+  if (!aligned16(w->codes) || !aligned16(x) || !aligned16(A) || !aligned16(B))
+    return NF4_ERR_ALIGNMENT;
+  if (w->double_quant ? (!aligned16(w->absmax_q) || !aligned4(w->absmax_scale))
+                      : !aligned16(w->absmax))
+    return NF4_ERR_ALIGNMENT;
+  return NF4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nf4_status_string(int status) {
+  switch (status) {
+    case NF4_OK: return "NF4_OK";
+    case NF4_ERR_INVALID_ARG: return "NF4_ERR_INVALID_ARG: invalid argument";
+    case NF4_ERR_SHAPE: return "NF4_ERR_SHAPE: unsupported shape";
+    case NF4_ERR_ALIGNMENT: return "NF4_ERR_ALIGNMENT: pointer not 16-byte aligned";
+    case NF4_ERR_UNSUPPORTED: return "NF4_ERR_UNSUPPORTED: not implemented in this build";
+    case NF4_ERR_WORKSPACE: return "NF4_ERR_WORKSPACE: workspace missing or too small";
+    case NF4_ERR_CUDA: return "NF4_ERR_CUDA: CUDA call failed";
+    case NF4_ERR_NONFINITE: return "NF4_ERR_NONFINITE: NaN or Inf in quantize input";
+    case NF4_ERR_TIMEOUT: return "NF4_ERR_TIMEOUT: device wait exceeded its limit";
+    default: return "unknown nf4 status";
+  }
+}
+
+int nf4_version(void) { return 100; }
+
+void nf4_codebook(float* levels, float* thresholds) {
+  if (levels != nullptr)
+    for (int i = 0; i < 16; ++i) std::memcpy(&levels[i], &nf4::kLevelBits[i], 4);
+  if (thresholds != nullptr)
+    for (int i = 0; i < 15; ++i) std::memcpy(&thresholds[i], &nf4::kThresholdBits[i], 4);
+}
+
+int64_t nf4_launch_count(void) { return g_launches.load(); }
+
+size_t nf4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r, int block_size,
+                           int double_quant) {
+  switch (op) {
+    case NF4_OP_QUANTIZE: return quantize_ws(N * K, block_size, double_quant);
+    case NF4_OP_DEQUANTIZE: return 0;
+    case NF4_OP_LINEAR_FWD: return nf4::kWsHeader + nf4::linear_workspace_bytes(false, M, N, K, r);
+    case NF4_OP_LINEAR_BWD: return nf4::kWsHeader + nf4::linear_workspace_bytes(true, M, N, K, r);
+    default: return 0;
+  }
+}
+
+nf4_status nf4_read_status(void* workspace, void* stream) {
+  if (workspace == nullptr) return NF4_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t host = 0;
+  uint32_t* dev = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + nf4::kWsStatus);
+  if (cudaMemcpyAsync(&host, dev, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return NF4_ERR_CUDA;
+  if (cudaMemsetAsync(dev, 0, sizeof(uint32_t), st) != cudaSuccess) return NF4_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return NF4_ERR_CUDA;
+  return static_cast<nf4_status>(host);
+}
+
+nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int block_size,
+                        int double_quant, uint8_t* codes, float* absmax, uint8_t* absmax_q,
+                        float* absmax_scale, void* workspace, size_t ws_bytes, void* stream) {
+  if (rows < 0 || cols < 0) return NF4_ERR_SHAPE;
+  if (block_size <= 0 || (block_size % 2) != 0) return NF4_ERR_SHAPE;
+  if (double_quant != 0 && double_quant != 1) return NF4_ERR_INVALID_ARG;
+  if (rows != 0 && cols > INT64_MAX / rows) return NF4_ERR_SHAPE;
+  const int64_t numel = rows * cols;
+  if (numel % block_size != 0) return NF4_ERR_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (numel == 0) {  // empty tensor: nothing to encode; the scale of no scales is 0
+    if (double_quant && absmax_scale != nullptr) {
+      if (!aligned4(absmax_scale)) return NF4_ERR_ALIGNMENT;
+      if (cudaMemsetAsync(absmax_scale, 0, sizeof(float), st) != cudaSuccess) return NF4_ERR_CUDA;
+    }
+    return NF4_OK;
+  }
+  if (w == nullptr || codes == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!double_quant && absmax == nullptr) return NF4_ERR_INVALID_ARG;
+  if (double_quant && (absmax_q == nullptr || absmax_scale == nullptr)) return NF4_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(codes) || (absmax && !aligned16(absmax)) ||
+      (absmax_q && !aligned16(absmax_q)) || (absmax_scale && !aligned4(absmax_scale)))
+    return NF4_ERR_ALIGNMENT;
+  if (workspace == nullptr || !aligned16(workspace)) return NF4_ERR_WORKSPACE;
+  if (ws_bytes < quantize_ws(numel, block_size, double_quant)) return NF4_ERR_WORKSPACE;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + nf4::kWsStatus);
+  uint32_t* gmax = reinterpret_cast<uint32_t*>(ws + nf4::kWsGlobalMax);
+  const int sms = sm_count();
+  int launches = 0;
+  cudaError_t e = cudaSuccess;
+  float* amax = absmax;
+  if (double_quant) {
+    if (amax == nullptr) amax = reinterpret_cast<float*>(ws + nf4::kWsHeader);
+    e = cudaMemsetAsync(gmax, 0, sizeof(uint32_t), st);
+  }
+  if (e == cudaSuccess)
+    e = nf4::launch_quantize(w, numel, block_size, codes, amax, status,
+                             double_quant ? gmax : nullptr, sms, st, &launches);
+  if (e == cudaSuccess && double_quant)
+    e = nf4::launch_double_quant(amax, numel / block_size, gmax, absmax_q, absmax_scale, sms, st,
+                                 &launches);
+  return finish(e, launches);
+}
+
+nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out, void* stream) {
+  if (w == nullptr || out == nullptr || w->codes == nullptr) return NF4_ERR_INVALID_ARG;
+  if (out_dtype != NF4_F32 && out_dtype != NF4_BF16 && out_dtype != NF4_F16)
+    return NF4_ERR_INVALID_ARG;
+  if (w->rows < 0 || w->cols < 0) return NF4_ERR_SHAPE;
+  if (w->block_size <= 0 || (w->block_size % 8) != 0) return NF4_ERR_SHAPE;
+  if (w->rows != 0 && w->cols > INT64_MAX / w->rows) return NF4_ERR_SHAPE;
+  const int64_t numel = w->rows * w->cols;
+  if (numel % w->block_size != 0) return NF4_ERR_SHAPE;
+  if (w->double_quant) {
+    if (w->absmax_q == nullptr || w->absmax_scale == nullptr) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(w->absmax_q) || !aligned4(w->absmax_scale)) return NF4_ERR_ALIGNMENT;
+  } else {
+    if (w->absmax == nullptr) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(w->absmax)) return NF4_ERR_ALIGNMENT;
+  }
+  if (!aligned16(w->codes) || !aligned16(out)) return NF4_ERR_ALIGNMENT;
+  if (numel == 0) return NF4_OK;
+  int launches = 0;
+  cudaError_t e = nf4::launch_dequantize(*w, out_dtype, out, sm_count(),
+                                         static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
+}
+
+nf4_status qlora_linear_fwd(const nf4_weight* w, const void* x, int64_t M, const void* A,
+                            const void* B, int r, float alpha, int compute_dtype,
+                            const void* bias, void* y, void* t_out, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  nf4_status s = check_linear(w, x, M, A, B, r, alpha, compute_dtype);
+  if (s != NF4_OK) return s;
+  if (y == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!aligned16(y) || (bias && !aligned16(bias)) || (t_out && !aligned16(t_out)))
+    return NF4_ERR_ALIGNMENT;
+  if (workspace == nullptr || !aligned16(workspace)) return NF4_ERR_WORKSPACE;
+  if (ws_bytes < nf4_workspace_bytes(NF4_OP_LINEAR_FWD, M, w->rows, w->cols, r, 64,
+                                     w->double_quant))
+    return NF4_ERR_WORKSPACE;
+  nf4::LinearArgs a{};
+  a.w = w;
+  a.M = M;
+  a.N = w->rows;
+  a.K = w->cols;
+  a.r = r;
+  a.s = alpha / float(r);
+  a.x = x;
+  a.A = A;
+  a.B = B;
+  a.bias = bias;
+  a.y = y;
+  a.t_out = t_out;
+  a.ws = static_cast<uint8_t*>(workspace);
+  a.ws_bytes = ws_bytes;
+  a.status = reinterpret_cast<uint32_t*>(a.ws + nf4::kWsStatus);
+  int launches = 0;
+  cudaError_t e = nf4::launch_linear_fwd(a, sm_count(), static_cast<cudaStream_t>(stream),
+                                         &launches);
+  if (e == cudaErrorNotSupported) { g_launches += launches; return NF4_ERR_UNSUPPORTED; }
+  return finish(e, launches);
+}
+
+nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const void* A,
+                            const void* B, int r, float alpha, int compute_dtype,
+                            const void* dy, const void* t, float* dA, float* dB, void* dx,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  nf4_status s = check_linear(w, x, M, A, B, r, alpha, compute_dtype);
+  if (s != NF4_OK) return s;
+  if (dy == nullptr || dA == nullptr || dB == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(dA) || !aligned16(dB) || (dx && !aligned16(dx)) ||
+      (t && !aligned16(t)))
+    return NF4_ERR_ALIGNMENT;
+  if (workspace == nullptr || !aligned16(workspace)) return NF4_ERR_WORKSPACE;
+  if (ws_bytes < nf4_workspace_bytes(NF4_OP_LINEAR_BWD, M, w->rows, w->cols, r, 64,
+                                     w->double_quant))
+    return NF4_ERR_WORKSPACE;
+  nf4::LinearArgs a{};
+  a.w = w;
+  a.M = M;
+  a.N = w->rows;
+  a.K = w->cols;
+  a.r = r;
+  a.s = alpha / float(r);
+  a.x = x;
+  a.A = A;
+  a.B = B;
+  a.dy = dy;
+  a.t_in = t;
+  a.dA = dA;
+  a.dB = dB;
+  a.dx = dx;
+  a.ws = static_cast<uint8_t*>(workspace);
+  a.ws_bytes = ws_bytes;
+  a.status = reinterpret_cast<uint32_t*>(a.ws + nf4::kWsStatus);
+  int launches = 0;
+  cudaError_t e = nf4::launch_linear_bwd(a, sm_count(), static_cast<cudaStream_t>(stream),
+                                         &launches);
+  if (e == cudaErrorNotSupported) { g_launches += launches; return NF4_ERR_UNSUPPORTED; }
+  return finish(e, launches);
+}
+
+}  // extern "C"

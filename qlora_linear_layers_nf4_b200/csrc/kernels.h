@@ -1,0 +1,50 @@
+// Internal launchers (host side).  Each returns the CUDA error of its launch
+// and increments *launches once per kernel it launched successfully.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/nf4qlora.h"
+
+namespace nf4 {
+
+cudaError_t launch_quantize(const float* w, int64_t numel, int bs, uint8_t* codes,
+                            float* absmax_out, uint32_t* status, uint32_t* gmax, int sms,
+                            cudaStream_t stream, int* launches);
+
+cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uint32_t* gmax,
+                                uint8_t* absmax_q, float* absmax_scale, int sms,
+                                cudaStream_t stream, int* launches);
+
+cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int sms,
+                              cudaStream_t stream, int* launches);
+
+// ---- QLoRA linear (qlora_gemm.cu) ----
+
+struct LinearArgs {
+  const nf4_weight* w;
+  int64_t M, N, K;
+  int r;
+  float s;                 // alpha / r
+  const void* x;           // [M, K] bf16
+  const void* A;           // [r, K] bf16
+  const void* B;           // [N, r] bf16
+  const void* bias;        // [N] bf16 or null
+  const void* dy;          // [M, N] bf16 (backward)
+  const void* t_in;        // [M, r] bf16 T = s x A^T (backward, may be null)
+  void* y;                 // [M, N] bf16
+  void* t_out;             // [M, r] bf16 (forward, may be null)
+  float* dA;               // [r, K] fp32
+  float* dB;               // [N, r] fp32
+  void* dx;                // [M, K] bf16 or null
+  uint8_t* ws;             // workspace base
+  size_t ws_bytes;
+  uint32_t* status;
+};
+
+size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, int r);
+cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
+cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
+
+}  // namespace nf4

@@ -1,0 +1,288 @@
+// NF4 quantize / double-quant / dequantize kernels (memory-bound).
+//
+// Quantize follows the qlora-rs README ("Honest capability matrix": NF4
+// pack/unpack + block absmax scales; "Double quantization (simplified)") and
+// the level construction of "LoRA and QLoRA, mathematically" ("NF4: quantizing
+// the frozen base").  Each thread owns 8 consecutive elements (32 bytes in,
+// one u32 of packed codes out); the absmax of a block of bs elements is a
+// shuffle-xor reduction over the bs/8 lanes that hold it.
+#include "nf4_common.cuh"
+#include "kernels.h"
+
+namespace nf4 {
+
+namespace {
+
+__device__ __forceinline__ float max_abs8(const float4& a, const float4& b) {
+  float m = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
+  return fmaxf(m, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
+}
+
+__device__ __forceinline__ bool finite8(const float4& a, const float4& b) {
+  return isfinite(a.x) && isfinite(a.y) && isfinite(a.z) && isfinite(a.w) && isfinite(b.x) &&
+         isfinite(b.y) && isfinite(b.z) && isfinite(b.w);
+}
+
+// Codes of two elements packed as one byte, even element in the high nibble.
+__device__ __forceinline__ uint32_t pair_byte(float w0, float w1, float amax) {
+  if (amax == 0.0f) return 0x77u;
+  const uint32_t c0 = encode(__fdiv_rn(w0, amax));
+  const uint32_t c1 = encode(__fdiv_rn(w1, amax));
+  return (c0 << 4) | c1;
+}
+
+// Block-wide max of a non-negative float, then one atomicMax per CTA on its
+// bit pattern (non-negative floats order like their unsigned bits).
+__device__ __forceinline__ void cta_global_max(float v, uint32_t* gmax) {
+  __shared__ float red[32];
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < int(blockDim.x >> 5) ? red[lane] : 0.0f;
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0 && v > 0.0f) atomicMax(gmax, __float_as_uint(v));
+  }
+}
+
+// G = block_size / 8 lanes per block (1, 2, 4, 8, 16 or 32).
+template <int G>
+__global__ void __launch_bounds__(256) quantize_vec_kernel(
+    const float4* __restrict__ w, int64_t n_words, int64_t blocks_per_row_unused,
+    uint32_t* __restrict__ codes, float* __restrict__ absmax, uint32_t* __restrict__ status,
+    uint32_t* __restrict__ gmax) {
+  (void)blocks_per_row_unused;
+  float cta_max = 0.0f;
+  bool bad = false;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  // Iterate in whole warps so every lane takes part in the shuffles.
+  for (int64_t base = int64_t(blockIdx.x) * blockDim.x; base < n_words; base += stride) {
+    const int64_t i = base + threadIdx.x;
+    const bool valid = i < n_words;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (valid) {
+      a = __ldcs(w + 2 * i);
+      b = __ldcs(w + 2 * i + 1);
+      bad |= !finite8(a, b);
+    }
+    float m = max_abs8(a, b);
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (valid) {
+      uint32_t word = pair_byte(a.x, a.y, m) | (pair_byte(a.z, a.w, m) << 8) |
+                      (pair_byte(b.x, b.y, m) << 16) | (pair_byte(b.z, b.w, m) << 24);
+      __stcs(codes + i, word);
+      if ((threadIdx.x & (G - 1)) == 0 && absmax != nullptr) absmax[i / G] = m;
+    }
+    cta_max = fmaxf(cta_max, m);
+  }
+  if (bad) report(status, NF4_ERR_NONFINITE);
+  if (gmax != nullptr) cta_global_max(cta_max, gmax);
+}
+
+// Any even block size: one thread per block, two passes over its elements.
+__global__ void __launch_bounds__(256) quantize_generic_kernel(
+    const float* __restrict__ w, int64_t n_blocks, int bs, uint8_t* __restrict__ codes,
+    float* __restrict__ absmax, uint32_t* __restrict__ status, uint32_t* __restrict__ gmax) {
+  float cta_max = 0.0f;
+  bool bad = false;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t base = int64_t(blockIdx.x) * blockDim.x; base < n_blocks; base += stride) {
+    const int64_t blk = base + threadIdx.x;
+    float m = 0.0f;
+    if (blk < n_blocks) {
+      const float* p = w + blk * bs;
+      for (int e = 0; e < bs; ++e) {
+        const float v = p[e];
+        bad |= !isfinite(v);
+        m = fmaxf(m, fabsf(v));
+      }
+      uint8_t* c = codes + blk * (bs / 2);
+      for (int e = 0; e < bs; e += 2) c[e / 2] = uint8_t(pair_byte(p[e], p[e + 1], m));
+      if (absmax != nullptr) absmax[blk] = m;
+    }
+    cta_max = fmaxf(cta_max, m);
+  }
+  if (bad) report(status, NF4_ERR_NONFINITE);
+  if (gmax != nullptr) cta_global_max(cta_max, gmax);
+}
+
+// Simplified double quant of the block scales: one global scale G / 255 and a
+// u8 per block, rint(absmax / s_g) with ties to even.
+__global__ void __launch_bounds__(256) double_quant_kernel(
+    const float* __restrict__ absmax, int64_t n_blocks, const uint32_t* __restrict__ gmax,
+    uint8_t* __restrict__ absmax_q, float* __restrict__ absmax_scale) {
+  const float g = __uint_as_float(*gmax);
+  const float s_g = __fdiv_rn(g, 255.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *absmax_scale = s_g;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n_blocks; i += stride) {
+    uint32_t q = 0;
+    if (g > 0.0f) {
+      const float ratio = __fdiv_rn(absmax[i], s_g);
+      q = uint32_t(min(max(__float2int_rn(ratio), 0), 255));
+    }
+    absmax_q[i] = uint8_t(q);
+  }
+}
+
+// ------------------------------------------------------------------ dequant
+
+template <typename OutT>
+struct Store8;
+
+template <>
+struct Store8<float> {
+  __device__ __forceinline__ static void run(float* out, int64_t word, const float (&v)[8]) {
+    float4* o = reinterpret_cast<float4*>(out) + 2 * word;
+    __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
+    __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+  }
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <>
+struct Store8<__nv_bfloat16> {
+  __device__ __forceinline__ static void run(__nv_bfloat16* out, int64_t word, const float (&v)[8]) {
+    uint4 u = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                         pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    __stcs(reinterpret_cast<uint4*>(out) + word, u);
+  }
+};
+
+template <>
+struct Store8<__half> {
+  __device__ __forceinline__ static void run(__half* out, int64_t word, const float (&v)[8]) {
+    uint4 u = make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
+                         pack_f16x2(v[6], v[7]));
+    __stcs(reinterpret_cast<uint4*>(out) + word, u);
+  }
+};
+
+// out[e] = fp32(L[code] * scale), one product per element; block_size % 8 == 0
+// so the 8 elements of one code word share a scale.
+template <typename OutT, bool kDouble>
+__global__ void __launch_bounds__(256) dequant_kernel(
+    const uint32_t* __restrict__ codes, int64_t n_words, int bs_words_shift, int bs_words,
+    const float* __restrict__ absmax, const uint8_t* __restrict__ absmax_q,
+    const float* __restrict__ absmax_scale, OutT* __restrict__ out) {
+  __shared__ float lut[16];
+  if (threadIdx.x < 16) lut[threadIdx.x] = level(threadIdx.x);
+  __syncthreads();
+  const float s_g = kDouble ? *absmax_scale : 0.0f;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n_words; i += stride) {
+    const uint32_t word = __ldcs(codes + i);
+    const int64_t blk = bs_words_shift >= 0 ? (i >> bs_words_shift) : (i / bs_words);
+    float scale;
+    if (kDouble) {
+      scale = __fmul_rn(float(__ldg(absmax_q + blk)), s_g);
+    } else {
+      scale = __ldg(absmax + blk);
+    }
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t byte = (word >> (8 * j)) & 0xffu;
+      v[2 * j] = __fmul_rn(lut[byte >> 4], scale);
+      v[2 * j + 1] = __fmul_rn(lut[byte & 15u], scale);
+    }
+    Store8<OutT>::run(out, i, v);
+  }
+}
+
+int grid_for(int64_t work_items, int threads, int sms, int per_sm) {
+  int64_t g = (work_items + threads - 1) / threads;
+  const int64_t cap = int64_t(sms) * per_sm;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return int(g);
+}
+
+int log2_exact(int v) {
+  if (v <= 0 || (v & (v - 1))) return -1;
+  int s = 0;
+  while ((1 << s) < v) ++s;
+  return s;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const float* w, int64_t numel, int bs, uint8_t* codes,
+                            float* absmax_out, uint32_t* status, uint32_t* gmax, int sms,
+                            cudaStream_t stream, int* launches) {
+  const int threads = 256;
+  const bool vec = (bs % 8 == 0) && bs <= 256 && log2_exact(bs) >= 0;
+  if (vec) {
+    const int64_t n_words = numel / 8;
+    const int grid = grid_for(n_words, threads, sms, 8);
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+    uint32_t* c32 = reinterpret_cast<uint32_t*>(codes);
+    switch (bs / 8) {
+      case 1: quantize_vec_kernel<1><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 2: quantize_vec_kernel<2><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 4: quantize_vec_kernel<4><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 8: quantize_vec_kernel<8><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 16: quantize_vec_kernel<16><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
+      default: quantize_vec_kernel<32><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
+    }
+  } else {
+    const int64_t n_blocks = numel / bs;
+    const int grid = grid_for(n_blocks, threads, sms, 8);
+    quantize_generic_kernel<<<grid, threads, 0, stream>>>(w, n_blocks, bs, codes, absmax_out,
+                                                          status, gmax);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uint32_t* gmax,
+                                uint8_t* absmax_q, float* absmax_scale, int sms,
+                                cudaStream_t stream, int* launches) {
+  const int threads = 256;
+  const int grid = grid_for(n_blocks, threads, sms, 4);
+  double_quant_kernel<<<grid, threads, 0, stream>>>(absmax, n_blocks, gmax, absmax_q,
+                                                    absmax_scale);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int sms,
+                              cudaStream_t stream, int* launches) {
+  const int64_t numel = w.rows * w.cols;
+  const int64_t n_words = numel / 8;
+  const int bs_words = w.block_size / 8;
+  const int shift = log2_exact(bs_words);
+  const int threads = 256;
+  const int grid = grid_for(n_words, threads, sms, 8);
+  const uint32_t* c = reinterpret_cast<const uint32_t*>(w.codes);
+  const bool dq = w.double_quant != 0;
+#define NF4_DQ_LAUNCH(T, D)                                                                 \
+  dequant_kernel<T, D><<<grid, threads, 0, stream>>>(c, n_words, shift, bs_words, w.absmax, \
+                                                     w.absmax_q, w.absmax_scale,            \
+                                                     reinterpret_cast<T*>(out))
+  if (out_dtype == NF4_F32) {
+    if (dq) NF4_DQ_LAUNCH(float, true); else NF4_DQ_LAUNCH(float, false);
+  } else if (out_dtype == NF4_BF16) {
+    if (dq) NF4_DQ_LAUNCH(__nv_bfloat16, true); else NF4_DQ_LAUNCH(__nv_bfloat16, false);
+  } else {
+    if (dq) NF4_DQ_LAUNCH(__half, true); else NF4_DQ_LAUNCH(__half, false);
+  }
+#undef NF4_DQ_LAUNCH
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+}  // namespace nf4

@@ -1,0 +1,256 @@
+"""Thin ctypes binding of libnf4qlora.so (declared in include/nf4qlora.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch provides device memory (and the workspace) and the current
+stream.  There is no fallback: if the library is missing or the GPU call
+fails, these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnf4qlora.so")
+
+NF4_OK = 0
+STATUS_NAMES = {
+    0: "NF4_OK", 1: "NF4_ERR_INVALID_ARG", 2: "NF4_ERR_SHAPE", 3: "NF4_ERR_ALIGNMENT",
+    4: "NF4_ERR_UNSUPPORTED", 5: "NF4_ERR_WORKSPACE", 6: "NF4_ERR_CUDA",
+    7: "NF4_ERR_NONFINITE", 8: "NF4_ERR_TIMEOUT",
+}
+NF4_F32, NF4_BF16, NF4_F16 = 0, 1, 2
+OP_QUANTIZE, OP_DEQUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD = 0, 1, 2, 3
+
+EXPORTED = (
+    "nf4_status_string", "nf4_version", "nf4_codebook", "nf4_launch_count",
+    "nf4_workspace_bytes", "nf4_read_status", "nf4_quantize", "nf4_dequantize",
+    "qlora_linear_fwd", "qlora_linear_bwd",
+)
+
+
+class NF4Error(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        name = STATUS_NAMES.get(self.status, str(status))
+        super().__init__(f"{what}: {name}" if what else name)
+
+
+class CWeight(ctypes.Structure):
+    """Mirror of `nf4_weight`."""
+    _fields_ = [
+        ("codes", ctypes.c_void_p),
+        ("absmax", ctypes.c_void_p),
+        ("absmax_q", ctypes.c_void_p),
+        ("absmax_scale", ctypes.c_void_p),
+        ("rows", ctypes.c_int64),
+        ("cols", ctypes.c_int64),
+        ("block_size", ctypes.c_int32),
+        ("double_quant", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library once; raise if it was not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m qlora_linear_layers_nf4_b200.build` "
+            "(there is no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.nf4_status_string.argtypes = [i32]
+    L.nf4_status_string.restype = ctypes.c_char_p
+    L.nf4_version.restype = i32
+    L.nf4_codebook.argtypes = [vp, vp]
+    L.nf4_codebook.restype = None
+    L.nf4_launch_count.restype = i64
+    L.nf4_workspace_bytes.argtypes = [i32, i64, i64, i64, i32, i32, i32]
+    L.nf4_workspace_bytes.restype = sz
+    L.nf4_read_status.argtypes = [vp, vp]
+    L.nf4_read_status.restype = i32
+    L.nf4_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]
+    L.nf4_quantize.restype = i32
+    L.nf4_dequantize.argtypes = [ctypes.POINTER(CWeight), i32, vp, vp]
+    L.nf4_dequantize.restype = i32
+    L.qlora_linear_fwd.argtypes = [ctypes.POINTER(CWeight), vp, i64, vp, vp, i32, f32, i32, vp, vp,
+                                   vp, vp, sz, vp]
+    L.qlora_linear_fwd.restype = i32
+    L.qlora_linear_bwd.argtypes = [ctypes.POINTER(CWeight), vp, i64, vp, vp, i32, f32, i32, vp, vp,
+                                   vp, vp, vp, vp, sz, vp]
+    L.qlora_linear_bwd.restype = i32
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str):
+    if status != NF4_OK:
+        raise NF4Error(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def codebook():
+    """(levels[16], thresholds[15]) as Python float lists, from the library."""
+    lv = (ctypes.c_float * 16)()
+    th = (ctypes.c_float * 15)()
+    lib().nf4_codebook(ctypes.cast(lv, ctypes.c_void_p), ctypes.cast(th, ctypes.c_void_p))
+    return list(lv), list(th)
+
+
+def launch_count() -> int:
+    return int(lib().nf4_launch_count())
+
+
+def workspace_bytes(op: int, M: int, N: int, K: int, r: int, block_size: int, double_quant: bool) -> int:
+    return int(lib().nf4_workspace_bytes(op, M, N, K, r, block_size, int(double_quant)))
+
+
+class Workspace:
+    """A zero-filled device byte buffer reused across calls (grown on demand)."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int):
+        import torch
+        nbytes = max(int(nbytes), 256)
+        if self.buf is None or self.buf.numel() < nbytes:
+            dev = self.device if self.device is not None else torch.device("cuda", torch.cuda.current_device())
+            self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        return self.buf
+
+    def read_status(self, stream=None) -> int:
+        if self.buf is None:
+            return NF4_OK
+        return int(lib().nf4_read_status(_ptr(self.buf), _stream(stream)))
+
+
+_default_ws = {}
+
+
+def default_workspace(device) -> Workspace:
+    key = str(device)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+@dataclass
+class QuantizedWeight:
+    """Device tensors of one NF4 weight (fields as in `nf4_weight`)."""
+    codes: object                    # uint8 [numel/2]
+    absmax: object | None            # fp32 [nblocks]
+    absmax_q: object | None          # uint8 [nblocks]
+    absmax_scale: object | None      # fp32 [1]
+    rows: int
+    cols: int
+    block_size: int
+    double_quant: bool
+
+    def c_struct(self) -> CWeight:
+        return CWeight(
+            codes=self.codes.data_ptr(),
+            absmax=None if (self.absmax is None or self.double_quant) else self.absmax.data_ptr(),
+            absmax_q=None if self.absmax_q is None else self.absmax_q.data_ptr(),
+            absmax_scale=None if self.absmax_scale is None else self.absmax_scale.data_ptr(),
+            rows=self.rows, cols=self.cols, block_size=self.block_size,
+            double_quant=int(self.double_quant))
+
+    @property
+    def device(self):
+        return self.codes.device
+
+
+def quantize(w, block_size: int = 64, double_quant: bool = False, keep_absmax: bool | None = None,
+             workspace: Workspace | None = None, stream=None, check_status: bool = False) -> QuantizedWeight:
+    """NF4-quantize an fp32 CUDA tensor (any shape; flattened row-major)."""
+    import torch
+    if w.dtype != torch.float32 or not w.is_cuda:
+        raise TypeError("quantize expects a float32 CUDA tensor")
+    w = w.contiguous()
+    rows = int(w.shape[0]) if w.dim() >= 1 else 1
+    cols = 1
+    for d in w.shape[1:]:
+        cols *= int(d)
+    numel = w.numel()
+    dev = w.device
+    nblocks = numel // block_size if block_size > 0 else 0
+    keep_absmax = (not double_quant) if keep_absmax is None else keep_absmax
+    codes = torch.empty(max(numel // 2, 1), dtype=torch.uint8, device=dev)
+    absmax = torch.empty(max(nblocks, 1), dtype=torch.float32, device=dev) if keep_absmax else None
+    absmax_q = torch.empty(max(nblocks, 1), dtype=torch.uint8, device=dev) if double_quant else None
+    absmax_scale = torch.empty(1, dtype=torch.float32, device=dev) if double_quant else None
+    ws = workspace or default_workspace(dev)
+    buf = ws.get(workspace_bytes(OP_QUANTIZE, 0, rows, cols, 0, block_size, double_quant))
+    st = lib().nf4_quantize(_ptr(w), rows, cols, block_size, int(double_quant), _ptr(codes),
+                            _ptr(absmax), _ptr(absmax_q), _ptr(absmax_scale), _ptr(buf),
+                            buf.numel(), _stream(stream))
+    _check(st, "nf4_quantize")
+    if check_status:
+        _check(ws.read_status(stream), "nf4_quantize (device)")
+    return QuantizedWeight(codes, absmax, absmax_q, absmax_scale, rows, cols, block_size, double_quant)
+
+
+def dequantize(q: QuantizedWeight, out_dtype: str = "f32", stream=None):
+    import torch
+    dt = {"f32": (NF4_F32, torch.float32), "bf16": (NF4_BF16, torch.bfloat16),
+          "f16": (NF4_F16, torch.float16)}[out_dtype]
+    out = torch.empty((q.rows, q.cols), dtype=dt[1], device=q.device)
+    cw = q.c_struct()
+    _check(lib().nf4_dequantize(ctypes.byref(cw), dt[0], _ptr(out), _stream(stream)), "nf4_dequantize")
+    return out
+
+
+def linear_fwd(q: QuantizedWeight, x, A, B, alpha: float, bias=None, want_t: bool = True,
+               out=None, t_out=None, workspace: Workspace | None = None, stream=None):
+    """y = x W'^T + (alpha/r) (x A^T) B^T (+ bias); returns (y, T or None)."""
+    import torch
+    M = x.shape[0]
+    r = A.shape[0]
+    y = out if out is not None else torch.empty((M, q.rows), dtype=torch.bfloat16, device=x.device)
+    if want_t and t_out is None:
+        t_out = torch.empty((M, r), dtype=torch.bfloat16, device=x.device)
+    ws = workspace or default_workspace(x.device)
+    buf = ws.get(workspace_bytes(OP_LINEAR_FWD, M, q.rows, q.cols, r, q.block_size, q.double_quant))
+    cw = q.c_struct()
+    st = lib().qlora_linear_fwd(ctypes.byref(cw), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
+                                NF4_BF16, _ptr(bias), _ptr(y), _ptr(t_out), _ptr(buf), buf.numel(),
+                                _stream(stream))
+    _check(st, "qlora_linear_fwd")
+    return y, t_out
+
+
+def linear_bwd(q: QuantizedWeight, x, A, B, alpha: float, dy, t=None, want_dx: bool = True,
+               dA=None, dB=None, dx=None, workspace: Workspace | None = None, stream=None):
+    """Adapter backward; returns (dA fp32 [r,K], dB fp32 [N,r], dx bf16 [M,K] or None)."""
+    import torch
+    M = x.shape[0]
+    r = A.shape[0]
+    dA = dA if dA is not None else torch.empty((r, q.cols), dtype=torch.float32, device=x.device)
+    dB = dB if dB is not None else torch.empty((q.rows, r), dtype=torch.float32, device=x.device)
+    if want_dx and dx is None:
+        dx = torch.empty((M, q.cols), dtype=torch.bfloat16, device=x.device)
+    ws = workspace or default_workspace(x.device)
+    buf = ws.get(workspace_bytes(OP_LINEAR_BWD, M, q.rows, q.cols, r, q.block_size, q.double_quant))
+    cw = q.c_struct()
+    st = lib().qlora_linear_bwd(ctypes.byref(cw), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
+                                NF4_BF16, _ptr(dy), _ptr(t), _ptr(dA), _ptr(dB), _ptr(dx),
+                                _ptr(buf), buf.numel(), _stream(stream))
+    _check(st, "qlora_linear_bwd")
+    return dA, dB, dx

@@ -1,0 +1,127 @@
+"""CPU checks of the C-ABI library: it loads, exports what the header
+declares, reports the oracle's codebook, and refuses bad arguments on the host
+before touching the GPU.  No compute call is made here."""
+import ctypes
+import os
+import re
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import nf4_oracle as O
+from qlora_linear_layers_nf4_b200 import nf4qlora as Q
+from tests.conftest import ROOT
+
+FAKE = 0x10000   # aligned, never dereferenced: every call below fails validation first
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "nf4qlora.h")).read()
+    return re.findall(r"NF4_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_library_exports_every_declared_symbol():
+    L = Q.lib()
+    names = _declared()
+    assert set(names) == set(Q.EXPORTED)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_codebook_matches_oracle_bit_for_bit():
+    lv, th = Q.codebook()
+    lv = np.array(lv, dtype=np.float32)
+    assert np.array_equal(lv.view(np.uint32), O.nf4_levels().view(np.uint32))
+    th = np.array(th, dtype=np.float32)
+    for i in range(15):
+        m = (Fraction(float(lv[i])) + Fraction(float(lv[i + 1]))) / 2
+        nxt = np.nextafter(th[i], np.float32(2), dtype=np.float32)
+        assert Fraction(float(th[i])) <= m < Fraction(float(nxt))
+
+
+def test_threshold_count_rule_equals_oracle_nearest():
+    # The library's encoding rule (count of thresholds below v) against the
+    # oracle's brute-force nearest level, on midpoint neighbourhoods and randoms.
+    _, th = Q.codebook()
+    th = np.array(th, dtype=np.float32)
+    rng = np.random.default_rng(1)
+    v = np.concatenate([rng.uniform(-1, 1, 200000).astype(np.float32), th,
+                        np.nextafter(th, np.float32(2)), np.nextafter(th, np.float32(-2)),
+                        np.array([0.0, -0.0, 1.0, -1.0], np.float32)])
+    count = (v[:, None] > th[None, :]).sum(axis=1)
+    assert np.array_equal(count.astype(np.uint8), O.nearest_code(v))
+
+
+def test_status_strings_and_version():
+    L = Q.lib()
+    for code, name in Q.STATUS_NAMES.items():
+        assert L.nf4_status_string(code).decode().startswith(name)
+    assert L.nf4_version() >= 100
+    assert Q.launch_count() >= 0
+
+
+def test_workspace_sizes():
+    assert Q.workspace_bytes(Q.OP_DEQUANTIZE, 0, 4096, 4096, 0, 64, False) == 0
+    assert Q.workspace_bytes(Q.OP_QUANTIZE, 0, 4096, 4096, 0, 64, False) >= 256
+    assert Q.workspace_bytes(Q.OP_QUANTIZE, 0, 4096, 4096, 0, 64, True) >= 256 + 4096 * 64 * 4
+    assert Q.workspace_bytes(Q.OP_LINEAR_FWD, 4096, 11008, 4096, 64, 64, True) >= 256
+    assert Q.workspace_bytes(Q.OP_LINEAR_BWD, 4096, 11008, 4096, 64, 64, True) >= 256
+
+
+def _quant(rows, cols, bs, dq, w=FAKE, codes=FAKE, absmax=FAKE, aq=FAKE, asc=FAKE, ws=FAKE, wsb=1 << 30):
+    return Q.lib().nf4_quantize(w, rows, cols, bs, dq, codes, absmax, aq, asc, ws, wsb, None)
+
+
+def test_quantize_host_validation():
+    assert _quant(4, 64, 63, 0) == 2          # odd block size
+    assert _quant(4, 64, 0, 0) == 2
+    assert _quant(3, 10, 64, 0) == 2          # numel not a multiple of the block
+    assert _quant(4, 64, 64, 2) == 1          # double_quant must be 0/1
+    assert _quant(4, 64, 64, 0, w=None) == 1
+    assert _quant(4, 64, 64, 0, absmax=None) == 1
+    assert _quant(4, 64, 64, 1, aq=None) == 1
+    assert _quant(4, 64, 64, 0, w=FAKE + 4) == 3
+    assert _quant(4, 64, 64, 0, codes=FAKE + 8) == 3
+    assert _quant(4, 64, 64, 0, ws=None) == 5
+    assert _quant(4, 64, 64, 1, wsb=16) == 5
+    assert _quant(-1, 64, 64, 0) == 2
+
+
+def _cw(rows=4096, cols=4096, bs=64, dq=1, codes=FAKE):
+    return Q.CWeight(codes=codes, absmax=FAKE, absmax_q=FAKE, absmax_scale=FAKE, rows=rows,
+                     cols=cols, block_size=bs, double_quant=dq)
+
+
+def test_dequantize_host_validation():
+    L = Q.lib()
+    assert L.nf4_dequantize(ctypes.byref(_cw(bs=6)), 0, FAKE, None) == 2
+    assert L.nf4_dequantize(ctypes.byref(_cw(rows=3, cols=8, bs=16)), 0, FAKE, None) == 2
+    assert L.nf4_dequantize(ctypes.byref(_cw()), 7, FAKE, None) == 1
+    assert L.nf4_dequantize(ctypes.byref(_cw(codes=None)), 0, FAKE, None) == 1
+    assert L.nf4_dequantize(ctypes.byref(_cw()), 0, FAKE + 2, None) == 3
+
+
+def _fwd(cw, M=16, r=16, dtype=1, alpha=32.0, x=FAKE, y=FAKE, wsb=1 << 40):
+    return Q.lib().qlora_linear_fwd(ctypes.byref(cw), x, M, FAKE, FAKE, r, alpha, dtype, None, y,
+                                    None, FAKE, wsb, None)
+
+
+def test_linear_host_validation():
+    assert _fwd(_cw(), r=4) == 1                  # r < 8
+    assert _fwd(_cw(), r=12) == 1                 # r % 8
+    assert _fwd(_cw(), r=512) == 1
+    assert _fwd(_cw(), dtype=2) == 4              # F16 compute: not in this build
+    assert _fwd(_cw(), dtype=0) == 4              # F32 compute: not in this build
+    assert _fwd(_cw(), dtype=9) == 1
+    assert _fwd(_cw(), M=0) == 2
+    assert _fwd(_cw(cols=4000)) == 2              # K % 64
+    assert _fwd(_cw(rows=4092)) == 2              # N % 8
+    assert _fwd(_cw(bs=128)) == 4                 # GEMMs take block 64
+    assert _fwd(_cw(), x=FAKE + 2) == 3
+    assert _fwd(_cw(), y=None) == 1
+    assert _fwd(_cw(), wsb=0) == 5
+    L = Q.lib()
+    st = L.qlora_linear_bwd(ctypes.byref(_cw()), FAKE, 16, FAKE, FAKE, 16, 32.0, 1, None, None,
+                            FAKE, FAKE, None, FAKE, 1 << 40, None)
+    assert st == 1                                # dy required

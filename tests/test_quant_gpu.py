@@ -1,0 +1,146 @@
+"""GPU parity: NF4 quantize / double quant / dequantize, bit for bit against the
+CPU oracle on the same seeded inputs, through the C ABI."""
+import numpy as np
+import pytest
+
+from oracle import nf4_oracle as O
+from qlora_linear_layers_nf4_b200 import workloads as WL
+
+pytestmark = pytest.mark.gpu
+
+
+def _q():
+    from qlora_linear_layers_nf4_b200 import nf4qlora as Q
+    return Q
+
+
+def _to_dev(a, dev):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def _check_quant(w, bs, dq, dev):
+    Q = _q()
+    import torch
+    ref = O.quantize(w, bs, double=dq)
+    q = Q.quantize(_to_dev(w, dev), block_size=bs, double_quant=dq, keep_absmax=True,
+                   check_status=True)
+    torch.cuda.synchronize()
+    codes = q.codes.cpu().numpy()[: ref["codes"].size]
+    assert np.array_equal(codes, ref["codes"]), "packed codes differ"
+    assert np.array_equal(q.absmax.cpu().numpy()[: ref["absmax"].size].view(np.uint32),
+                          ref["absmax"].view(np.uint32))
+    if dq:
+        assert np.array_equal(q.absmax_q.cpu().numpy()[: ref["absmax_q"].size], ref["absmax_q"])
+        assert q.absmax_scale.cpu().numpy()[0].view(np.uint32) == np.float32(ref["absmax_scale"]).view(np.uint32)
+    return q, ref
+
+
+def _check_dequant(q, ref, dev):
+    Q = _q()
+    for kind in ("f32", "bf16", "f16"):
+        got = Q.dequantize(q, kind).cpu()
+        want = O.dequantize(ref, kind)
+        if kind == "f32":
+            assert np.array_equal(got.numpy().view(np.uint32), want.reshape(got.shape).view(np.uint32))
+        elif kind == "bf16":
+            import torch
+            g = got.view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(g, want.reshape(g.shape))
+        else:
+            assert np.array_equal(got.numpy().view(np.uint16), want.reshape(got.shape).view(np.uint16))
+
+
+def test_tiny_layer_weight(cuda_device):
+    inp = WL.draw_linear(WL.TINY)
+    q, ref = _check_quant(inp.w, 64, False, cuda_device)
+    _check_dequant(q, ref, cuda_device)
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_full_4096_square(cuda_device, dq):
+    w = WL.draw_weight(WL.QUANT_SHAPE, WL.QUANT_SEED)
+    q, ref = _check_quant(w, 64, dq, cuda_device)
+    _check_dequant(q, ref, cuda_device)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32, 128, 256, 2, 6, 24, 40, 512])
+def test_block_sizes_and_ragged_grid(cuda_device, bs):
+    # 7 rows x (bs * 37) columns: the element count is not a multiple of the
+    # launch width, and non-power-of-two sizes take the per-block path.
+    w = WL.draw_weight((7, bs * 37), seed=100 + bs)
+    q, ref = _check_quant(w, bs, True, cuda_device)
+    if bs % 8 == 0:
+        _check_dequant(q, ref, cuda_device)
+
+
+def test_edge_values(cuda_device):
+    lv = O.nf4_levels()
+    rng = np.random.default_rng(7)
+    blocks = []
+    # exact midpoints and neighbours, scaled by powers of two (absmax = 2^e)
+    from fractions import Fraction
+    mids = []
+    for i in range(15):
+        m = np.float32(float((Fraction(float(lv[i])) + Fraction(float(lv[i + 1]))) / 2))
+        mids += [m, np.nextafter(m, np.float32(2)), np.nextafter(m, np.float32(-2))]
+    mids = np.array(mids, dtype=np.float32)
+    for e in (-10, -3, 0, 5):
+        blk = np.resize(mids, 63).astype(np.float32) * np.float32(2.0 ** e)
+        blocks.append(np.concatenate([blk, [np.float32(2.0 ** e)]]))
+    blocks.append(np.zeros(64, np.float32))                          # absmax 0
+    z = np.zeros(64, np.float32)
+    z[5] = -0.0
+    z[9] = np.float32(-3e-3)
+    blocks.append(z)                                                 # negative absmax element
+    blocks.append(np.full(64, np.float32(1e-38)))                    # tiny values
+    d = np.zeros(64, np.float32)
+    d[0] = np.float32(1e-42)                                         # denormal absmax
+    d[1] = np.float32(-7e-43)
+    blocks.append(d)
+    blocks.append(rng.permutation(np.resize(lv, 64)).astype(np.float32) * np.float32(3.0))
+    w = np.stack(blocks)
+    for dq in (False, True):
+        q, ref = _check_quant(w, 64, dq, cuda_device)
+        _check_dequant(q, ref, cuda_device)
+
+
+def test_absmax_element_exact(cuda_device):
+    # values a for which multiplying by a reciprocal would not give exactly 1
+    rng = np.random.default_rng(5)
+    a = (rng.random(200000, dtype=np.float32) * np.float32(0.1) + np.float32(1e-3)).astype(np.float32)
+    bad = a[(a * (np.float32(1.0) / a)).astype(np.float32) != np.float32(1.0)][:256]
+    blocks = rng.standard_normal((bad.size, 64)).astype(np.float32) * np.float32(1e-4)
+    blocks[:, 17] = bad
+    blocks[::2, 17] *= -1
+    q, ref = _check_quant(blocks, 64, False, cuda_device)
+    _check_dequant(q, ref, cuda_device)
+
+
+def test_all_zero_and_single_block(cuda_device):
+    for shape in [(32, 32), (1, 64), (2, 2)]:
+        w = np.zeros(shape, np.float32)
+        bs = 64 if w.size % 64 == 0 else 4
+        q, ref = _check_quant(w, bs, True, cuda_device)
+
+
+def test_nonfinite_is_flagged(cuda_device):
+    Q = _q()
+    import torch
+    w = WL.draw_weight((16, 64), seed=3)
+    w[3, 5] = np.nan
+    ws = Q.Workspace(cuda_device)
+    Q.quantize(_to_dev(w, cuda_device), 64, False, workspace=ws)
+    assert ws.read_status() == 7
+    assert ws.read_status() == 0            # read clears it
+    w[3, 5] = np.inf
+    Q.quantize(_to_dev(w, cuda_device), 64, True, workspace=ws)
+    assert ws.read_status() == 7
+
+
+def test_empty_input(cuda_device):
+    Q = _q()
+    import torch
+    q = Q.quantize(torch.zeros((0, 64), dtype=torch.float32, device=cuda_device), 64, True)
+    torch.cuda.synchronize()
+    assert q.absmax_scale.item() == 0.0
