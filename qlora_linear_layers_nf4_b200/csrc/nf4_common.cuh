@@ -22,6 +22,12 @@ namespace nf4 {
 constexpr uint32_t kLevelBits[16] = NF4_LEVEL_BITS;        // host copy
 static __constant__ uint32_t kLevelBitsDev[16] = NF4_LEVEL_BITS;
 
+// Level i as a compile-time constant (i must be a literal after inlining).
+__host__ __device__ constexpr uint32_t level_bits(int i) {
+  constexpr uint32_t t[16] = NF4_LEVEL_BITS;
+  return t[i];
+}
+
 // Decision thresholds: kThresholdBits[i] is the largest fp32 value not above
 // the exact midpoint of levels i and i+1.  For an fp32 value v, v > t_i holds
 // exactly when v is strictly nearer to level i+1 than to level i, so

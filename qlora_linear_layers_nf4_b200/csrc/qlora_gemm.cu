@@ -1,17 +1,822 @@
-// QLoRA linear forward / backward launchers (tensor-core path in progress).
-#include "nf4_common.cuh"
+// QLoRA linear forward and adapter backward on the sm_100a tensor cores.
+//
+// The layer (qlora-rs README, QuantizedLinear::forward; "LoRA and QLoRA,
+// mathematically", equation 6.3.6 read as a layer) is
+//     y  = x W'^T + T B^T,          T = s x A^T,  s = alpha / r
+// and its backward for L = sum(dy * y) with W frozen is
+//     U  = s dy B,  dB = dy^T T,  dA = U^T x,  dx = dy W' + U A.
+// W' = bf16(L[code] * scale) is never written to HBM: the fused kernel
+// dequantizes each NF4 tile into shared memory, in the 128-byte-swizzled
+// layout the tensor core reads, right before the MMA that consumes it.  The
+// adapter product rides in the same TMEM accumulator as extra K steps
+// ([x | T] [W' | B]^T forward, [dy | U] [W' ; A] backward).
+//
+// Kernels
+//   fused_nf4_gemm<kFwd>  y[M,N]  = x W'^T + T B^T (+ bias)   K-major W' tiles
+//   fused_nf4_gemm<kDx>   dx[M,K] = dy W' + U A                 MN-major W' tiles
+//   adapter_gemm          the rank-r products T, U, dB, dA^T, split along the
+//                         reduction with fp32 partials
+//   adapter_finalize      sums the partials, scales/rounds/transposes
+#include <algorithm>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
 #include "kernels.h"
+#include "nf4_common.cuh"
+#include "tc_common.cuh"
 
 namespace nf4 {
+namespace {
 
-size_t linear_workspace_bytes(bool, int64_t, int64_t, int64_t, int) { return 0; }
+using namespace tc;
 
-cudaError_t launch_linear_fwd(const LinearArgs&, int, cudaStream_t, int*) {
-  return cudaErrorNotSupported;
+// ------------------------------------------------------------------ dequant
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
 }
 
-cudaError_t launch_linear_bwd(const LinearArgs&, int, cudaStream_t, int*) {
-  return cudaErrorNotSupported;
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// The sixteen dequantized values of one block, bf16(L[c] * scale) with the
+// fp32 product rounded to nearest even, split into byte planes so a lookup is
+// a register byte-permute: lo[q] holds the low bytes of entries 4q..4q+3,
+// hi[q] their high bytes.
+struct BlockTable {
+  uint32_t lo[4];
+  uint32_t hi[4];
+};
+
+__device__ __forceinline__ BlockTable make_table(float scale) {
+  uint32_t p[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    p[j] = bf16x2_rn(__fmul_rn(__uint_as_float(level_bits(2 * j)), scale),
+                     __fmul_rn(__uint_as_float(level_bits(2 * j + 1)), scale));
+  }
+  BlockTable t;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    t.lo[q] = prmt(p[2 * q], p[2 * q + 1], 0x6420u);
+    t.hi[q] = prmt(p[2 * q], p[2 * q + 1], 0x7531u);
+  }
+  return t;
+}
+
+// Four codes (the low 16 bits of `w`: two packed bytes, even element in the
+// high nibble) -> four bf16 values as two bf16x2 words in element order.
+__device__ __forceinline__ uint2 decode4(uint32_t w, const BlockTable& t) {
+  const uint32_t sel = w & 0x7777u;                          // code & 7 per nibble
+  const uint32_t pick = ((w >> 1) & 0x4444u) | 0x3210u;      // code >= 8 -> upper plane
+  const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], sel), prmt(t.lo[2], t.lo[3], sel), pick);
+  const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], sel), prmt(t.hi[2], t.hi[3], sel), pick);
+  // lo/hi bytes are in nibble order (odd element first within a byte).
+  return make_uint2(prmt(lo, hi, 0x4051u), prmt(lo, hi, 0x6273u));
+}
+
+// Dequantize one 64-element block (32 code bytes at `codes`, smem) into row
+// `row` of a 128-byte-swizzled bf16 tile at `tile` (smem).
+__device__ __forceinline__ void dequant_row(const uint8_t* codes, float scale, uint8_t* tile,
+                                            uint32_t row) {
+  const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
+  const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
+  const BlockTable t = make_table(scale);
+  const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint2 a = decode4(words[k], t);
+    const uint2 b = decode4(words[k] >> 16, t);
+    *reinterpret_cast<uint4*>(tile + sw128_offset(row, k)) = make_uint4(a.x, a.y, b.x, b.y);
+  }
+}
+
+__device__ __forceinline__ float load_scale(const uint8_t* absmax_q, const float* absmax,
+                                            float s_g, bool dq, int64_t idx) {
+  return dq ? __fmul_rn(float(__ldg(absmax_q + idx)), s_g) : __ldg(absmax + idx);
+}
+
+// ------------------------------------------------------------------ fused GEMM
+
+constexpr int kFwd = 0;
+constexpr int kDx = 1;
+
+constexpr int kTileM = 256;     // two UMMA M=128 halves
+constexpr int kTileN = 256;
+constexpr int kTileK = 64;      // one 128-byte swizzle row of bf16
+constexpr int kStages = 3;
+constexpr int kDeqWarps = 8;
+constexpr int kFusedThreads = 64 + kDeqWarps * 32;  // TMA warp, MMA warp, 8 dequant/epilogue
+constexpr uint32_t kHalfABytes = 128 * 128;         // 128 rows x 128 B
+constexpr uint32_t kABytes = 2 * kHalfABytes;
+constexpr uint32_t kBBytes = kTileN * 128;
+constexpr uint32_t kCBytes = kTileN * 32;           // 256 blocks x 32 code bytes
+constexpr uint32_t kStageBytes = kABytes + kBBytes + kCBytes;
+constexpr size_t kFusedSmem = size_t(kStages) * kStageBytes + 1024 + 256;
+
+struct FusedParams {
+  int M;             // rows of x / dy
+  int N;             // W rows (out features)
+  int K;             // W cols (in features)
+  int r;
+  int main_steps;    // fwd: K / 64; dx: ceil(N / 64)
+  int adapter_steps; // ceil(r / 64)
+  int out_cols;      // N (fwd) or K (dx)
+  int kb_per_row;    // K / 64 NF4 blocks per W row
+  int double_quant;
+  const uint8_t* absmax_q;
+  const float* absmax;
+  const float* absmax_scale;
+  const __nv_bfloat16* bias;
+  __nv_bfloat16* out;
+  uint32_t* status;
+};
+
+struct FusedShared {
+  uint64_t full[kStages];    // TMA bytes landed (A + codes, or A2 + B2)
+  uint64_t bready[kStages];  // dequantized B tile written (8 warp arrivals)
+  uint64_t empty[kStages];   // MMAs reading the stage finished (umma_commit)
+  uint64_t accum;            // all MMAs finished
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a2,
+                   const __grid_constant__ CUtensorMap tm_b2,
+                   const __grid_constant__ CUtensorMap tm_codes, const FusedParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  FusedShared* sh = reinterpret_cast<FusedShared*>(smem + kStages * kStageBytes);
+  auto stage_a = [&](int s) { return smem + s * kStageBytes; };
+  auto stage_b = [&](int s) { return smem + s * kStageBytes + kABytes; };
+  auto stage_c = [&](int s) { return smem + s * kStageBytes + kABytes + kBBytes; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tile_n0 = blockIdx.x * kTileN;   // fwd: W rows; dx: W cols (output cols)
+  const int m0 = blockIdx.y * kTileM;
+  const int total_steps = p.main_steps + p.adapter_steps;
+  volatile uint32_t* abort_flag = &sh->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->bready[s], kDeqWarps);
+      mbar_init(&sh->empty[s], 1);
+    }
+    mbar_init(&sh->accum, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    tma_prefetch(&tm_a);
+    tma_prefetch(&tm_a2);
+    tma_prefetch(&tm_b2);
+    tma_prefetch(&tm_codes);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < total_steps; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (!mbar_wait(&sh->empty[s], ph ^ 1, abort_flag, p.status)) break;
+        uint8_t* a = stage_a(s);
+        if (it < p.main_steps) {
+          mbar_arrive_expect_tx(&sh->full[s], kABytes + kCBytes);
+          const int k0 = it * kTileK;  // fwd: K index; dx: N index (the reduction)
+          tma_load_2d(a, &tm_a, &sh->full[s], k0, m0);
+          tma_load_2d(a + kHalfABytes, &tm_a, &sh->full[s], k0, m0 + 128);
+          if (MODE == kFwd) {
+            tma_load_2d(stage_c(s), &tm_codes, &sh->full[s], k0 / 2, tile_n0);
+          } else {
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              tma_load_2d(stage_c(s) + g * 2048, &tm_codes, &sh->full[s], (tile_n0 + 64 * g) / 2, k0);
+          }
+        } else {
+          const int r0 = (it - p.main_steps) * kTileK;
+          mbar_arrive_expect_tx(&sh->full[s], kABytes + kBBytes);
+          tma_load_2d(a, &tm_a2, &sh->full[s], r0, m0);
+          tma_load_2d(a + kHalfABytes, &tm_a2, &sh->full[s], r0, m0 + 128);
+          if (MODE == kFwd) {
+            tma_load_2d(stage_b(s), &tm_b2, &sh->full[s], r0, tile_n0);
+          } else {
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              tma_load_2d(stage_b(s) + g * 8192, &tm_b2, &sh->full[s], tile_n0 + 64 * g, r0);
+          }
+        }
+        ++issued;
+      }
+      // Unwind after an abort: wait (bounded) for the copies still in flight.
+      if (*abort_flag) {
+        for (int it = issued - 1; it >= 0 && it >= issued - kStages; --it) {
+          uint32_t dummy_abort = 0;
+          mbar_wait(&sh->full[it % kStages], (it / kStages) & 1, &dummy_abort, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, kTileN, false, MODE == kDx);
+      bool ok = true;
+      for (int it = 0; it < total_steps && ok; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        const bool adapter = it >= p.main_steps;
+        ok = mbar_wait(&sh->full[s], ph, abort_flag, p.status);
+        if (ok && !adapter) ok = mbar_wait(&sh->bready[s], ph, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(stage_a(s));
+        const uint32_t b_base = smem_u32(stage_b(s));
+        int ksub = 4;
+        if (adapter) {
+          const int left = p.r - (it - p.main_steps) * kTileK;
+          ksub = left >= 64 ? 4 : (left + 15) / 16;
+        }
+        for (int kk = 0; kk < ksub; ++kk) {
+          const uint64_t bdesc = (MODE == kFwd) ? smem_desc_sw128(b_base + kk * 32, 16, 1024)
+                                                : smem_desc_sw128(b_base + kk * 2048, 8192, 1024);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint64_t adesc = smem_desc_sw128(a_base + h * kHalfABytes + kk * 32, 16, 1024);
+            umma_f16(tmem + h * kTileN, adesc, bdesc, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&sh->empty[s]);
+      }
+      if (ok) {
+        umma_commit(&sh->accum);
+      } else {
+        umma_commit(&sh->drain);
+        uint32_t dummy_abort = 0;
+        mbar_wait(&sh->drain, 0, &dummy_abort, nullptr);
+      }
+    }
+  } else {
+    // ---------------- dequant warps (one NF4 block = one tile row per thread)
+    const int t = threadIdx.x - 64;                  // 0..255 = tile row
+    const bool dq = p.double_quant != 0;
+    const float s_g = dq ? __ldg(p.absmax_scale) : 0.0f;
+    // Row of W and block column for main step `it`.
+    int64_t w_row;
+    int block_col0;
+    int row_step;
+    if (MODE == kFwd) {
+      w_row = int64_t(tile_n0) + t;                  // fixed W row, block column = it
+      block_col0 = 0;
+      row_step = 0;
+    } else {
+      w_row = t & 63;                                // W row = it * 64 + (t & 63)
+      block_col0 = tile_n0 / 64 + (t >> 6);          // fixed block column
+      row_step = 64;
+    }
+    auto scale_at = [&](int it) -> float {
+      const int64_t row = w_row + int64_t(row_step) * it;
+      if (row >= p.N) return 0.0f;
+      const int bcol = (MODE == kFwd) ? it : block_col0;
+      if (MODE == kDx && bcol >= p.kb_per_row) return 0.0f;
+      return load_scale(p.absmax_q, p.absmax, s_g, dq, row * p.kb_per_row + bcol);
+    };
+    float next_scale = p.main_steps > 0 ? scale_at(0) : 0.0f;
+    for (int it = 0; it < p.main_steps; ++it) {
+      const int s = it % kStages;
+      const uint32_t ph = (it / kStages) & 1;
+      const float scale = next_scale;
+      if (it + 1 < p.main_steps) next_scale = scale_at(it + 1);
+      if (!mbar_wait(&sh->full[s], ph, abort_flag, p.status)) break;
+      dequant_row(stage_c(s) + t * 32, scale, stage_b(s), uint32_t(t));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->bready[s]);
+    }
+
+    // ---------------- epilogue: TMEM -> registers -> bf16 -> global
+    const bool ok = mbar_wait(&sh->accum, 0, abort_flag, p.status);
+    tc_fence_after();
+    if (ok) {
+      const int quad = warp & 3;                     // TMEM lanes 32*quad .. +31
+      const int half = (warp - 2) >> 2;              // accumulator half
+      const int row = m0 + half * 128 + quad * 32 + lane;
+      for (int c = 0; c < kTileN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + half * kTileN + c * 32, v);
+        tmem_ld_wait();
+        const int col0 = tile_n0 + c * 32;
+        if (row < p.M) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int col = col0 + 8 * g;
+            if (col < p.out_cols) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
+              if (MODE == kFwd && p.bias != nullptr) {
+                const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
+                const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 bf = __bfloat1622float2(b2[e]);
+                  f[2 * e] += bf.x;
+                  f[2 * e + 1] += bf.y;
+                }
+              }
+              const uint4 o = make_uint4(bf16x2_rn(f[0], f[1]), bf16x2_rn(f[2], f[3]),
+                                         bf16x2_rn(f[4], f[5]), bf16x2_rn(f[6], f[7]));
+              *reinterpret_cast<uint4*>(p.out + int64_t(row) * p.out_cols + col) = o;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ adapter GEMM
+//
+// D[Mo, NP] = sum over a reduction range of A[Mo, red] * B[NP, red], one
+// 128-row tile per CTA and one slice of the reduction per blockIdx.y; fp32
+// partials land in part[slice][Mo][NP].  Operands come by TMA in 64-deep
+// steps, each either K-major (rows of the reduction) or MN-major.
+
+constexpr int kAdStages = 4;
+constexpr int kAdThreads = 192;    // TMA warp, MMA warp, 4 epilogue warps
+constexpr uint32_t kAdABytes = 128 * 128;
+
+struct AdapterParams {
+  int Mo;            // output rows
+  int NP;            // output cols (r rounded up to 64)
+  int red_steps;     // ceil(reduction / 64)
+  int steps_per_slice;
+  int a_mn;          // A operand MN-major
+  int b_mn;          // B operand MN-major
+  float* part;       // [slices][Mo][NP]
+  uint32_t* status;
+};
+
+struct AdapterShared {
+  uint64_t full[kAdStages];
+  uint64_t empty[kAdStages];
+  uint64_t accum;
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+__global__ void __launch_bounds__(kAdThreads, 1)
+    adapter_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                 const AdapterParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t b_bytes = uint32_t(p.NP) * 128u;
+  const uint32_t stage_bytes = kAdABytes + b_bytes;
+  AdapterShared* sh = reinterpret_cast<AdapterShared*>(smem + kAdStages * stage_bytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int mo0 = blockIdx.x * 128;
+  const int step0 = blockIdx.y * p.steps_per_slice;
+  const int step1 = min(step0 + p.steps_per_slice, p.red_steps);
+  const int nsteps = max(step1 - step0, 0);
+  volatile uint32_t* abort_flag = &sh->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAdStages; ++s) {
+      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->empty[s], 1);
+    }
+    mbar_init(&sh->accum, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    tma_prefetch(&tm_a);
+    tma_prefetch(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % kAdStages;
+        const uint32_t ph = (i / kAdStages) & 1;
+        if (!mbar_wait(&sh->empty[s], ph ^ 1, abort_flag, p.status)) break;
+        uint8_t* a = smem + s * stage_bytes;
+        uint8_t* b = a + kAdABytes;
+        const int red0 = (step0 + i) * 64;
+        mbar_arrive_expect_tx(&sh->full[s], stage_bytes);
+        if (p.a_mn) {
+          tma_load_2d(a, &tm_a, &sh->full[s], mo0, red0);
+          tma_load_2d(a + 8192, &tm_a, &sh->full[s], mo0 + 64, red0);
+        } else {
+          tma_load_2d(a, &tm_a, &sh->full[s], red0, mo0);
+        }
+        if (p.b_mn) {
+          for (int g = 0; g < p.NP / 64; ++g) tma_load_2d(b + g * 8192, &tm_b, &sh->full[s], 64 * g, red0);
+        } else {
+          tma_load_2d(b, &tm_b, &sh->full[s], red0, 0);
+        }
+        ++issued;
+      }
+      if (*abort_flag) {
+        for (int i = issued - 1; i >= 0 && i >= issued - kAdStages; --i) {
+          uint32_t dummy_abort = 0;
+          mbar_wait(&sh->full[i % kAdStages], (i / kAdStages) & 1, &dummy_abort, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, p.NP, p.a_mn != 0, p.b_mn != 0);
+      bool ok = true;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % kAdStages;
+        const uint32_t ph = (i / kAdStages) & 1;
+        ok = mbar_wait(&sh->full[s], ph, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + s * stage_bytes);
+        const uint32_t b_base = a_base + kAdABytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t adesc = p.a_mn ? smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                        : smem_desc_sw128(a_base + kk * 32, 16, 1024);
+          const uint64_t bdesc = p.b_mn ? smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
+                                        : smem_desc_sw128(b_base + kk * 32, 16, 1024);
+          umma_f16(tmem, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&sh->empty[s]);
+      }
+      if (ok) {
+        umma_commit(&sh->accum);
+      } else {
+        umma_commit(&sh->drain);
+        uint32_t dummy_abort = 0;
+        mbar_wait(&sh->drain, 0, &dummy_abort, nullptr);
+      }
+    }
+  } else {
+    // epilogue warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1
+    const bool ok = mbar_wait(&sh->accum, 0, abort_flag, p.status);
+    tc_fence_after();
+    const int quad = warp & 3;
+    const int row = mo0 + quad * 32 + lane;
+    float* dst = p.part + (int64_t(blockIdx.y) * p.Mo + row) * p.NP;
+    for (int c = 0; c < p.NP / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + c * 32, v);
+      tmem_ld_wait();
+      if (row < p.Mo) {
+        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          float4 f;
+          if (ok && nsteps > 0) {
+            f = make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
+                            __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+          } else {
+            f = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          d4[g] = f;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// out = sum of the slices, for columns < r:
+//   kind 0: bf16(scale * sum) into out_bf16[Mo][r]
+//   kind 1: fp32 sum into out_f32[Mo][r]
+//   kind 2: fp32 sum transposed into out_f32[r][Mo]
+__global__ void __launch_bounds__(256) adapter_finalize(const float* __restrict__ part, int slices,
+                                                        int Mo, int NP, int r, int kind, float scale,
+                                                        __nv_bfloat16* __restrict__ out_bf16,
+                                                        float* __restrict__ out_f32) {
+  const int64_t total = int64_t(Mo) * r;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    int64_t row, col;
+    if (kind == 2) {        // walk the transposed output contiguously
+      col = i / Mo;
+      row = i % Mo;
+    } else {
+      row = i / r;
+      col = i % r;
+    }
+    float acc = 0.0f;
+    for (int s = 0; s < slices; ++s) acc += part[(int64_t(s) * Mo + row) * NP + col];
+    if (kind == 0) {
+      out_bf16[row * r + col] = __float2bfloat16_rn(acc * scale);
+    } else if (kind == 1) {
+      out_f32[row * r + col] = acc;
+    } else {
+      out_f32[col * int64_t(Mo) + row] = acc;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major matrix: `inner` elements per row, `outer` rows.
+bool make_map(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+              uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const uint32_t esize = bf16 ? 2 : 1;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * esize};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult res = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                    const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS;
+}
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Split of a reduction of `red_steps` 64-deep steps over Mo/128 tiles so that
+// about two CTAs per SM of a 148-SM part run; independent of the device so
+// the workspace size is a pure function of the shapes.
+struct SplitPlan {
+  int tiles, slices, per;
+};
+SplitPlan plan_split(int64_t Mo, int64_t red) {
+  SplitPlan sp;
+  sp.tiles = int(cdiv(Mo, 128));
+  const int steps = int(std::max<int64_t>(cdiv(red, 64), 1));
+  int want = int(cdiv(296, sp.tiles));
+  want = std::max(1, std::min(want, std::min(16, std::max(1, steps / 4))));
+  sp.per = int(cdiv(steps, want));
+  sp.slices = int(cdiv(steps, sp.per));
+  return sp;
+}
+
+int round_np(int r) { return int(cdiv(r, 64) * 64); }
+
+size_t part_bytes(int64_t Mo, int64_t red, int r) {
+  const SplitPlan sp = plan_split(Mo, red);
+  return align256(size_t(sp.slices) * size_t(Mo) * size_t(round_np(r)) * sizeof(float));
+}
+
+bool g_attr_done = false;
+
+cudaError_t set_attrs() {
+  if (g_attr_done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm<kFwd>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(kFusedSmem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fused_nf4_gemm<kDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kFusedSmem));
+  const size_t ad_smem = kAdStages * (kAdABytes + 256 * 128) + 1024 + 256;
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(adapter_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, int(ad_smem));
+  if (e == cudaSuccess) g_attr_done = true;
+  return e;
+}
+
+// One rank-r product through adapter_gemm + adapter_finalize.
+//   a_mn/b_mn: operand majorness; a_base/b_base: matrices as [outer][inner].
+struct AdapterJob {
+  const void* a; uint64_t a_inner, a_outer; bool a_mn;
+  const void* b; uint64_t b_inner, b_outer; bool b_mn;
+  int64_t Mo, red;
+  int r;
+  int kind;          // see adapter_finalize
+  float scale;
+  __nv_bfloat16* out_bf16;
+  float* out_f32;
+};
+
+cudaError_t run_adapter(const AdapterJob& j, float* part, uint32_t* status, int sms,
+                        cudaStream_t st, int* launches) {
+  const int NP = round_np(j.r);
+  CUtensorMap ma, mb;
+  bool ok = j.a_mn ? make_map(&ma, j.a, true, j.a_inner, j.a_outer, 64, 64, true)
+                   : make_map(&ma, j.a, true, j.a_inner, j.a_outer, 64, 128, true);
+  ok = ok && (j.b_mn ? make_map(&mb, j.b, true, j.b_inner, j.b_outer, 64, 64, true)
+                     : make_map(&mb, j.b, true, j.b_inner, j.b_outer, 64, uint32_t(NP), true));
+  if (!ok) return cudaErrorInvalidValue;
+  const SplitPlan sp = plan_split(j.Mo, j.red);
+  AdapterParams p;
+  p.Mo = int(j.Mo);
+  p.NP = NP;
+  p.red_steps = int(std::max<int64_t>(cdiv(j.red, 64), 1));
+  p.steps_per_slice = sp.per;
+  p.a_mn = j.a_mn;
+  p.b_mn = j.b_mn;
+  p.part = part;
+  p.status = status;
+  const size_t smem = kAdStages * (kAdABytes + size_t(NP) * 128) + 1024 + 256;
+  adapter_gemm<<<dim3(sp.tiles, sp.slices), kAdThreads, smem, st>>>(ma, mb, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ++*launches;
+  const int64_t total = j.Mo * j.r;
+  const int grid = int(std::min<int64_t>(cdiv(total, 256), int64_t(sms) * 8));
+  adapter_finalize<<<std::max(grid, 1), 256, 0, st>>>(part, sp.slices, int(j.Mo), NP, j.r, j.kind,
+                                                      j.scale, j.out_bf16, j.out_f32);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+FusedParams fused_params(const LinearArgs& a, int mode) {
+  FusedParams p;
+  p.M = int(a.M);
+  p.N = int(a.N);
+  p.K = int(a.K);
+  p.r = a.r;
+  p.main_steps = mode == kFwd ? int(a.K / 64) : int(cdiv(a.N, 64));
+  p.adapter_steps = int(cdiv(a.r, 64));
+  p.out_cols = mode == kFwd ? int(a.N) : int(a.K);
+  p.kb_per_row = int(a.K / 64);
+  p.double_quant = a.w->double_quant;
+  p.absmax_q = a.w->absmax_q;
+  p.absmax = a.w->absmax;
+  p.absmax_scale = a.w->absmax_scale;
+  p.bias = static_cast<const __nv_bfloat16*>(mode == kFwd ? a.bias : nullptr);
+  p.out = static_cast<__nv_bfloat16*>(mode == kFwd ? a.y : a.dx);
+  p.status = a.status;
+  return p;
+}
+
+// Workspace regions after the header (all 256-byte aligned):
+//   fwd: [T bf16 M x r (when t_out is null)] [partials]
+//   bwd: [T bf16 M x r (when t is null)] [U bf16 M x r] [partials]
+size_t mr_bytes(int64_t M, int r) { return align256(size_t(M) * size_t(r) * 2); }
+
+size_t fwd_part_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  (void)N;
+  return part_bytes(M, K, r);
+}
+
+size_t bwd_part_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  size_t b = part_bytes(M, K, r);                 // T recompute
+  b = std::max(b, part_bytes(M, N, r));           // U
+  b = std::max(b, part_bytes(N, M, r));           // dB
+  b = std::max(b, part_bytes(K, M, r));           // dA^T
+  return b;
+}
+
+cudaError_t forward_adapter_T(const LinearArgs& a, __nv_bfloat16* T, float* part, int sms,
+                              cudaStream_t st, int* launches) {
+  AdapterJob j{};
+  j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = false;
+  j.b = a.A; j.b_inner = a.K; j.b_outer = a.r; j.b_mn = false;
+  j.Mo = a.M; j.red = a.K; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = T;
+  return run_adapter(j, part, a.status, sms, st, launches);
+}
+
+}  // namespace
+
+size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, int r) {
+  if (!backward) return mr_bytes(M, r) + fwd_part_bytes(M, N, K, r);
+  return 2 * mr_bytes(M, r) + bwd_part_bytes(M, N, K, r);
+}
+
+cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches) {
+  cudaError_t e = set_attrs();
+  if (e != cudaSuccess) return e;
+  uint8_t* ws = a.ws + kWsHeader;
+  __nv_bfloat16* T = a.t_out ? static_cast<__nv_bfloat16*>(a.t_out) : reinterpret_cast<__nv_bfloat16*>(ws);
+  float* part = reinterpret_cast<float*>(ws + mr_bytes(a.M, a.r));
+
+  e = forward_adapter_T(a, T, part, sms, st, launches);
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap ta, ta2, tb2, tc;
+  bool ok = make_map(&ta, a.x, true, a.K, a.M, 64, 128, true);
+  ok = ok && make_map(&ta2, T, true, a.r, a.M, 64, 128, true);
+  ok = ok && make_map(&tb2, a.B, true, a.r, a.N, 64, 256, true);
+  ok = ok && make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, 256, false);
+  if (!ok) return cudaErrorInvalidValue;
+  const FusedParams p = fused_params(a, kFwd);
+  dim3 grid(unsigned(cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kTileM)));
+  fused_nf4_gemm<kFwd><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches) {
+  cudaError_t e = set_attrs();
+  if (e != cudaSuccess) return e;
+  uint8_t* ws = a.ws + kWsHeader;
+  __nv_bfloat16* T_ws = reinterpret_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* U = reinterpret_cast<__nv_bfloat16*>(ws + mr_bytes(a.M, a.r));
+  float* part = reinterpret_cast<float*>(ws + 2 * mr_bytes(a.M, a.r));
+
+  const __nv_bfloat16* T = static_cast<const __nv_bfloat16*>(a.t_in);
+  if (T == nullptr) {
+    e = forward_adapter_T(a, T_ws, part, sms, st, launches);
+    if (e != cudaSuccess) return e;
+    T = T_ws;
+  }
+  // U = s dy B   (A: dy K-major over n; B: B_lora [N, r] MN-major over n)
+  {
+    AdapterJob j{};
+    j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = false;
+    j.b = a.B; j.b_inner = a.r; j.b_outer = a.N; j.b_mn = true;
+    j.Mo = a.M; j.red = a.N; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = U;
+    e = run_adapter(j, part, a.status, sms, st, launches);
+    if (e != cudaSuccess) return e;
+  }
+  // dB = dy^T T   (A: dy^T MN-major over m; B: T [M, r] MN-major over m)
+  {
+    AdapterJob j{};
+    j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = true;
+    j.b = T; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
+    j.Mo = a.N; j.red = a.M; j.r = a.r; j.kind = 1; j.scale = 1.0f; j.out_f32 = a.dB;
+    e = run_adapter(j, part, a.status, sms, st, launches);
+    if (e != cudaSuccess) return e;
+  }
+  // dA^T = x^T U  (A: x^T MN-major over m; B: U [M, r] MN-major over m), stored as dA [r, K]
+  {
+    AdapterJob j{};
+    j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = true;
+    j.b = U; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
+    j.Mo = a.K; j.red = a.M; j.r = a.r; j.kind = 2; j.scale = 1.0f; j.out_f32 = a.dA;
+    e = run_adapter(j, part, a.status, sms, st, launches);
+    if (e != cudaSuccess) return e;
+  }
+  if (a.dx == nullptr) return cudaSuccess;
+  // dx = dy W' + U A
+  CUtensorMap ta, ta2, tb2, tc;
+  bool ok = make_map(&ta, a.dy, true, a.N, a.M, 64, 128, true);
+  ok = ok && make_map(&ta2, U, true, a.r, a.M, 64, 128, true);
+  ok = ok && make_map(&tb2, a.A, true, a.K, a.r, 64, 64, true);
+  ok = ok && make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, 64, false);
+  if (!ok) return cudaErrorInvalidValue;
+  const FusedParams p = fused_params(a, kDx);
+  dim3 grid(unsigned(cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kTileM)));
+  fused_nf4_gemm<kDx><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 }  // namespace nf4

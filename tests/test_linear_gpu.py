@@ -1,0 +1,153 @@
+"""GPU parity for the QLoRA linear forward and adapter backward, through the C
+ABI, against the fp64 CPU oracle on the same seeded inputs.
+
+Tolerance (per tensor): max |gpu - oracle| <= 1e-2 * max |oracle|.  The
+adapter term is ~1-2% of y and dx at these distributions, so every case is
+also run with an all-zero base weight, which leaves only the adapter path.
+"""
+import numpy as np
+import pytest
+
+from oracle import nf4_oracle as O
+from qlora_linear_layers_nf4_b200 import workloads as WL
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-2
+
+
+def _Q():
+    from qlora_linear_layers_nf4_b200 import nf4qlora as Q
+    return Q
+
+
+def _bf(dev, bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def _f(t):
+    return t.float().cpu().double().numpy()
+
+
+def _close(name, got, want, tol=TOL):
+    scale = np.max(np.abs(want))
+    err = np.max(np.abs(got - want))
+    assert err <= tol * scale, f"{name}: max err {err:.3e} vs {tol} * {scale:.3e}"
+
+
+class Run:
+    """Quantize W on the GPU, run fwd + bwd, keep everything for checks."""
+
+    def __init__(self, case, dev, m=None, zero_w=False, bias=False, rows=None, pass_t=True):
+        import torch
+        Q = _Q()
+        self.case = case
+        inp = WL.draw_linear(case, m=m)
+        if zero_w:
+            inp.w = np.zeros_like(inp.w)
+        self.inp = inp
+        self.ref_q = O.quantize(inp.w, case.block_size, double=case.double_quant)
+        self.q = Q.quantize(torch.from_numpy(inp.w).to(dev), case.block_size, case.double_quant)
+        self.x, self.A, self.B, self.dy = (_bf(dev, v) for v in (inp.x, inp.a, inp.b, inp.dy))
+        self.bias = None
+        self.bias_np = None
+        if bias:
+            rng = np.random.default_rng(case.seed + 99)
+            bb = WL.to_bf16_bits(rng.standard_normal(case.n).astype(np.float32) * np.float32(0.1))
+            self.bias = _bf(dev, bb)
+            self.bias_np = WL.bf16_bits_to_f32(bb).astype(np.float64)
+        self.y, self.T = Q.linear_fwd(self.q, self.x, self.A, self.B, case.alpha, bias=self.bias)
+        self.dA, self.dB, self.dx = Q.linear_bwd(self.q, self.x, self.A, self.B, case.alpha, self.dy,
+                                                 t=self.T if pass_t else None)
+        torch.cuda.synchronize()
+        self.w_hat = O.bf16_to_f32(O.dequantize(self.ref_q, "bf16")).astype(np.float64)
+        f = WL.bf16_bits_to_f32
+        self.xn, self.an, self.bn, self.dyn = (f(v).astype(np.float64) for v in (inp.x, inp.a, inp.b, inp.dy))
+        self.s = case.alpha / case.r
+
+    def check_forward(self, rows=None):
+        rows = np.arange(self.xn.shape[0]) if rows is None else rows
+        y_ref, t_ref = O.qlora_forward(self.xn[rows], self.w_hat, self.an, self.bn, self.case.alpha,
+                                       bias=self.bias_np)
+        _close("y", _f(self.y)[rows], y_ref)
+        _close("T", _f(self.T)[rows], self.s * t_ref)
+
+    def check_backward(self, rows=None):
+        d_a, d_b, _ = O.qlora_backward(self.xn, self.w_hat, self.an, self.bn, self.case.alpha, self.dyn)
+        _close("dA", _f(self.dA), d_a)
+        _close("dB", _f(self.dB), d_b)
+        rows = np.arange(self.xn.shape[0]) if rows is None else rows
+        _, _, d_x = O.qlora_backward(self.xn[rows], self.w_hat, self.an, self.bn, self.case.alpha,
+                                     self.dyn[rows])
+        _close("dx", _f(self.dx)[rows], d_x)
+
+
+def test_tiny_layer(cuda_device):
+    r = Run(WL.TINY, cuda_device)
+    r.check_forward()
+    r.check_backward()
+
+
+def test_tiny_layer_adapter_only(cuda_device):
+    r = Run(WL.TINY, cuda_device, zero_w=True)
+    assert np.all(r.ref_q["codes"] == 0x77)
+    r.check_forward()
+    r.check_backward()
+
+
+@pytest.mark.parametrize("m,n,k,rank,dq,bias", [
+    (300, 264, 320, 16, True, True),      # ragged M, N not a multiple of the 256 tile
+    (512, 512, 512, 64, True, False),     # several full tiles
+    (257, 1032, 192, 24, False, True),    # r not a multiple of 16, N % 64 != 0
+    (64, 768, 1024, 128, True, False),    # r spanning two 64-wide adapter steps
+    (33, 256, 4096, 8, True, False),      # smallest rank, long K
+])
+def test_ragged_shapes(cuda_device, m, n, k, rank, dq, bias):
+    case = WL.LinearCase(f"ragged {m}x{n}x{k} r={rank}", n=n, k=k, m=m, r=rank, alpha=2.0 * rank,
+                         seed=1000 + m + n + k + rank, double_quant=dq)
+    for zero_w in (False, True):
+        r = Run(case, cuda_device, zero_w=zero_w, bias=bias and not zero_w)
+        r.check_forward()
+        r.check_backward()
+
+
+def test_recomputed_t_matches(cuda_device):
+    import torch
+    case = WL.LinearCase("recompute t", n=512, k=512, m=200, r=32, alpha=64.0, seed=77)
+    r1 = Run(case, cuda_device, pass_t=True)
+    r2 = Run(case, cuda_device, pass_t=False)
+    assert torch.equal(r1.dA, r2.dA) and torch.equal(r1.dB, r2.dB) and torch.equal(r1.dx, r2.dx)
+
+
+@pytest.mark.parametrize("case", WL.DECODE, ids=lambda c: c.name)
+def test_decode_shapes(cuda_device, case):
+    r = Run(case, cuda_device)
+    r.check_forward()
+    r.check_backward()
+    r0 = Run(case, cuda_device, zero_w=True)
+    r0.check_forward()
+
+
+def test_prefill_full_size_sampled(cuda_device):
+    # Full 11008x4096 layer, M = 4096: dA and dB checked whole, y and dx on
+    # 64 sampled token rows (the oracle computes those one by one).
+    r = Run(WL.PREFILL, cuda_device)
+    rows = np.random.default_rng(0).choice(r.xn.shape[0], 64, replace=False)
+    rows = np.concatenate([rows, [0, r.xn.shape[0] - 1]])
+    r.check_forward(rows)
+    r.check_backward(rows)
+
+
+def test_prefill_full_size_adapter_only(cuda_device):
+    r = Run(WL.PREFILL, cuda_device, zero_w=True)
+    rows = np.random.default_rng(1).choice(r.xn.shape[0], 32, replace=False)
+    r.check_forward(rows)
+    r.check_backward(rows)
+
+
+@pytest.mark.parametrize("case", WL.BLOCK, ids=lambda c: c.name.split()[1])
+def test_decoder_block_targets_sampled(cuda_device, case):
+    r = Run(case, cuda_device)
+    rows = np.random.default_rng(2).choice(r.xn.shape[0], 32, replace=False)
+    r.check_forward(rows)
+    r.check_backward(rows)
