@@ -1,0 +1,532 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 linear hot path on B200.
+
+Headline (the JSON line's `value`): forward + adapter backward of the
+prefill/training layer -- W 11008x4096 NF4 (block 64, double quant), x of
+4096 tokens, r = 64, alpha = 16 -- in TFLOP/s of algorithmic work
+(4 M N K + 6 M r (N + K) per step), inputs resident in HBM, L2 flushed
+before every timed step.  The same line carries the dominant kernel's
+roofline, the CPU oracle's time on this host, an end-to-end figure through
+the C ABI from pinned host buffers, the SM clocks seen while timing, and the
+other rows of the hot path (quantize / dequantize GB/s, decode GEMV GB/s,
+the seven-target decoder block).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs the same layer on its own 4096 tokens (weak
+scaling) and the adapter gradients are all-reduced over NCCL each step.
+--impl reference times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA NF4 linear fwd+bwd TFLOP/s; NF4 (de)quant & GEMV GB/s vs B200 roofline"
+FLUSH_BYTES = 256 << 20          # > 2x the 126 MB L2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture, keyed by
+# the hash of the kernel source it was taken on (see profiles/); reported as
+# null once the source changes.
+NCU_TRAFFIC = {}
+
+
+def linear_flops(m, n, k, r):
+    return 4 * m * n * k + 6 * m * r * (n + k)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for name in ("qlora_gemm.cu", "tc_common.cuh", "nf4_common.cuh"):
+        with open(os.path.join(ROOT, "qlora_linear_layers_nf4_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while timing."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for name, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------- helpers
+
+def bf16_dev(bits, dev):
+    import numpy as np
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def cpu_cores():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    threads = n
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            threads = max(i.get("num_threads", n) for i in info)
+    except Exception:
+        pass
+    return n, threads
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_step_sample(case, m_sample):
+    """One bounded oracle step: dequantize W (bf16) and run fwd + bwd on
+    m_sample tokens of the workload.  Returns (seconds, flops)."""
+    import numpy as np
+    from oracle import nf4_oracle as O
+    from qlora_linear_layers_nf4_b200 import workloads as WL
+    inp = WL.draw_linear(case, m=m_sample)
+    ref_q = O.quantize(inp.w, case.block_size, double=case.double_quant)
+    f = WL.bf16_bits_to_f32
+    x, a, b, dy = (f(v) for v in (inp.x, inp.a, inp.b, inp.dy))
+
+    def step():
+        w_hat = O.bf16_to_f32(O.dequantize(ref_q, "bf16"))
+        O.qlora_forward(x, w_hat, a, b, case.alpha)
+        O.qlora_backward(x, w_hat, a, b, case.alpha, dy)
+
+    return step, linear_flops(m_sample, case.n, case.k, case.r)
+
+
+# --------------------------------------------------------------------- our arm
+
+class Timer:
+    def __init__(self, n):
+        import torch
+        self.s = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        self.e = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    def total_ms(self):
+        return sum(a.elapsed_time(b) for a, b in zip(self.s, self.e))
+
+
+def time_steps(fn, steps, warmup, flush=None, barrier=None):
+    """Run warmup + timed steps; each timed step bracketed by events, with an
+    L2 flush before it (outside the brackets).  Returns total ms."""
+    import torch
+    for _ in range(warmup):
+        if flush is not None:
+            flush()
+        fn()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    t = Timer(steps)
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        t.s[i].record()
+        fn()
+        t.e[i].record()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    return t.total_ms()
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from qlora_linear_layers_nf4_b200 import nf4qlora as Q
+    from qlora_linear_layers_nf4_b200 import workloads as WL
+    from qlora_linear_layers_nf4_b200.dp import AdapterGradBuffer, max_over_ranks
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    barrier = (lambda: dist.barrier()) if world > 1 else None
+    Q.lib()
+
+    case = WL.PREFILL
+    M, N, K, r = case.m, case.n, case.k, case.r
+    inp = WL.draw_linear(case)
+    q = Q.quantize(torch.from_numpy(inp.w).to(dev), case.block_size, case.double_quant)
+    x, A, B, dy = (bf16_dev(v, dev) for v in (inp.x, inp.a, inp.b, inp.dy))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    grads = AdapterGradBuffer(r, K, N, dev)
+    ws = Q.Workspace(dev)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = lambda: flush_buf.zero_()
+
+    def step():
+        Q.linear_fwd(q, x, A, B, case.alpha, out=y, t_out=T, workspace=ws)
+        Q.linear_bwd(q, x, A, B, case.alpha, dy, t=T, dA=grads.dA, dB=grads.dB, dx=dx, workspace=ws)
+        if world > 1:
+            grads.all_reduce()
+
+    flops = linear_flops(M, N, K, r)
+    clocks = ClockSampler(local)
+    for _ in range(max(args.warmup, 0)):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    launches0 = Q.launch_count()
+    Q.profile_begin()
+    clocks.start()
+    t = Timer(args.steps)
+    for i in range(args.steps):
+        flush()
+        t.s[i].record()
+        step()
+        t.e[i].record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    kernels = Q.profile_end()
+    if barrier:
+        barrier()
+    launches = Q.launch_count() - launches0
+    total_ms = max_over_ranks(t.total_ms(), dev)
+    ms_per_step = total_ms / args.steps
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    if ws.read_status() != 0:
+        raise RuntimeError("device status reported an error during the benchmark")
+
+    pk, pk_kind = peaks()
+    # dominant kernel: the fused dequant + tcgen05 GEMM (forward and dx launches)
+    fwd_n, fwd_ms = kernels.get("fused_nf4_gemm_fwd", (0, 0.0))
+    dx_n, dx_ms = kernels.get("fused_nf4_gemm_dx", (0, 0.0))
+    fwd_flops = 2 * M * N * K + 2 * M * r * N
+    dx_flops = 2 * M * N * K + 2 * M * r * K
+    total_kernel_ms = sum(v[1] for v in kernels.values())
+    fused_launches = fwd_n + dx_n
+    achieved = ((fwd_n * fwd_flops + dx_n * dx_flops) / ((fwd_ms + dx_ms) * 1e-3) / 1e12
+                if fused_launches else None)
+    peak = pk.get("bf16_tflops_sustained") or pk.get("bf16_tflops")
+    src = source_hash()
+    traffic = NCU_TRAFFIC.get(src)
+    roofline = {
+        "kernel": "fused_nf4_gemm (fwd + dx launches)",
+        "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+        "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside a long step)",
+        "flops_per_launch": {"fwd": fwd_flops, "dx": dx_flops},
+        "share_of_step_kernel_time": (fwd_ms + dx_ms) / total_kernel_ms if total_kernel_ms else None,
+        "source_hash": src,
+    }
+    kern = {k: {"launches": n, "avg_us": 1e3 * ms / n, "share": ms / total_kernel_ms}
+            for k, (n, ms) in kernels.items()}
+
+    # ---- end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hx = x.cpu().pin_memory()
+        hdy = dy.cpu().pin_memory()
+        hdA = torch.empty_like(grads.dA, device="cpu").pin_memory()
+        hdB = torch.empty_like(grads.dB, device="cpu").pin_memory()
+        xd = torch.empty_like(x)
+        dyd = torch.empty_like(dy)
+
+        def e2e_step():
+            xd.copy_(hx, non_blocking=True)
+            dyd.copy_(hdy, non_blocking=True)
+            Q.linear_fwd(q, xd, A, B, case.alpha, out=y, t_out=T, workspace=ws)
+            Q.linear_bwd(q, xd, A, B, case.alpha, dyd, t=T, dA=grads.dA, dB=grads.dB, dx=dx,
+                         workspace=ws)
+            if world > 1:
+                grads.all_reduce()
+            hdA.copy_(grads.dA, non_blocking=True)
+            hdB.copy_(grads.dB, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 10))
+        ms = time_steps(e2e_step, e2e_steps, 2, flush=flush, barrier=barrier)
+        ms = max_over_ranks(ms, dev)
+        e2e = {"value": flops * world * e2e_steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": hx.numel() * 2 + hdy.numel() * 2,
+               "d2h_bytes_per_step": (hdA.numel() + hdB.numel()) * 4,
+               "ms_per_step": ms / e2e_steps}
+
+    rows = {}
+    if not args.no_rows:
+        rows = measure_rows(args, dev, flush, pk, pk_kind, barrier)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(case, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded normal draws (W ~ N(0, 0.02^2), x, dy ~ N(0, 1), "
+                "A ~ N(0, 1/K), B ~ N(0, 0.01^2)), bf16 inputs, NF4 weight quantized on device",
+        "config": {
+            "workload": "QLoRA linear fwd+bwd, W 11008x4096 NF4 block 64 double-quant, "
+                        "M=4096 tokens per GPU, r=64, alpha=16 (dA, dB, dx)",
+            "tokens_per_gpu": M, "out_features": N, "in_features": K, "rank": r,
+            "flops_per_step_per_gpu": flops, "parallelism": f"dp{world}",
+            "l2": "flushed before every timed step (256 MiB memset outside the step events)",
+            "grad_allreduce": "NCCL all-reduce of dA+dB (fp32) per step" if world > 1 else "none (1 GPU)",
+        },
+        "roofline": roofline,
+        "kernels": kern,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk,
+        "gpu_launches": launches,
+        "gpu_launches_per_step": launches / args.steps,
+        "rows": rows,
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure_rows(args, dev, flush, pk, pk_kind, barrier):
+    """The other rows of the hot path, each timed on its own."""
+    import numpy as np
+    import torch
+    from qlora_linear_layers_nf4_b200 import nf4qlora as Q
+    from qlora_linear_layers_nf4_b200 import workloads as WL
+
+    hbm = pk.get("hbm_gbs")
+    out = {}
+    reps = max(5, min(args.steps, 20))
+
+    def mem_row(name, fn, nbytes, kernel_names):
+        Q.profile_begin()
+        ms = time_steps(fn, reps, 3, flush=flush, barrier=barrier)
+        k = Q.profile_end()
+        kms = sum(k.get(n, (0, 0.0))[1] for n in kernel_names)
+        kn = sum(k.get(n, (0, 0.0))[0] for n in kernel_names)
+        gbs = nbytes * reps / (ms * 1e-3) / 1e9
+        kgbs = nbytes * reps / (kms * 1e-3) / 1e9 if kms else None
+        out[name] = {"GB/s": gbs, "kernel_GB/s": kgbs, "frac_hbm": (kgbs / hbm) if kgbs else None,
+                     "us_per_call": 1e3 * ms / reps, "bytes": nbytes,
+                     "kernel_launches_per_call": kn / reps if reps else None}
+
+    w = torch.from_numpy(WL.draw_weight(WL.QUANT_SHAPE, WL.QUANT_SEED)).to(dev)
+    numel = w.numel()
+    nb = numel // 64
+    ws = Q.Workspace(dev)
+    q0 = Q.quantize(w, 64, False, workspace=ws)
+    q1 = Q.quantize(w, 64, True, workspace=ws)
+    mem_row("quantize_4096x4096_noDQ", lambda: Q.quantize(w, 64, False, workspace=ws),
+            numel * 4 + numel // 2 + nb * 4, ["nf4_quantize"])
+    mem_row("quantize_4096x4096_DQ", lambda: Q.quantize(w, 64, True, workspace=ws),
+            numel * 4 + numel // 2 + nb + 4, ["nf4_quantize", "nf4_double_quant"])
+    out32 = torch.empty((4096, 4096), dtype=torch.float32, device=dev)
+    for dq, qq in (("noDQ", q0), ("DQ", q1)):
+        sb = nb * 4 if dq == "noDQ" else nb + 4
+        for kind, esz in (("f32", 4), ("bf16", 2)):
+            mem_row(f"dequantize_{kind}_{dq}", lambda qq=qq, kind=kind: Q.dequantize(qq, kind),
+                    numel // 2 + sb + numel * esz, ["nf4_dequantize"])
+    del out32
+
+    # decode-shape forward (weight streaming)
+    for case in WL.DECODE:
+        inp = WL.draw_linear(case)
+        qd = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True, workspace=ws)
+        x, A, B = (bf16_dev(v, dev) for v in (inp.x, inp.a, inp.b))
+        y = torch.empty((case.m, case.n), dtype=torch.bfloat16, device=dev)
+        wsd = Q.Workspace(dev)
+        nbytes = (case.n * case.k // 2 + case.n * case.k // 64 + 4 + 2 * case.r * case.k
+                  + 2 * case.n * case.r + 2 * case.m * (case.k + case.n))
+        mem_row(f"decode_fwd_M{case.m}", lambda: Q.linear_fwd(qd, x, A, B, case.alpha, out=y,
+                                                               want_t=False, workspace=wsd),
+                nbytes, ["nf4_gemv", "nf4_gemv_reduce", "adapter_gemm", "adapter_finalize",
+                         "fused_nf4_gemm_fwd"])
+
+    # the seven targets of one decoder block, fwd + bwd each
+    if not args.no_block:
+        layers = []
+        for case in WL.BLOCK:
+            inp = WL.draw_linear(case)
+            qb = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True, workspace=ws)
+            x, A, B, dy = (bf16_dev(v, dev) for v in (inp.x, inp.a, inp.b, inp.dy))
+            layers.append((case, qb, x, A, B, dy,
+                           torch.empty((case.m, case.n), dtype=torch.bfloat16, device=dev),
+                           torch.empty((case.m, case.r), dtype=torch.bfloat16, device=dev),
+                           torch.empty((case.m, case.k), dtype=torch.bfloat16, device=dev)))
+        wsb = Q.Workspace(dev)
+
+        def block_step():
+            for case, qb, x, A, B, dy, y, T, dx in layers:
+                Q.linear_fwd(qb, x, A, B, case.alpha, out=y, t_out=T, workspace=wsb)
+                Q.linear_bwd(qb, x, A, B, case.alpha, dy, t=T, dx=dx, workspace=wsb)
+
+        flops = sum(linear_flops(c.m, c.n, c.k, c.r) for c in WL.BLOCK)
+        bsteps = max(3, min(args.steps, 10))
+        ms = time_steps(block_step, bsteps, 2, flush=flush, barrier=barrier)
+        out["decoder_block_7_targets_fwd_bwd"] = {
+            "TFLOP/s": flops * bsteps / (ms * 1e-3) / 1e12, "ms_per_block": ms / bsteps,
+            "flops": flops, "frac_bf16_sustained": flops * bsteps / (ms * 1e-3) / 1e12 /
+            (pk.get("bf16_tflops_sustained") or pk.get("bf16_tflops"))}
+    return out
+
+
+def cpu_baseline(case, seconds):
+    """The oracle on this host's cores, on a bounded sample of the workload."""
+    n_cores, threads = cpu_cores()
+    m_sample = 256
+    step, flops = oracle_step_sample(case, m_sample)
+    t0 = time.perf_counter()
+    step()
+    one = time.perf_counter() - t0
+    reps = max(1, int(seconds / max(one, 1e-3)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        step()
+    dt = time.perf_counter() - t0
+    return {"value": flops * reps / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{m_sample} of the 4096 tokens of the 11008x4096 r=64 layer: NF4 dequant of "
+                      f"the whole weight + fp64 fwd+bwd on those tokens, {reps} reps "
+                      f"({dt:.1f} s); NumPy fp64, BLAS threads={threads}, host cores={n_cores}, "
+                      f"cpu={cpu_model()}"}
+
+
+# --------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from qlora_linear_layers_nf4_b200 import workloads as WL
+    case = WL.PREFILL
+    n_cores, threads = cpu_cores()
+    m_sample = 128
+    step, flops = oracle_step_sample(case, m_sample)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    sample = (f"each step: NF4 dequant of the whole 11008x4096 weight + fp64 fwd+bwd on "
+              f"{m_sample} of the 4096 tokens; NumPy, BLAS threads={threads}, host cores={n_cores}, "
+              f"cpu={cpu_model()}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same recipe as our arm)",
+        "config": {"workload": "QLoRA linear fwd+bwd, W 11008x4096 NF4 block 64 double-quant, "
+                               "M=4096 tokens per GPU, r=64, alpha=16 (dA, dB, dx)",
+                   "reference": "CPU oracle (oracle/nf4_oracle.py) on the host cores, bounded sample"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
+    ap.add_argument("--no-block", action="store_true", help="skip the decoder-block row")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -126,6 +126,23 @@ NF4_API void nf4_codebook(float* levels, float* thresholds);
 NF4_API int64_t nf4_launch_count(void);
 
 /*
+ * Per-kernel timing, for benchmarks.  nf4_profile_begin() turns recording on
+ * (and clears earlier totals): every kernel the library launches is then
+ * bracketed by two CUDA events on its launch stream.  nf4_profile_end()
+ * waits for the recorded events, adds each bracket's elapsed time to its
+ * kernel's total and turns recording off.  nf4_profile_get() returns the
+ * number of timed launches and their summed milliseconds for a kernel id
+ * (0 <= id < nf4_profile_kernel_count()); nf4_kernel_name() names it.
+ * The events are created by the library (no device memory).  Returns
+ * NF4_OK, NF4_ERR_INVALID_ARG for a bad id, NF4_ERR_CUDA on event failure.
+ */
+NF4_API nf4_status nf4_profile_begin(void);
+NF4_API nf4_status nf4_profile_end(void);
+NF4_API int nf4_profile_kernel_count(void);
+NF4_API const char* nf4_kernel_name(int kernel_id);
+NF4_API nf4_status nf4_profile_get(int kernel_id, int64_t* launches, double* total_ms);
+
+/*
  * Bytes of workspace an operation needs (0 = none).  M, N, K, r are the
  * linear-layer sizes (N = W rows, K = W cols); for NF4_OP_QUANTIZE and
  * NF4_OP_DEQUANTIZE pass N = rows, K = cols and M = r = 0.  Needs no GPU.

@@ -3,6 +3,8 @@
 // the stream was left untouched (the "refuse before writing anything" rule).
 #include <atomic>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "nf4_common.cuh"
 #include "kernels.h"
@@ -64,9 +66,103 @@ nf4_status check_linear(const nf4_weight* w, const void* x, int64_t M, const voi
   return NF4_OK;
 }
 
+// Event brackets recorded while profiling is on.
+struct ProfRecord {
+  cudaEvent_t start;
+  cudaEvent_t stop;
+  int id;
+};
+
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof_pending;
+std::vector<cudaEvent_t> g_prof_free;
+ProfRecord g_prof_open{nullptr, nullptr, -1};
+int64_t g_prof_count[nf4::kNumKernelIds];
+double g_prof_ms[nf4::kNumKernelIds];
+
+const char* const kKernelNames[nf4::kNumKernelIds] = {
+    "nf4_quantize", "nf4_double_quant", "nf4_dequantize", "adapter_gemm",
+    "adapter_finalize", "fused_nf4_gemm_fwd", "fused_nf4_gemm_dx", "nf4_gemv", "nf4_gemv_reduce"};
+
+cudaEvent_t prof_event() {
+  if (!g_prof_free.empty()) {
+    cudaEvent_t e = g_prof_free.back();
+    g_prof_free.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
 }  // namespace
 
+namespace nf4 {
+void prof_mark(cudaStream_t stream, int kernel_id, bool after) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (!g_prof_on) return;
+  if (!after) {
+    g_prof_open.start = prof_event();
+    g_prof_open.id = kernel_id;
+    if (g_prof_open.start) cudaEventRecord(g_prof_open.start, stream);
+  } else if (g_prof_open.start != nullptr && g_prof_open.id == kernel_id) {
+    g_prof_open.stop = prof_event();
+    if (g_prof_open.stop) {
+      cudaEventRecord(g_prof_open.stop, stream);
+      g_prof_pending.push_back(g_prof_open);
+    }
+    g_prof_open = ProfRecord{nullptr, nullptr, -1};
+  }
+}
+}  // namespace nf4
+
 extern "C" {
+
+nf4_status nf4_profile_begin(void) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  for (int i = 0; i < nf4::kNumKernelIds; ++i) {
+    g_prof_count[i] = 0;
+    g_prof_ms[i] = 0.0;
+  }
+  g_prof_on = true;
+  return NF4_OK;
+}
+
+nf4_status nf4_profile_end(void) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  g_prof_on = false;
+  nf4_status st = NF4_OK;
+  for (const ProfRecord& r : g_prof_pending) {
+    float ms = 0.0f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+      st = NF4_ERR_CUDA;
+    } else {
+      g_prof_count[r.id] += 1;
+      g_prof_ms[r.id] += ms;
+    }
+    g_prof_free.push_back(r.start);
+    g_prof_free.push_back(r.stop);
+  }
+  g_prof_pending.clear();
+  return st;
+}
+
+int nf4_profile_kernel_count(void) { return nf4::kNumKernelIds; }
+
+const char* nf4_kernel_name(int kernel_id) {
+  if (kernel_id < 0 || kernel_id >= nf4::kNumKernelIds) return "unknown";
+  return kKernelNames[kernel_id];
+}
+
+nf4_status nf4_profile_get(int kernel_id, int64_t* launches, double* total_ms) {
+  if (kernel_id < 0 || kernel_id >= nf4::kNumKernelIds) return NF4_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (launches) *launches = g_prof_count[kernel_id];
+  if (total_ms) *total_ms = g_prof_ms[kernel_id];
+  return NF4_OK;
+}
 
 const char* nf4_status_string(int status) {
   switch (status) {

@@ -48,3 +48,27 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t stream,
 cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 
 }  // namespace nf4
+
+// ---- per-kernel event profiling (api.cu) ----
+namespace nf4 {
+
+enum KernelId {
+  kKQuantize = 0,
+  kKDoubleQuant,
+  kKDequantize,
+  kKAdapterGemm,
+  kKAdapterFinalize,
+  kKFusedFwd,
+  kKFusedDx,
+  kKGemv,
+  kKGemvReduce,
+  kNumKernelIds
+};
+
+// When profiling is on, record an event on `stream` before / after a launch.
+void prof_mark(cudaStream_t stream, int kernel_id, bool after);
+
+}  // namespace nf4
+
+#define NF4_PROF_BEGIN(st, id) ::nf4::prof_mark((st), (id), false)
+#define NF4_PROF_END(st, id) ::nf4::prof_mark((st), (id), true)

@@ -671,14 +671,18 @@ cudaError_t run_adapter(const AdapterJob& j, float* part, uint32_t* status, int 
   p.part = part;
   p.status = status;
   const size_t smem = kAdStages * (kAdABytes + size_t(NP) * 128) + 1024 + 256;
+  NF4_PROF_BEGIN(st, kKAdapterGemm);
   adapter_gemm<<<dim3(sp.tiles, sp.slices), kAdThreads, smem, st>>>(ma, mb, p);
+  NF4_PROF_END(st, kKAdapterGemm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ++*launches;
   const int64_t total = j.Mo * j.r;
   const int grid = int(std::min<int64_t>(cdiv(total, 256), int64_t(sms) * 8));
+  NF4_PROF_BEGIN(st, kKAdapterFinalize);
   adapter_finalize<<<std::max(grid, 1), 256, 0, st>>>(part, sp.slices, int(j.Mo), NP, j.r, j.kind,
                                                       j.scale, j.out_bf16, j.out_f32);
+  NF4_PROF_END(st, kKAdapterFinalize);
   e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;
@@ -756,7 +760,9 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   if (!ok) return cudaErrorInvalidValue;
   const FusedParams p = fused_params(a, kFwd);
   dim3 grid(unsigned(cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kTileM)));
+  NF4_PROF_BEGIN(st, kKFusedFwd);
   fused_nf4_gemm<kFwd><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+  NF4_PROF_END(st, kKFusedFwd);
   e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;
@@ -813,7 +819,9 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
   if (!ok) return cudaErrorInvalidValue;
   const FusedParams p = fused_params(a, kDx);
   dim3 grid(unsigned(cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kTileM)));
+  NF4_PROF_BEGIN(st, kKFusedDx);
   fused_nf4_gemm<kDx><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+  NF4_PROF_END(st, kKFusedDx);
   e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;

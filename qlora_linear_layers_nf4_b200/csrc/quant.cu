@@ -222,6 +222,7 @@ cudaError_t launch_quantize(const float* w, int64_t numel, int bs, uint8_t* code
                             cudaStream_t stream, int* launches) {
   const int threads = 256;
   const bool vec = (bs % 8 == 0) && bs <= 256 && log2_exact(bs) >= 0;
+  NF4_PROF_BEGIN(stream, kKQuantize);
   if (vec) {
     const int64_t n_words = numel / 8;
     const int grid = grid_for(n_words, threads, sms, 8);
@@ -241,6 +242,7 @@ cudaError_t launch_quantize(const float* w, int64_t numel, int bs, uint8_t* code
     quantize_generic_kernel<<<grid, threads, 0, stream>>>(w, n_blocks, bs, codes, absmax_out,
                                                           status, gmax);
   }
+  NF4_PROF_END(stream, kKQuantize);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;
@@ -251,8 +253,10 @@ cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uin
                                 cudaStream_t stream, int* launches) {
   const int threads = 256;
   const int grid = grid_for(n_blocks, threads, sms, 4);
+  NF4_PROF_BEGIN(stream, kKDoubleQuant);
   double_quant_kernel<<<grid, threads, 0, stream>>>(absmax, n_blocks, gmax, absmax_q,
                                                     absmax_scale);
+  NF4_PROF_END(stream, kKDoubleQuant);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;
@@ -272,6 +276,7 @@ cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int
   dequant_kernel<T, D><<<grid, threads, 0, stream>>>(c, n_words, shift, bs_words, w.absmax, \
                                                      w.absmax_q, w.absmax_scale,            \
                                                      reinterpret_cast<T*>(out))
+  NF4_PROF_BEGIN(stream, kKDequantize);
   if (out_dtype == NF4_F32) {
     if (dq) NF4_DQ_LAUNCH(float, true); else NF4_DQ_LAUNCH(float, false);
   } else if (out_dtype == NF4_BF16) {
@@ -280,6 +285,7 @@ cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int
     if (dq) NF4_DQ_LAUNCH(__half, true); else NF4_DQ_LAUNCH(__half, false);
   }
 #undef NF4_DQ_LAUNCH
+  NF4_PROF_END(stream, kKDequantize);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;

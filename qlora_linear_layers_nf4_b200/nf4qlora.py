@@ -25,8 +25,9 @@ OP_QUANTIZE, OP_DEQUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD = 0, 1, 2, 3
 
 EXPORTED = (
     "nf4_status_string", "nf4_version", "nf4_codebook", "nf4_launch_count",
-    "nf4_workspace_bytes", "nf4_read_status", "nf4_quantize", "nf4_dequantize",
-    "qlora_linear_fwd", "qlora_linear_bwd",
+    "nf4_profile_begin", "nf4_profile_end", "nf4_profile_kernel_count", "nf4_kernel_name",
+    "nf4_profile_get", "nf4_workspace_bytes", "nf4_read_status", "nf4_quantize",
+    "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
 )
 
 
@@ -71,6 +72,13 @@ def lib() -> ctypes.CDLL:
     L.nf4_codebook.argtypes = [vp, vp]
     L.nf4_codebook.restype = None
     L.nf4_launch_count.restype = i64
+    L.nf4_profile_begin.restype = i32
+    L.nf4_profile_end.restype = i32
+    L.nf4_profile_kernel_count.restype = i32
+    L.nf4_kernel_name.argtypes = [i32]
+    L.nf4_kernel_name.restype = ctypes.c_char_p
+    L.nf4_profile_get.argtypes = [i32, ctypes.POINTER(i64), ctypes.POINTER(ctypes.c_double)]
+    L.nf4_profile_get.restype = i32
     L.nf4_workspace_bytes.argtypes = [i32, i64, i64, i64, i32, i32, i32]
     L.nf4_workspace_bytes.restype = sz
     L.nf4_read_status.argtypes = [vp, vp]
@@ -114,6 +122,24 @@ def codebook():
 
 def launch_count() -> int:
     return int(lib().nf4_launch_count())
+
+
+def profile_begin():
+    _check(lib().nf4_profile_begin(), "nf4_profile_begin")
+
+
+def profile_end() -> dict:
+    """Stop recording; {kernel name: (timed launches, total ms)} for kernels that ran."""
+    _check(lib().nf4_profile_end(), "nf4_profile_end")
+    out = {}
+    L = lib()
+    for i in range(L.nf4_profile_kernel_count()):
+        n = ctypes.c_int64()
+        ms = ctypes.c_double()
+        _check(L.nf4_profile_get(i, ctypes.byref(n), ctypes.byref(ms)), "nf4_profile_get")
+        if n.value:
+            out[L.nf4_kernel_name(i).decode()] = (int(n.value), float(ms.value))
+    return out
 
 
 def workspace_bytes(op: int, M: int, N: int, K: int, r: int, block_size: int, double_quant: bool) -> int:
