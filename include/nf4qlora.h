@@ -186,6 +186,30 @@ NF4_API nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int 
                         float* absmax_scale, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * nf4_quantize without a workspace, for callers that cannot allocate device
+ * memory at all: an engine plugin handed fixed buffers and no scratch
+ * allocator, an application whose own pool owns all device memory, a serving
+ * path that must not allocate after start-up.  The pages describe no such
+ * entry point; it exists for those callers.
+ * Arguments and results are those of nf4_quantize (same kernels, bit-identical
+ * output); the scratch that nf4_quantize keeps in `workspace` lives instead in
+ * a fixed device array inside the library, 4 MiB + 256 B, which every GPU
+ * that loads the library holds until the process exits.  With double_quant
+ * and absmax == NULL the block scales are kept there, so rows*cols/block_size
+ * may not exceed 1048576 (NF4_ERR_WORKSPACE otherwise); with a caller absmax
+ * buffer there is no size limit.  Calls no allocator (no cudaMalloc or
+ * cudaFree).  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and should come before any stream capture.  All
+ * calls share the array and it keeps the last call's contents (the global-max
+ * word is cleared at the start of each call); calls whose GPU work overlaps
+ * race.  Non-finite input is not reported (there is no status word to read).
+ */
+NF4_API nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t cols,
+                                        int block_size, int double_quant, uint8_t* codes,
+                                        float* absmax, uint8_t* absmax_q, float* absmax_scale,
+                                        void* stream);
+
+/*
  * Dequantization (qlora-rs dequantize_nf4; "Honor compute_dtype
  * (BF16/F16/F32) in forward dequant").  out[e] = fp32(L[code_e] * scale_b)
  * as one fp32 product; NF4_BF16 / NF4_F16 store its round-to-nearest-even.

@@ -27,7 +27,7 @@ EXPORTED = (
     "nf4_status_string", "nf4_version", "nf4_codebook", "nf4_launch_count",
     "nf4_profile_begin", "nf4_profile_end", "nf4_profile_kernel_count", "nf4_kernel_name",
     "nf4_profile_get", "nf4_workspace_bytes", "nf4_read_status", "nf4_quantize",
-    "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
+    "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "nf4_quantize_noalloc",
 )
 
 
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
     L.nf4_read_status.restype = i32
     L.nf4_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]
     L.nf4_quantize.restype = i32
+    L.nf4_quantize_noalloc.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp, vp]
+    L.nf4_quantize_noalloc.restype = i32
     L.nf4_dequantize.argtypes = [ctypes.POINTER(CWeight), i32, vp, vp]
     L.nf4_dequantize.restype = i32
     L.qlora_linear_fwd.argtypes = [ctypes.POINTER(CWeight), vp, i64, vp, vp, i32, f32, i32, vp, vp,
