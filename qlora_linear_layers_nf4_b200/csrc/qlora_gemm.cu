@@ -96,6 +96,21 @@ __device__ __forceinline__ void dequant_row(const uint8_t* codes, float scale, u
   }
 }
 
+// Half a block (32 elements, 16 code bytes at `codes`, smem) into 16-byte
+// chunks 4*half .. 4*half+3 of row `row` of a 128-byte-swizzled bf16 tile.
+__device__ __forceinline__ void dequant_half_row(const uint8_t* codes, float scale, uint8_t* tile,
+                                                 uint32_t row, uint32_t half) {
+  const uint4 c = *reinterpret_cast<const uint4*>(codes);
+  const BlockTable t = make_table(scale);
+  const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint2 a = decode4(words[k], t);
+    const uint2 b = decode4(words[k] >> 16, t);
+    *reinterpret_cast<uint4*>(tile + sw128_offset(row, 4 * half + k)) = make_uint4(a.x, a.y, b.x, b.y);
+  }
+}
+
 __device__ __forceinline__ float load_scale(const uint8_t* absmax_q, const float* absmax,
                                             float s_g, bool dq, int64_t idx) {
   return dq ? __fmul_rn(float(__ldg(absmax_q + idx)), s_g) : __ldg(absmax + idx);
@@ -305,7 +320,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const uint32_t ph = (it / kStages) & 1;
       const float scale = next_scale;
       if (it + 1 < p.main_steps) next_scale = scale_at(it + 1);
-      if (!mbar_wait(&sh->full[s], ph, abort_flag, p.status)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sh->full[s], ph, abort_flag, p.status))) break;
       dequant_row(stage_c(s) + t * 32, scale, stage_b(s), uint32_t(t));
       fence_proxy_async_smem();
       __syncwarp();
@@ -313,7 +328,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
 
     // ---------------- epilogue: TMEM -> registers -> bf16 -> global
-    const bool ok = mbar_wait(&sh->accum, 0, abort_flag, p.status);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&sh->accum, 0, abort_flag, p.status));
     tc_fence_after();
     if (ok) {
       const int quad = warp & 3;                     // TMEM lanes 32*quad .. +31
@@ -357,6 +372,280 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ pair-CTA fused GEMM
+//
+// The same product on a cluster of two CTAs issuing tcgen05 cta_group::2
+// MMAs (M = 256 rows per MMA, half from each CTA).  A pair tile is 512 x 256:
+// two M = 256 accumulators of 256 columns fill each CTA's TMEM, and each CTA
+// dequantizes only its 128-row half of the W' tile per K step, so every
+// dequantized element feeds twice the MMA work of the single-CTA kernel and
+// each CTA reads half the B operand from shared memory.
+//   rank r of the pair: A rows m0 + 256 h + 128 r (h = 0, 1) and W' half
+//   n0 + 128 r; the leader (rank 0) issues the MMAs, both CTAs' A loads
+//   complete on the leader's barrier, the leader's commits multicast to both.
+
+constexpr int kP2Stages = 4;
+constexpr int kP2DeqWarps = 8;                          // 2 threads per W' row
+constexpr int kP2Threads = 64 + kP2DeqWarps * 32;
+constexpr uint32_t kP2ABytes = 2 * kHalfABytes;        // two 128-row A blocks
+constexpr uint32_t kP2BBytes = 128 * 128;              // this CTA's 128 W' rows
+constexpr uint32_t kP2CBytes = 128 * 32;               // their codes
+constexpr uint32_t kP2StageBytes = kP2ABytes + kP2BBytes + kP2CBytes;
+constexpr size_t kP2Smem = size_t(kP2Stages) * kP2StageBytes + 1024 + 256;
+constexpr int kP2TileM = 512;
+
+struct PairShared {
+  uint64_t afull[kP2Stages];   // leader: A (+ adapter B) bytes of both CTAs landed
+  uint64_t cfull[kP2Stages];   // each CTA: its code tile landed
+  uint64_t bready[kP2Stages];  // leader: both CTAs' W' halves written (16 warp arrivals)
+  uint64_t empty[kP2Stages];   // each CTA: the MMAs reading the stage finished
+  uint64_t accum;
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
+    fused_nf4_gemm_pair(const __grid_constant__ CUtensorMap tm_a,
+                        const __grid_constant__ CUtensorMap tm_a2,
+                        const __grid_constant__ CUtensorMap tm_b2,
+                        const __grid_constant__ CUtensorMap tm_codes, const FusedParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  PairShared* sh = reinterpret_cast<PairShared*>(smem + kP2Stages * kP2StageBytes);
+  auto stage_a = [&](int s) { return smem + s * kP2StageBytes; };
+  auto stage_b = [&](int s) { return smem + s * kP2StageBytes + kP2ABytes; };
+  auto stage_c = [&](int s) { return smem + s * kP2StageBytes + kP2ABytes + kP2BBytes; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int tile_n0 = (blockIdx.x >> 1) * kTileN;     // fwd: W rows; dx: output cols
+  const int my_n0 = tile_n0 + 128 * int(rank);        // this CTA's half of the tile
+  const int m0 = blockIdx.y * kP2TileM;
+  const int total_steps = p.main_steps + p.adapter_steps;
+  volatile uint32_t* abort_flag = &sh->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kP2Stages; ++s) {
+      mbar_init(&sh->afull[s], 1);
+      mbar_init(&sh->cfull[s], 1);
+      // leader: its own 8 dequant warps + one forwarded arrival from the peer
+      mbar_init(&sh->bready[s], rank == 0 ? kP2DeqWarps + 1 : kP2DeqWarps);
+      mbar_init(&sh->empty[s], 1);
+    }
+    mbar_init(&sh->accum, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    tma_prefetch(&tm_a);
+    tma_prefetch(&tm_a2);
+    tma_prefetch(&tm_b2);
+    tma_prefetch(&tm_codes);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sh->tmem_base, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < total_steps; ++it) {
+        const int s = it % kP2Stages;
+        const uint32_t ph = (it / kP2Stages) & 1;
+        if (!mbar_wait_cluster(&sh->empty[s], ph ^ 1, abort_flag, p.status)) break;
+        const uint32_t afull_leader = mapa_shared(smem_u32(&sh->afull[s]), 0);
+        uint8_t* a = stage_a(s);
+        if (it < p.main_steps) {
+          if (rank == 0) mbar_arrive_expect_tx(&sh->afull[s], 2 * kP2ABytes);
+          mbar_arrive_expect_tx(&sh->cfull[s], kP2CBytes);
+          const int k0 = it * kTileK;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d_pair(a + h * kHalfABytes, &tm_a, afull_leader, k0, m0 + 256 * h + 128 * int(rank));
+          if (MODE == kFwd) {
+            tma_load_2d(stage_c(s), &tm_codes, &sh->cfull[s], k0 / 2, my_n0);
+          } else {
+#pragma unroll
+            for (int g = 0; g < 2; ++g)
+              tma_load_2d(stage_c(s) + g * 2048, &tm_codes, &sh->cfull[s], (my_n0 + 64 * g) / 2, k0);
+          }
+        } else {
+          const int r0 = (it - p.main_steps) * kTileK;
+          if (rank == 0) mbar_arrive_expect_tx(&sh->afull[s], 2 * (kP2ABytes + kP2BBytes));
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d_pair(a + h * kHalfABytes, &tm_a2, afull_leader, r0, m0 + 256 * h + 128 * int(rank));
+          if (MODE == kFwd) {
+            tma_load_2d_pair(stage_b(s), &tm_b2, afull_leader, r0, my_n0);
+          } else {
+#pragma unroll
+            for (int g = 0; g < 2; ++g)
+              tma_load_2d_pair(stage_b(s) + g * 8192, &tm_b2, afull_leader, my_n0 + 64 * g, r0);
+          }
+        }
+        ++issued;
+      }
+      if (*abort_flag) {
+        // Unwind: wait (bounded) for this CTA's code copies still in flight.
+        for (int it = issued - 1; it >= 0 && it >= issued - kP2Stages; --it) {
+          if (it >= p.main_steps) continue;
+          uint32_t dummy_abort = 0;
+          mbar_wait(&sh->cfull[it % kP2Stages], (it / kP2Stages) & 1, &dummy_abort, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- peer CTA: forward "W' half written" to the leader, one
+    // cluster-scope arrival per step (the dequant warps arrive locally).
+    if (lane == 0 && rank == 1) {
+      const uint32_t leader_bready0 = mapa_shared(smem_u32(&sh->bready[0]), 0);
+      for (int it = 0; it < p.main_steps; ++it) {
+        const int s = it % kP2Stages;
+        const uint32_t ph = (it / kP2Stages) & 1;
+        if (!mbar_wait(&sh->bready[s], ph, abort_flag, p.status)) break;
+        mbar_arrive_cluster(leader_bready0 + uint32_t(s) * uint32_t(sizeof(uint64_t)));
+      }
+    }
+    // ---------------- MMA issuer (leader CTA only)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(256, kTileN, false, MODE == kDx);
+      bool ok = true;
+      for (int it = 0; it < total_steps && ok; ++it) {
+        const int s = it % kP2Stages;
+        const uint32_t ph = (it / kP2Stages) & 1;
+        const bool adapter = it >= p.main_steps;
+        ok = mbar_wait_cluster(&sh->afull[s], ph, abort_flag, p.status);
+        if (ok && !adapter) ok = mbar_wait_cluster(&sh->bready[s], ph, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(stage_a(s));
+        const uint32_t b_base = smem_u32(stage_b(s));
+        int ksub = 4;
+        if (adapter) {
+          const int left = p.r - (it - p.main_steps) * kTileK;
+          ksub = left >= 64 ? 4 : (left + 15) / 16;
+        }
+        for (int kk = 0; kk < ksub; ++kk) {
+          const uint64_t bdesc = (MODE == kFwd) ? smem_desc_sw128(b_base + kk * 32, 16, 1024)
+                                                : smem_desc_sw128(b_base + kk * 2048, 8192, 1024);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint64_t adesc = smem_desc_sw128(a_base + h * kHalfABytes + kk * 32, 16, 1024);
+            umma_f16_pair(tmem + h * kTileN, adesc, bdesc, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit_pair_mc(&sh->empty[s], 0x3);
+      }
+      if (ok) {
+        umma_commit_pair_mc(&sh->accum, 0x3);
+      } else {
+        umma_commit_pair_mc(&sh->drain, 0x1);
+        uint32_t dummy_abort = 0;
+        mbar_wait_cluster(&sh->drain, 0, &dummy_abort, nullptr);
+      }
+    }
+  } else {
+    // ---------------- dequant warps: thread pair per W' row (one NF4 block)
+    const int t = threadIdx.x - 64;                   // 0..255
+    const int row = t >> 1;                           // 0..127 tile row
+    const uint32_t half = uint32_t(t & 1);
+    const bool dq = p.double_quant != 0;
+    const float s_g = dq ? __ldg(p.absmax_scale) : 0.0f;
+    int64_t w_row;
+    int block_col0, row_step;
+    if (MODE == kFwd) {
+      w_row = int64_t(my_n0) + row;
+      block_col0 = 0;
+      row_step = 0;
+    } else {
+      w_row = row & 63;
+      block_col0 = my_n0 / 64 + (row >> 6);
+      row_step = 64;
+    }
+    auto scale_at = [&](int it) -> float {
+      const int64_t wr = w_row + int64_t(row_step) * it;
+      if (wr >= p.N) return 0.0f;
+      const int bcol = (MODE == kFwd) ? it : block_col0;
+      if (MODE == kDx && bcol >= p.kb_per_row) return 0.0f;
+      return load_scale(p.absmax_q, p.absmax, s_g, dq, wr * p.kb_per_row + bcol);
+    };
+    // scales of the next four steps in flight (a small register ring)
+    float sc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sc[j] = j < p.main_steps ? scale_at(j) : 0.0f;
+    for (int it = 0; it < p.main_steps; ++it) {
+      const int s = it % kP2Stages;
+      const uint32_t ph = (it / kP2Stages) & 1;
+      const float scale = sc[0];
+      sc[0] = sc[1];
+      sc[1] = sc[2];
+      sc[2] = sc[3];
+      sc[3] = (it + 4 < p.main_steps) ? scale_at(it + 4) : 0.0f;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sh->cfull[s], ph, abort_flag, p.status))) break;
+      dequant_half_row(stage_c(s) + row * 32 + half * 16, scale, stage_b(s), uint32_t(row), half);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->bready[s]);
+    }
+
+    // ---------------- epilogue: this CTA's 128 rows of both accumulators
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_cluster(&sh->accum, 0, abort_flag, p.status));
+    tc_fence_after();
+    if (ok) {
+      const int quad = warp & 3;
+      const int h = (warp - 2) >> 2;
+      const int grow = m0 + 256 * h + 128 * int(rank) + quad * 32 + lane;
+      for (int c = 0; c < kTileN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + h * kTileN + c * 32, v);
+        tmem_ld_wait();
+        const int col0 = tile_n0 + c * 32;
+        if (grow < p.M) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int col = col0 + 8 * g;
+            if (col < p.out_cols) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
+              if (MODE == kFwd && p.bias != nullptr) {
+                const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
+                const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 bf = __bfloat1622float2(b2[e]);
+                  f[2 * e] += bf.x;
+                  f[2 * e + 1] += bf.y;
+                }
+              }
+              const uint4 o = make_uint4(bf16x2_rn(f[0], f[1]), bf16x2_rn(f[2], f[3]),
+                                         bf16x2_rn(f[4], f[5]), bf16x2_rn(f[6], f[7]));
+              *reinterpret_cast<uint4*>(p.out + int64_t(grow) * p.out_cols + col) = o;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -492,7 +781,7 @@ __global__ void __launch_bounds__(kAdThreads, 1)
     }
   } else {
     // epilogue warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1
-    const bool ok = mbar_wait(&sh->accum, 0, abort_flag, p.status);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&sh->accum, 0, abort_flag, p.status));
     tc_fence_after();
     const int quad = warp & 3;
     const int row = mo0 + quad * 32 + lane;
@@ -631,6 +920,12 @@ cudaError_t set_attrs() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(fused_nf4_gemm<kDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(kFusedSmem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fused_nf4_gemm_pair<kFwd>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kP2Smem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fused_nf4_gemm_pair<kDx>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kP2Smem));
   const size_t ad_smem = kAdStages * (kAdABytes + 256 * 128) + 1024 + 256;
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(adapter_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, int(ad_smem));
@@ -687,6 +982,9 @@ cudaError_t run_adapter(const AdapterJob& j, float* part, uint32_t* status, int 
   if (e == cudaSuccess) ++*launches;
   return e;
 }
+
+// Pair-CTA tiles (512 rows) once M fills them; single-CTA 256-row tiles below.
+bool use_pair(int64_t M) { return M > 256; }
 
 FusedParams fused_params(const LinearArgs& a, int mode) {
   FusedParams p;
@@ -752,16 +1050,23 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   e = forward_adapter_T(a, T, part, sms, st, launches);
   if (e != cudaSuccess) return e;
 
+  const bool pair = use_pair(a.M);
+  const uint32_t brows = pair ? 128 : 256;     // W' rows per CTA
   CUtensorMap ta, ta2, tb2, tc;
   bool ok = make_map(&ta, a.x, true, a.K, a.M, 64, 128, true);
   ok = ok && make_map(&ta2, T, true, a.r, a.M, 64, 128, true);
-  ok = ok && make_map(&tb2, a.B, true, a.r, a.N, 64, 256, true);
-  ok = ok && make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, 256, false);
+  ok = ok && make_map(&tb2, a.B, true, a.r, a.N, 64, brows, true);
+  ok = ok && make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, brows, false);
   if (!ok) return cudaErrorInvalidValue;
   const FusedParams p = fused_params(a, kFwd);
-  dim3 grid(unsigned(cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kTileM)));
   NF4_PROF_BEGIN(st, kKFusedFwd);
-  fused_nf4_gemm<kFwd><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+  if (pair) {
+    dim3 grid(unsigned(2 * cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kP2TileM)));
+    fused_nf4_gemm_pair<kFwd><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, p);
+  } else {
+    dim3 grid(unsigned(cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kTileM)));
+    fused_nf4_gemm<kFwd><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+  }
   NF4_PROF_END(st, kKFusedFwd);
   e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
@@ -818,9 +1123,14 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
   ok = ok && make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, 64, false);
   if (!ok) return cudaErrorInvalidValue;
   const FusedParams p = fused_params(a, kDx);
-  dim3 grid(unsigned(cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kTileM)));
   NF4_PROF_BEGIN(st, kKFusedDx);
-  fused_nf4_gemm<kDx><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+  if (use_pair(a.M)) {
+    dim3 grid(unsigned(2 * cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kP2TileM)));
+    fused_nf4_gemm_pair<kDx><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, p);
+  } else {
+    dim3 grid(unsigned(cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kTileM)));
+    fused_nf4_gemm<kDx><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+  }
   NF4_PROF_END(st, kKFusedDx);
   e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
