@@ -16,7 +16,7 @@
 //   fused_nf4_gemm<kDx>   dx[M,K] = dy W' + U A                 MN-major W' tiles
 //   adapter_gemm          the rank-r products T, U, dB, dA^T, split along the
 //                         reduction with fp32 partials
-//   adapter_finalize      sums the partials, scales/rounds/transposes
+//                         (the last CTA of each tile adds the slices in order)
 #include <algorithm>
 
 #include <cuda.h>
@@ -653,7 +653,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
 //
 // D[Mo, NP] = sum over a reduction range of A[Mo, red] * B[NP, red], one
 // 128-row tile per CTA and one slice of the reduction per blockIdx.y; fp32
-// partials land in part[slice][Mo][NP].  Operands come by TMA in 64-deep
+// the slices of a tile form one thread-block cluster and are summed through
+// distributed shared memory.  Operands come by TMA in 64-deep
 // steps, each either K-major (rows of the reduction) or MN-major.
 
 constexpr int kAdStages = 4;
@@ -663,13 +664,35 @@ constexpr uint32_t kAdABytes = 128 * 128;
 struct AdapterParams {
   int Mo;            // output rows
   int NP;            // output cols (r rounded up to 64)
+  int r;             // output cols kept
   int red_steps;     // ceil(reduction / 64)
   int steps_per_slice;
+  int slices;
   int a_mn;          // A operand MN-major
   int b_mn;          // B operand MN-major
-  float* part;       // [slices][Mo][NP]
+  int kind;          // 0: bf16(scale * D) [Mo][r]; 1: fp32 D [Mo][r]; 2: fp32 D^T [r][Mo]
+  float scale;
+  __nv_bfloat16* out_bf16;
+  float* out_f32;
   uint32_t* status;
 };
+
+// Write 4 consecutive output columns (col .. col+3 < r) of one row.
+__device__ __forceinline__ void adapter_store4(const AdapterParams& p, int row, int col, float4 v) {
+  if (p.kind == 0) {
+    const uint2 o = make_uint2(bf16x2_rn(v.x * p.scale, v.y * p.scale),
+                               bf16x2_rn(v.z * p.scale, v.w * p.scale));
+    *reinterpret_cast<uint2*>(p.out_bf16 + int64_t(row) * p.r + col) = o;
+  } else if (p.kind == 1) {
+    *reinterpret_cast<float4*>(p.out_f32 + int64_t(row) * p.r + col) = v;
+  } else {
+    float* o = p.out_f32 + int64_t(col) * p.Mo + row;
+    o[0] = v.x;
+    o[int64_t(p.Mo)] = v.y;
+    o[2 * int64_t(p.Mo)] = v.z;
+    o[3 * int64_t(p.Mo)] = v.w;
+  }
+}
 
 struct AdapterShared {
   uint64_t full[kAdStages];
@@ -780,69 +803,80 @@ __global__ void __launch_bounds__(kAdThreads, 1)
       }
     }
   } else {
-    // epilogue warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1
+    // epilogue warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1: with one slice
+    // the result goes straight out, otherwise this slice's fp32 partial.
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&sh->accum, 0, abort_flag, p.status));
     tc_fence_after();
     const int quad = warp & 3;
     const int row = mo0 + quad * 32 + lane;
-    float* dst = p.part + (int64_t(blockIdx.y) * p.Mo + row) * p.NP;
+    // partial tile [128][NP] fp32 over the (now idle) stage buffers
+    float* dst = reinterpret_cast<float*>(smem) + (quad * 32 + lane) * p.NP;
     for (int c = 0; c < p.NP / 32; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + c * 32, v);
       tmem_ld_wait();
       if (row < p.Mo) {
-        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
-          float4 f;
-          if (ok && nsteps > 0) {
+          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (ok && nsteps > 0)
             f = make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
                             __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+          const int col = c * 32 + 4 * g;
+          if (p.slices == 1) {
+            if (col < p.r) adapter_store4(p, row, col, f);
           } else {
-            f = make_float4(0.f, 0.f, 0.f, 0.f);
+            reinterpret_cast<float4*>(dst + col)[0] = f;
           }
-          d4[g] = f;
         }
+      } else if (p.slices > 1) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          reinterpret_cast<float4*>(dst + c * 32 + 4 * g)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (p.slices > 1) {
+    // The slices of this tile are the CTAs of one cluster (along y).  After
+    // all partials are in shared memory, CTA q sums rows [q*128/S, (q+1)*128/S)
+    // over the cluster's partials in slice order (deterministic) and writes
+    // them out; a second cluster barrier keeps every partial alive until read.
+    cluster_sync();
+    const uint32_t q = cluster_ctarank();
+    const int rows_per = 128 / p.slices;
+    const int vec_per_row = p.r / 4;
+    const int total = rows_per * vec_per_row;
+    const uint32_t base = smem_u32(smem);
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+      int rr, cv;
+      if (p.kind == 2) {            // consecutive threads -> consecutive rows (coalesced D^T)
+        cv = i / rows_per;
+        rr = i % rows_per;
+      } else {
+        rr = i / vec_per_row;
+        cv = i % vec_per_row;
+      }
+      const int trow = int(q) * rows_per + rr;
+      const uint32_t off = uint32_t((trow * p.NP + 4 * cv) * 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sl = 0; sl < p.slices; ++sl) {
+        const float4 v = ld_shared_cluster_f4(mapa_shared(base + off, uint32_t(sl)));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      const int row = mo0 + trow;
+      if (row < p.Mo) adapter_store4(p, row, 4 * cv, acc);
+    }
+    cluster_sync();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
-  }
-}
-
-// out = sum of the slices, for columns < r:
-//   kind 0: bf16(scale * sum) into out_bf16[Mo][r]
-//   kind 1: fp32 sum into out_f32[Mo][r]
-//   kind 2: fp32 sum transposed into out_f32[r][Mo]
-__global__ void __launch_bounds__(256) adapter_finalize(const float* __restrict__ part, int slices,
-                                                        int Mo, int NP, int r, int kind, float scale,
-                                                        __nv_bfloat16* __restrict__ out_bf16,
-                                                        float* __restrict__ out_f32) {
-  const int64_t total = int64_t(Mo) * r;
-  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-    int64_t row, col;
-    if (kind == 2) {        // walk the transposed output contiguously
-      col = i / Mo;
-      row = i % Mo;
-    } else {
-      row = i / r;
-      col = i % r;
-    }
-    float acc = 0.0f;
-    for (int s = 0; s < slices; ++s) acc += part[(int64_t(s) * Mo + row) * NP + col];
-    if (kind == 0) {
-      out_bf16[row * r + col] = __float2bfloat16_rn(acc * scale);
-    } else if (kind == 1) {
-      out_f32[row * r + col] = acc;
-    } else {
-      out_f32[col * int64_t(Mo) + row] = acc;
-    }
   }
 }
 
@@ -897,19 +931,18 @@ SplitPlan plan_split(int64_t Mo, int64_t red) {
   SplitPlan sp;
   sp.tiles = int(cdiv(Mo, 128));
   const int steps = int(std::max<int64_t>(cdiv(red, 64), 1));
-  int want = int(cdiv(296, sp.tiles));
-  want = std::max(1, std::min(want, std::min(16, std::max(1, steps / 4))));
-  sp.per = int(cdiv(steps, want));
-  sp.slices = int(cdiv(steps, sp.per));
+  // one wave of 2 CTAs per SM; the slices of a tile form one cluster (<= 8)
+  const int cap = std::max(1, std::min(std::min(296 / sp.tiles, 8), std::max(1, steps / 4)));
+  int sl = 1;
+  while (sl * 2 <= cap) sl *= 2;
+  sp.slices = sl;
+  sp.per = int(cdiv(steps, sl));
   return sp;
 }
 
 int round_np(int r) { return int(cdiv(r, 64) * 64); }
 
-size_t part_bytes(int64_t Mo, int64_t red, int r) {
-  const SplitPlan sp = plan_split(Mo, red);
-  return align256(size_t(sp.slices) * size_t(Mo) * size_t(round_np(r)) * sizeof(float));
-}
+
 
 bool g_attr_done = false;
 
@@ -946,8 +979,8 @@ struct AdapterJob {
   float* out_f32;
 };
 
-cudaError_t run_adapter(const AdapterJob& j, float* part, uint32_t* status, int sms,
-                        cudaStream_t st, int* launches) {
+cudaError_t run_adapter(const AdapterJob& j, uint32_t* status, int sms, cudaStream_t st,
+                        int* launches) {
   const int NP = round_np(j.r);
   CUtensorMap ma, mb;
   bool ok = j.a_mn ? make_map(&ma, j.a, true, j.a_inner, j.a_outer, 64, 64, true)
@@ -959,26 +992,35 @@ cudaError_t run_adapter(const AdapterJob& j, float* part, uint32_t* status, int 
   AdapterParams p;
   p.Mo = int(j.Mo);
   p.NP = NP;
+  p.r = j.r;
   p.red_steps = int(std::max<int64_t>(cdiv(j.red, 64), 1));
   p.steps_per_slice = sp.per;
+  p.slices = sp.slices;
   p.a_mn = j.a_mn;
   p.b_mn = j.b_mn;
-  p.part = part;
+  p.kind = j.kind;
+  p.scale = j.scale;
+  p.out_bf16 = j.out_bf16;
+  p.out_f32 = j.out_f32;
   p.status = status;
+  (void)sms;
   const size_t smem = kAdStages * (kAdABytes + size_t(NP) * 128) + 1024 + 256;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(sp.tiles), unsigned(sp.slices), 1);
+  cfg.blockDim = dim3(kAdThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = unsigned(sp.slices);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   NF4_PROF_BEGIN(st, kKAdapterGemm);
-  adapter_gemm<<<dim3(sp.tiles, sp.slices), kAdThreads, smem, st>>>(ma, mb, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, adapter_gemm, ma, mb, p);
   NF4_PROF_END(st, kKAdapterGemm);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  ++*launches;
-  const int64_t total = j.Mo * j.r;
-  const int grid = int(std::min<int64_t>(cdiv(total, 256), int64_t(sms) * 8));
-  NF4_PROF_BEGIN(st, kKAdapterFinalize);
-  adapter_finalize<<<std::max(grid, 1), 256, 0, st>>>(part, sp.slices, int(j.Mo), NP, j.r, j.kind,
-                                                      j.scale, j.out_bf16, j.out_f32);
-  NF4_PROF_END(st, kKAdapterFinalize);
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;
 }
@@ -1006,38 +1048,26 @@ FusedParams fused_params(const LinearArgs& a, int mode) {
   return p;
 }
 
-// Workspace regions after the header (all 256-byte aligned):
-//   fwd: [T bf16 M x r (when t_out is null)] [partials]
-//   bwd: [T bf16 M x r (when t is null)] [U bf16 M x r] [partials]
+// Workspace regions after the header (256-byte aligned):
+//   fwd: [T bf16 M x r (when t_out is null)]
+//   bwd: [T bf16 M x r (when t is null)] [U bf16 M x r]
 size_t mr_bytes(int64_t M, int r) { return align256(size_t(M) * size_t(r) * 2); }
 
-size_t fwd_part_bytes(int64_t M, int64_t N, int64_t K, int r) {
-  (void)N;
-  return part_bytes(M, K, r);
-}
-
-size_t bwd_part_bytes(int64_t M, int64_t N, int64_t K, int r) {
-  size_t b = part_bytes(M, K, r);                 // T recompute
-  b = std::max(b, part_bytes(M, N, r));           // U
-  b = std::max(b, part_bytes(N, M, r));           // dB
-  b = std::max(b, part_bytes(K, M, r));           // dA^T
-  return b;
-}
-
-cudaError_t forward_adapter_T(const LinearArgs& a, __nv_bfloat16* T, float* part, int sms,
-                              cudaStream_t st, int* launches) {
+cudaError_t forward_adapter_T(const LinearArgs& a, __nv_bfloat16* T, int sms, cudaStream_t st,
+                              int* launches) {
   AdapterJob j{};
   j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = false;
   j.b = a.A; j.b_inner = a.K; j.b_outer = a.r; j.b_mn = false;
   j.Mo = a.M; j.red = a.K; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = T;
-  return run_adapter(j, part, a.status, sms, st, launches);
+  return run_adapter(j, a.status, sms, st, launches);
 }
 
 }  // namespace
 
 size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, int r) {
-  if (!backward) return mr_bytes(M, r) + fwd_part_bytes(M, N, K, r);
-  return 2 * mr_bytes(M, r) + bwd_part_bytes(M, N, K, r);
+  (void)N;
+  (void)K;
+  return (backward ? 2 : 1) * mr_bytes(M, r);
 }
 
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches) {
@@ -1045,9 +1075,8 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   if (e != cudaSuccess) return e;
   uint8_t* ws = a.ws + kWsHeader;
   __nv_bfloat16* T = a.t_out ? static_cast<__nv_bfloat16*>(a.t_out) : reinterpret_cast<__nv_bfloat16*>(ws);
-  float* part = reinterpret_cast<float*>(ws + mr_bytes(a.M, a.r));
 
-  e = forward_adapter_T(a, T, part, sms, st, launches);
+  e = forward_adapter_T(a, T, sms, st, launches);
   if (e != cudaSuccess) return e;
 
   const bool pair = use_pair(a.M);
@@ -1079,11 +1108,10 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
   uint8_t* ws = a.ws + kWsHeader;
   __nv_bfloat16* T_ws = reinterpret_cast<__nv_bfloat16*>(ws);
   __nv_bfloat16* U = reinterpret_cast<__nv_bfloat16*>(ws + mr_bytes(a.M, a.r));
-  float* part = reinterpret_cast<float*>(ws + 2 * mr_bytes(a.M, a.r));
 
   const __nv_bfloat16* T = static_cast<const __nv_bfloat16*>(a.t_in);
   if (T == nullptr) {
-    e = forward_adapter_T(a, T_ws, part, sms, st, launches);
+    e = forward_adapter_T(a, T_ws, sms, st, launches);
     if (e != cudaSuccess) return e;
     T = T_ws;
   }
@@ -1093,7 +1121,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = false;
     j.b = a.B; j.b_inner = a.r; j.b_outer = a.N; j.b_mn = true;
     j.Mo = a.M; j.red = a.N; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = U;
-    e = run_adapter(j, part, a.status, sms, st, launches);
+    e = run_adapter(j, a.status, sms, st, launches);
     if (e != cudaSuccess) return e;
   }
   // dB = dy^T T   (A: dy^T MN-major over m; B: T [M, r] MN-major over m)
@@ -1102,7 +1130,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = true;
     j.b = T; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
     j.Mo = a.N; j.red = a.M; j.r = a.r; j.kind = 1; j.scale = 1.0f; j.out_f32 = a.dB;
-    e = run_adapter(j, part, a.status, sms, st, launches);
+    e = run_adapter(j, a.status, sms, st, launches);
     if (e != cudaSuccess) return e;
   }
   // dA^T = x^T U  (A: x^T MN-major over m; B: U [M, r] MN-major over m), stored as dA [r, K]
@@ -1111,7 +1139,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = true;
     j.b = U; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
     j.Mo = a.K; j.red = a.M; j.r = a.r; j.kind = 2; j.scale = 1.0f; j.out_f32 = a.dA;
-    e = run_adapter(j, part, a.status, sms, st, launches);
+    e = run_adapter(j, a.status, sms, st, launches);
     if (e != cudaSuccess) return e;
   }
   if (a.dx == nullptr) return cudaSuccess;
