@@ -367,67 +367,139 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
+def graph_time(calls, replays, warmup=2):
+    """GPU time per call of `calls` (a list of zero-argument launches), captured
+    into one CUDA graph and replayed `replays` times; host overhead is out."""
+    import torch
+    for _ in range(warmup):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in calls:
+            c()
+    g.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(replays):
+        g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / (replays * len(calls))
+    del g
+    return ms
+
+
 def measure_rows(args, dev, flush, pk, pk_kind, barrier):
-    """The other rows of the hot path, each timed on its own."""
+    """The other rows of the hot path.  Each is a short kernel, so it is timed
+    as CUDA-graph replays of calls on rotating buffers whose footprint exceeds
+    the 126 MB L2 (no flush needed, no host launch overhead)."""
+    import ctypes
     import numpy as np
     import torch
     from qlora_linear_layers_nf4_b200 import nf4qlora as Q
     from qlora_linear_layers_nf4_b200 import workloads as WL
 
+    L = Q.lib()
     hbm = pk.get("hbm_gbs")
     out = {}
-    reps = max(5, min(args.steps, 20))
+    stream = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
 
-    def mem_row(name, fn, nbytes, kernel_names):
-        Q.profile_begin()
-        ms = time_steps(fn, reps, 3, flush=flush, barrier=barrier)
-        k = Q.profile_end()
-        kms = sum(k.get(n, (0, 0.0))[1] for n in kernel_names)
-        kn = sum(k.get(n, (0, 0.0))[0] for n in kernel_names)
-        gbs = nbytes * reps / (ms * 1e-3) / 1e9
-        kgbs = nbytes * reps / (kms * 1e-3) / 1e9 if kms else None
-        out[name] = {"GB/s": gbs, "kernel_GB/s": kgbs, "frac_hbm": (kgbs / hbm) if kgbs else None,
-                     "us_per_call": 1e3 * ms / reps, "bytes": nbytes,
-                     "kernel_launches_per_call": kn / reps if reps else None}
+    def row(name, calls, nbytes, replays=20):
+        ms = graph_time(calls, replays)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"GB/s": gbs, "frac_hbm": gbs / hbm, "us_per_call": 1e3 * ms, "bytes": nbytes,
+                     "method": f"CUDA graph of {len(calls)} calls on rotating buffers, {replays} replays"}
 
-    w = torch.from_numpy(WL.draw_weight(WL.QUANT_SHAPE, WL.QUANT_SEED)).to(dev)
-    numel = w.numel()
-    nb = numel // 64
-    ws = Q.Workspace(dev)
-    q0 = Q.quantize(w, 64, False, workspace=ws)
-    q1 = Q.quantize(w, 64, True, workspace=ws)
-    mem_row("quantize_4096x4096_noDQ", lambda: Q.quantize(w, 64, False, workspace=ws),
-            numel * 4 + numel // 2 + nb * 4, ["nf4_quantize"])
-    mem_row("quantize_4096x4096_DQ", lambda: Q.quantize(w, 64, True, workspace=ws),
-            numel * 4 + numel // 2 + nb + 4, ["nf4_quantize", "nf4_double_quant"])
-    out32 = torch.empty((4096, 4096), dtype=torch.float32, device=dev)
-    for dq, qq in (("noDQ", q0), ("DQ", q1)):
-        sb = nb * 4 if dq == "noDQ" else nb + 4
-        for kind, esz in (("f32", 4), ("bf16", 2)):
-            mem_row(f"dequantize_{kind}_{dq}", lambda qq=qq, kind=kind: Q.dequantize(qq, kind),
-                    numel // 2 + sb + numel * esz, ["nf4_dequantize"])
-    del out32
+    # ---- quantize / dequantize of 4096x4096 (3 rotating matrices: 192 MiB fp32)
+    R = 3
+    ws = [Q.Workspace(dev) for _ in range(R)]
+    ws_bytes = Q.workspace_bytes(Q.OP_QUANTIZE, 0, 4096, 4096, 0, 64, True)
+    ws_bufs = [w.get(ws_bytes) for w in ws]
+    ws_s = [w.numel() for w in ws_bufs]
+    mats = [torch.from_numpy(WL.draw_weight(WL.QUANT_SHAPE, WL.QUANT_SEED + i)).to(dev) for i in range(R)]
+    numel, nb = 4096 * 4096, 4096 * 4096 // 64
+    codes = [torch.empty(numel // 2, dtype=torch.uint8, device=dev) for _ in range(R)]
+    amax = [torch.empty(nb, dtype=torch.float32, device=dev) for _ in range(R)]
+    aq = [torch.empty(nb, dtype=torch.uint8, device=dev) for _ in range(R)]
+    asc = [torch.empty(1, dtype=torch.float32, device=dev) for _ in range(R)]
 
-    # decode-shape forward (weight streaming)
+    def qcall(i, dq):
+        def f():
+            st = L.nf4_quantize(ptr(mats[i]), 4096, 4096, 64, int(dq), ptr(codes[i]),
+                                None if dq else ptr(amax[i]), ptr(aq[i]) if dq else None,
+                                ptr(asc[i]) if dq else None, ptr(ws_bufs[i]), ws_s[i], stream())
+            assert st == 0, st
+        return f
+
+    row("quantize_4096x4096_noDQ", [qcall(i, False) for i in range(R)], numel * 4 + numel // 2 + nb * 4)
+    row("quantize_4096x4096_DQ", [qcall(i, True) for i in range(R)], numel * 4 + numel // 2 + nb + 4)
+    # both forms of each weight now exist (codes[i] are identical for both)
+    for i in range(R):
+        qcall(i, False)()
+    torch.cuda.synchronize()
+    outs = {"f32": [torch.empty(numel, dtype=torch.float32, device=dev) for _ in range(R)],
+            "bf16": [torch.empty(numel, dtype=torch.bfloat16, device=dev) for _ in range(R)]}
+    kinds = {"f32": (Q.NF4_F32, 4), "bf16": (Q.NF4_BF16, 2)}
+
+    def dcall(i, dq, kind):
+        cw = Q.CWeight(codes=codes[i].data_ptr(), absmax=None if dq else amax[i].data_ptr(),
+                       absmax_q=aq[i].data_ptr() if dq else None,
+                       absmax_scale=asc[i].data_ptr() if dq else None, rows=4096, cols=4096,
+                       block_size=64, double_quant=int(dq))
+        def f():
+            st = L.nf4_dequantize(ctypes.byref(cw), kinds[kind][0], ptr(outs[kind][i]), stream())
+            assert st == 0, st
+        return f
+
+    for dq in (False, True):
+        if dq:
+            for i in range(R):
+                qcall(i, True)()
+        sb = nb * 4 if not dq else nb + 4
+        for kind in ("f32", "bf16"):
+            row(f"dequantize_{kind}_{'DQ' if dq else 'noDQ'}", [dcall(i, dq, kind) for i in range(R)],
+                numel // 2 + sb + numel * kinds[kind][1])
+    del mats, outs, codes, amax, aq, asc
+    torch.cuda.empty_cache()
+
+    # ---- decode forward: 16 rotating 4096x4096 NF4 weights (142 MB)
+    RD = 16
+    base = WL.DECODE[0]
+    qws = [Q.quantize(torch.from_numpy(WL.draw_weight((base.n, base.k), seed=200 + i)).to(dev), 64, True)
+           for i in range(RD)]
     for case in WL.DECODE:
         inp = WL.draw_linear(case)
-        qd = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True, workspace=ws)
         x, A, B = (bf16_dev(v, dev) for v in (inp.x, inp.a, inp.b))
         y = torch.empty((case.m, case.n), dtype=torch.bfloat16, device=dev)
         wsd = Q.Workspace(dev)
+        buf = wsd.get(Q.workspace_bytes(Q.OP_LINEAR_FWD, case.m, case.n, case.k, case.r, 64, True))
+        cws = [qq.c_struct() for qq in qws]
+
+        def fcall(cw):
+            def f():
+                st = L.qlora_linear_fwd(ctypes.byref(cw), ptr(x), case.m, ptr(A), ptr(B), case.r,
+                                        float(case.alpha), Q.NF4_BF16, None, ptr(y), None, ptr(buf),
+                                        buf.numel(), stream())
+                assert st == 0, st
+            return f
+
         nbytes = (case.n * case.k // 2 + case.n * case.k // 64 + 4 + 2 * case.r * case.k
                   + 2 * case.n * case.r + 2 * case.m * (case.k + case.n))
-        mem_row(f"decode_fwd_M{case.m}", lambda: Q.linear_fwd(qd, x, A, B, case.alpha, out=y,
-                                                               want_t=False, workspace=wsd),
-                nbytes, ["nf4_gemv", "nf4_gemv_reduce", "adapter_gemm", "adapter_finalize",
-                         "fused_nf4_gemm_fwd"])
+        row(f"decode_fwd_M{case.m}", [fcall(cw) for cw in cws], nbytes, replays=50)
+    del qws
+    torch.cuda.empty_cache()
 
-    # the seven targets of one decoder block, fwd + bwd each
+    # ---- the seven targets of one decoder block, fwd + bwd each (long kernels: eager)
     if not args.no_block:
+        ws_q = Q.Workspace(dev)
         layers = []
         for case in WL.BLOCK:
             inp = WL.draw_linear(case)
-            qb = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True, workspace=ws)
+            qb = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True, workspace=ws_q)
             x, A, B, dy = (bf16_dev(v, dev) for v in (inp.x, inp.a, inp.b, inp.dy))
             layers.append((case, qb, x, A, B, dy,
                            torch.empty((case.m, case.n), dtype=torch.bfloat16, device=dev),

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/nf4qlora.h"
@@ -44,6 +45,15 @@ struct LinearArgs {
 };
 
 size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, int r);
+
+// 2-D TMA map over a row-major matrix (`inner` elements per row, `outer`
+// rows; bf16 or u8), optional 128-byte swizzle.  False if it cannot be encoded.
+bool make_map_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+                 uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+
+// Decode-shape forward (gemv.cu): one kernel for M <= 32 tokens.
+bool decode_supported(int64_t M, int64_t N, int64_t K, int r);
+cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 

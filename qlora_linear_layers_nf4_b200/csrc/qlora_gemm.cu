@@ -1064,6 +1064,11 @@ cudaError_t forward_adapter_T(const LinearArgs& a, __nv_bfloat16* T, int sms, cu
 
 }  // namespace
 
+bool make_map_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+                 uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  return make_map(map, base, bf16, inner, outer, box_inner, box_outer, swizzle128);
+}
+
 size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, int r) {
   (void)N;
   (void)K;
@@ -1071,6 +1076,10 @@ size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, in
 }
 
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches) {
+  if (decode_supported(a.M, a.N, a.K, a.r)) {
+    const cudaError_t d = launch_decode_fwd(a, sms, st, launches);
+    if (d != cudaErrorNotSupported) return d;
+  }
   cudaError_t e = set_attrs();
   if (e != cudaSuccess) return e;
   uint8_t* ws = a.ws + kWsHeader;
