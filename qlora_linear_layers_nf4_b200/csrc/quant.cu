@@ -23,6 +23,65 @@ __device__ __forceinline__ bool finite8(const float4& a, const float4& b) {
          isfinite(b.y) && isfinite(b.z) && isfinite(b.w);
 }
 
+// Fast encode.  v = RN(w / a) is formed without a division: y = RN(1/a) once
+// per block (CUDA's correctly rounded reciprocal), q = RN(w y), then one
+// FMA-based correction q' = q + (w - a q) y.  That is Markstein's correction
+// step; with a correctly rounded reciprocal it yields the correctly rounded
+// quotient when nothing overflows or underflows, which the callers ensure by
+// keeping 2^-120 < a < 2^120 (other blocks take the division).
+//
+// The nearest level then comes from a 65-entry bucket table over [-1, 1]:
+// bucket i = floor(32 (v + 1)) holds base_i = #{thresholds below the bucket's
+// lower edge} and the one threshold inside it (or +inf); code = base_i +
+// (v > threshold_i).  No threshold lies within 0.0016 of a bucket edge, far
+// beyond the 2^-24 rounding of the bucket index, so an index that lands one
+// bucket off for v next to an edge still gives the same code.
+struct Bucket {
+  float thr;
+  uint32_t base;
+};
+
+__device__ __forceinline__ void init_buckets(Bucket* b) {
+  for (int i = threadIdx.x; i < 65; i += blockDim.x) {
+    const float lo = float(i) / 32.0f - 1.0f;           // exact
+    const float hi = lo + 1.0f / 32.0f;
+    uint32_t base = 0;
+    float thr = __int_as_float(0x7f800000);               // +inf
+#pragma unroll
+    for (int j = 0; j < 15; ++j) {
+      const float t = __uint_as_float(threshold_bits(j));
+      base += (t < lo) ? 1u : 0u;
+      if (t >= lo && t < hi) thr = t;
+    }
+    b[i].thr = thr;
+    b[i].base = base;
+  }
+}
+
+__device__ __forceinline__ uint32_t encode_bucket(float v, const Bucket* b) {
+  const float y = fmaf(v, 32.0f, 31.5f);
+  // Round to an integer in 0..64 for |v| <= 1; the min keeps a NaN (outside
+  // the contract, flagged by the absmax pass) inside the 65-entry table.
+  const uint32_t idx = min(__float_as_uint(__fadd_rn(y, 12582912.0f)) & 0x7fu, 64u);
+  const Bucket e = b[idx];
+  return e.base + (v > e.thr ? 1u : 0u);
+}
+
+__device__ __forceinline__ float div_corrected(float w, float a, float y) {
+  const float q = __fmul_rn(w, y);
+  return fmaf(fmaf(-a, q, w), y, q);
+}
+
+__device__ __forceinline__ bool fast_scale(float a) {
+  return a > 0x1p-120f && a < 0x1p120f;
+}
+
+// Codes of two elements packed as one byte, even element in the high nibble.
+__device__ __forceinline__ uint32_t pair_byte_fast(float w0, float w1, float a, float y,
+                                                   const Bucket* b) {
+  return (encode_bucket(div_corrected(w0, a, y), b) << 4) | encode_bucket(div_corrected(w1, a, y), b);
+}
+
 // Codes of two elements packed as one byte, even element in the high nibble.
 __device__ __forceinline__ uint32_t pair_byte(float w0, float w1, float amax) {
   if (amax == 0.0f) return 0x77u;
@@ -53,6 +112,11 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
     uint32_t* __restrict__ codes, float* __restrict__ absmax, uint32_t* __restrict__ status,
     uint32_t* __restrict__ gmax) {
   (void)blocks_per_row_unused;
+  // let a programmatic dependent (the double-quant kernel) start launching
+  asm volatile("griddepcontrol.launch_dependents;");
+  __shared__ Bucket buckets[65];
+  init_buckets(buckets);
+  __syncthreads();
   float cta_max = 0.0f;
   bool bad = false;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
@@ -70,8 +134,16 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
 #pragma unroll
     for (int o = G / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (valid) {
-      uint32_t word = pair_byte(a.x, a.y, m) | (pair_byte(a.z, a.w, m) << 8) |
-                      (pair_byte(b.x, b.y, m) << 16) | (pair_byte(b.z, b.w, m) << 24);
+      uint32_t word;
+      if (fast_scale(m)) {
+        const float y = __frcp_rn(m);
+        word = pair_byte_fast(a.x, a.y, m, y, buckets) | (pair_byte_fast(a.z, a.w, m, y, buckets) << 8) |
+               (pair_byte_fast(b.x, b.y, m, y, buckets) << 16) |
+               (pair_byte_fast(b.z, b.w, m, y, buckets) << 24);
+      } else {
+        word = pair_byte(a.x, a.y, m) | (pair_byte(a.z, a.w, m) << 8) |
+               (pair_byte(b.x, b.y, m) << 16) | (pair_byte(b.z, b.w, m) << 24);
+      }
       __stcs(codes + i, word);
       if ((threadIdx.x & (G - 1)) == 0 && absmax != nullptr) absmax[i / G] = m;
     }
@@ -85,6 +157,7 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
 __global__ void __launch_bounds__(256) quantize_generic_kernel(
     const float* __restrict__ w, int64_t n_blocks, int bs, uint8_t* __restrict__ codes,
     float* __restrict__ absmax, uint32_t* __restrict__ status, uint32_t* __restrict__ gmax) {
+  asm volatile("griddepcontrol.launch_dependents;");
   float cta_max = 0.0f;
   bool bad = false;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
@@ -110,17 +183,24 @@ __global__ void __launch_bounds__(256) quantize_generic_kernel(
 
 // Simplified double quant of the block scales: one global scale G / 255 and a
 // u8 per block, rint(absmax / s_g) with ties to even.
+// Launched as a programmatic dependent of the quantize kernel: it starts
+// early and waits (griddepcontrol.wait) until the quantize grid has finished
+// and its writes are visible.
 __global__ void __launch_bounds__(256) double_quant_kernel(
     const float* __restrict__ absmax, int64_t n_blocks, const uint32_t* __restrict__ gmax,
     uint8_t* __restrict__ absmax_q, float* __restrict__ absmax_scale) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const float g = __uint_as_float(*gmax);
   const float s_g = __fdiv_rn(g, 255.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *absmax_scale = s_g;
+  const bool fast = fast_scale(s_g);
+  const float y = fast ? __frcp_rn(s_g) : 0.0f;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n_blocks; i += stride) {
     uint32_t q = 0;
     if (g > 0.0f) {
-      const float ratio = __fdiv_rn(absmax[i], s_g);
+      const float a = absmax[i];
+      const float ratio = fast ? div_corrected(a, s_g, y) : __fdiv_rn(a, s_g);
       q = uint32_t(min(max(__float2int_rn(ratio), 0), 255));
     }
     absmax_q[i] = uint8_t(q);
@@ -168,10 +248,10 @@ struct Store8<__half> {
   }
 };
 
-// out[e] = fp32(L[code] * scale), one product per element; block_size % 8 == 0
-// so the 8 elements of one code word share a scale.
+// Four code words per thread per iteration, a grid-stride apart, so every
+// warp-wide load and store stays contiguous while four loads are in flight.
 template <typename OutT, bool kDouble>
-__global__ void __launch_bounds__(256) dequant_kernel(
+__global__ void __launch_bounds__(256) dequant_x4_kernel(
     const uint32_t* __restrict__ codes, int64_t n_words, int bs_words_shift, int bs_words,
     const float* __restrict__ absmax, const uint8_t* __restrict__ absmax_q,
     const float* __restrict__ absmax_scale, OutT* __restrict__ out) {
@@ -180,23 +260,32 @@ __global__ void __launch_bounds__(256) dequant_kernel(
   __syncthreads();
   const float s_g = kDouble ? *absmax_scale : 0.0f;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n_words; i += stride) {
-    const uint32_t word = __ldcs(codes + i);
-    const int64_t blk = bs_words_shift >= 0 ? (i >> bs_words_shift) : (i / bs_words);
-    float scale;
-    if (kDouble) {
-      scale = __fmul_rn(float(__ldg(absmax_q + blk)), s_g);
-    } else {
-      scale = __ldg(absmax + blk);
-    }
-    float v[8];
+  for (int64_t base = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; base < n_words;
+       base += 4 * stride) {
+    uint32_t words[4];
+    float scales[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t byte = (word >> (8 * j)) & 0xffu;
-      v[2 * j] = __fmul_rn(lut[byte >> 4], scale);
-      v[2 * j + 1] = __fmul_rn(lut[byte & 15u], scale);
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = base + u * stride;
+      words[u] = i < n_words ? __ldcs(codes + i) : 0u;
+      const int64_t blk = bs_words_shift >= 0 ? (i >> bs_words_shift) : (i / bs_words);
+      scales[u] = i < n_words ? (kDouble ? __fmul_rn(float(__ldg(absmax_q + blk)), s_g)
+                                         : __ldg(absmax + blk))
+                              : 0.0f;
     }
-    Store8<OutT>::run(out, i, v);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = base + u * stride;
+      if (i >= n_words) break;
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t byte = (words[u] >> (8 * j)) & 0xffu;
+        v[2 * j] = __fmul_rn(lut[byte >> 4], scales[u]);
+        v[2 * j + 1] = __fmul_rn(lut[byte & 15u], scales[u]);
+      }
+      Store8<OutT>::run(out, i, v);
+    }
   }
 }
 
@@ -253,11 +342,20 @@ cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uin
                                 cudaStream_t stream, int* launches) {
   const int threads = 256;
   const int grid = grid_for(n_blocks, threads, sms, 4);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid), 1, 1);
+  cfg.blockDim = dim3(unsigned(threads), 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   NF4_PROF_BEGIN(stream, kKDoubleQuant);
-  double_quant_kernel<<<grid, threads, 0, stream>>>(absmax, n_blocks, gmax, absmax_q,
-                                                    absmax_scale);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, double_quant_kernel, absmax, n_blocks, gmax, absmax_q,
+                                     absmax_scale);
   NF4_PROF_END(stream, kKDoubleQuant);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;
 }
@@ -269,26 +367,28 @@ cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int
   const int bs_words = w.block_size / 8;
   const int shift = log2_exact(bs_words);
   const int threads = 256;
-  const int grid = grid_for(n_words, threads, sms, 8);
-  const uint32_t* c = reinterpret_cast<const uint32_t*>(w.codes);
   const bool dq = w.double_quant != 0;
-#define NF4_DQ_LAUNCH(T, D)                                                                 \
-  dequant_kernel<T, D><<<grid, threads, 0, stream>>>(c, n_words, shift, bs_words, w.absmax, \
-                                                     w.absmax_q, w.absmax_scale,            \
-                                                     reinterpret_cast<T*>(out))
-  NF4_PROF_BEGIN(stream, kKDequantize);
-  if (out_dtype == NF4_F32) {
-    if (dq) NF4_DQ_LAUNCH(float, true); else NF4_DQ_LAUNCH(float, false);
-  } else if (out_dtype == NF4_BF16) {
-    if (dq) NF4_DQ_LAUNCH(__nv_bfloat16, true); else NF4_DQ_LAUNCH(__nv_bfloat16, false);
-  } else {
-    if (dq) NF4_DQ_LAUNCH(__half, true); else NF4_DQ_LAUNCH(__half, false);
+  {
+    const int grid = grid_for((n_words + 3) / 4, threads, sms, 8);
+    const uint32_t* c = reinterpret_cast<const uint32_t*>(w.codes);
+#define NF4_DQ4_LAUNCH(T, D)                                                                    \
+  dequant_x4_kernel<T, D><<<grid, threads, 0, stream>>>(c, n_words, shift, bs_words, w.absmax, \
+                                                        w.absmax_q, w.absmax_scale,            \
+                                                        reinterpret_cast<T*>(out))
+    NF4_PROF_BEGIN(stream, kKDequantize);
+    if (out_dtype == NF4_F32) {
+      if (dq) NF4_DQ4_LAUNCH(float, true); else NF4_DQ4_LAUNCH(float, false);
+    } else if (out_dtype == NF4_BF16) {
+      if (dq) NF4_DQ4_LAUNCH(__nv_bfloat16, true); else NF4_DQ4_LAUNCH(__nv_bfloat16, false);
+    } else {
+      if (dq) NF4_DQ4_LAUNCH(__half, true); else NF4_DQ4_LAUNCH(__half, false);
+    }
+#undef NF4_DQ4_LAUNCH
+    NF4_PROF_END(stream, kKDequantize);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) ++*launches;
+    return e;
   }
-#undef NF4_DQ_LAUNCH
-  NF4_PROF_END(stream, kKDequantize);
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) ++*launches;
-  return e;
 }
 
 }  // namespace nf4

@@ -125,3 +125,16 @@ def test_linear_host_validation():
     st = L.qlora_linear_bwd(ctypes.byref(_cw()), FAKE, 16, FAKE, FAKE, 16, 32.0, 1, None, None,
                             FAKE, FAKE, None, FAKE, 1 << 40, None)
     assert st == 1                                # dy required
+
+
+def test_bucket_encoding_conditions():
+    # The quantize kernel's fast encode indexes 64 buckets of width 1/32 over
+    # [-1, 1] and compares with the single threshold inside the bucket.  It is
+    # exact only if no bucket holds two thresholds and no threshold lies
+    # within the index rounding (2^-24) of a bucket edge.
+    _, th = Q.codebook()
+    th = np.array(th, dtype=np.float64)
+    edges = np.arange(65) / 32.0 - 1.0
+    assert np.min(np.abs(th[:, None] - edges[None, :])) > 2.0 ** -20
+    counts = [np.sum((th >= edges[j]) & (th < edges[j] + 1 / 32)) for j in range(64)]
+    assert max(counts) <= 1

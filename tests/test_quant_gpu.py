@@ -99,6 +99,11 @@ def test_edge_values(cuda_device):
     d[1] = np.float32(-7e-43)
     blocks.append(d)
     blocks.append(rng.permutation(np.resize(lv, 64)).astype(np.float32) * np.float32(3.0))
+    # block scales outside the fast-reciprocal range (above 2^120, below 2^-120)
+    big = np.resize(mids, 63).astype(np.float32) * np.float32(2.0 ** 124)
+    blocks.append(np.concatenate([big, [np.float32(2.0 ** 124)]]))
+    small = np.resize(mids, 63).astype(np.float32) * np.float32(2.0 ** -122)
+    blocks.append(np.concatenate([small, [np.float32(2.0 ** -122)]]))
     w = np.stack(blocks)
     for dq in (False, True):
         q, ref = _check_quant(w, 64, dq, cuda_device)
