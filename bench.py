@@ -543,6 +543,43 @@ def cpu_baseline(case, seconds):
                       f"cpu={cpu_model()}"}
 
 
+def profile_row(args):
+    """Eager launches of one secondary row, for an ncu capture of its kernels:
+    `warmup + steps` calls of each variant, no timing, no JSON line."""
+    import torch
+    from qlora_linear_layers_nf4_b200 import nf4qlora as Q
+    from qlora_linear_layers_nf4_b200 import workloads as WL
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n = args.warmup + args.steps
+    ws = Q.Workspace(dev)
+    if args.profile_row in ("quantize", "dequantize"):
+        w = torch.from_numpy(WL.draw_weight(WL.QUANT_SHAPE, WL.QUANT_SEED)).to(dev)
+        if args.profile_row == "quantize":
+            for _ in range(n):
+                Q.quantize(w, 64, False, workspace=ws)
+                Q.quantize(w, 64, True, workspace=ws)
+        else:
+            qs = [Q.quantize(w, 64, dq, workspace=ws) for dq in (False, True)]
+            for _ in range(n):
+                for q in qs:
+                    Q.dequantize(q, "f32")
+                    Q.dequantize(q, "bf16")
+    elif args.profile_row == "decode":
+        base = WL.DECODE[0]
+        q = Q.quantize(torch.from_numpy(WL.draw_weight((base.n, base.k), seed=200)).to(dev), 64, True)
+        for case in WL.DECODE:
+            inp = WL.draw_linear(case)
+            x, A, B = (bf16_dev(v, dev) for v in (inp.x, inp.a, inp.b))
+            for _ in range(n):
+                Q.linear_fwd(q, x, A, B, case.alpha, workspace=ws)
+    torch.cuda.synchronize()
+    if ws.read_status() != 0:
+        raise RuntimeError("device status reported an error")
+    print(f"profile_row {args.profile_row}: {Q.launch_count()} launches", flush=True)
+
+
 # --------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -591,10 +628,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile-row", choices=["quantize", "dequantize", "decode"],
+                    help="only launch one secondary row eagerly (for ncu); no bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile_row:
+        profile_row(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -15,8 +15,9 @@
 //   fused_nf4_gemm<kFwd>  y[M,N]  = x W'^T + T B^T (+ bias)   K-major W' tiles
 //   fused_nf4_gemm<kDx>   dx[M,K] = dy W' + U A                 MN-major W' tiles
 //   adapter_gemm          the rank-r products T, U, dB, dA^T, split along the
-//                         reduction with fp32 partials
-//                         (the last CTA of each tile adds the slices in order)
+//                         reduction over a thread-block cluster whose CTAs
+//                         sum their fp32 partials through distributed
+//                         shared memory
 #include <algorithm>
 
 #include <cuda.h>
@@ -218,8 +219,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         if (it < p.main_steps) {
           mbar_arrive_expect_tx(&sh->full[s], kABytes + kCBytes);
           const int k0 = it * kTileK;  // fwd: K index; dx: N index (the reduction)
-          tma_load_2d(a, &tm_a, &sh->full[s], k0, m0);
-          tma_load_2d(a + kHalfABytes, &tm_a, &sh->full[s], k0, m0 + 128);
+          tma_load_2d(a, &tm_a, &sh->full[s], k0, m0);     // 256 rows: both halves
           if (MODE == kFwd) {
             tma_load_2d(stage_c(s), &tm_codes, &sh->full[s], k0 / 2, tile_n0);
           } else {
@@ -231,7 +231,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           const int r0 = (it - p.main_steps) * kTileK;
           mbar_arrive_expect_tx(&sh->full[s], kABytes + kBBytes);
           tma_load_2d(a, &tm_a2, &sh->full[s], r0, m0);
-          tma_load_2d(a + kHalfABytes, &tm_a2, &sh->full[s], r0, m0 + 128);
           if (MODE == kFwd) {
             tma_load_2d(stage_b(s), &tm_b2, &sh->full[s], r0, tile_n0);
           } else {
@@ -383,30 +382,65 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 // dequantizes only its 128-row half of the W' tile per K step, so every
 // dequantized element feeds twice the MMA work of the single-CTA kernel and
 // each CTA reads half the B operand from shared memory.
-//   rank r of the pair: A rows m0 + 256 h + 128 r (h = 0, 1) and W' half
-//   n0 + 128 r; the leader (rank 0) issues the MMAs, both CTAs' A loads
-//   complete on the leader's barrier, the leader's commits multicast to both.
+//   rank r of the pair: A rows m0 + 256 r .. + 255 (one 256-row TMA box per
+//   K step; its 128-row halves h = 0, 1 are the A operands of the two
+//   accumulators, so accumulator h of rank r holds rows m0 + 256 r + 128 h)
+//   and W' half n0 + 128 r; the leader (rank 0) issues the MMAs, both CTAs'
+//   A loads complete on the leader's barrier, the leader's commits multicast
+//   to both.
 
 constexpr int kP2Stages = 4;
 constexpr int kP2DeqWarps = 8;                          // 2 threads per W' row
-constexpr int kP2Threads = 64 + kP2DeqWarps * 32;
-constexpr uint32_t kP2ABytes = 2 * kHalfABytes;        // two 128-row A blocks
+constexpr int kP2CodeWarp = 2 + kP2DeqWarps;            // code-tile TMA producer
+// The A tile of a step is split over this many producer warps (warp 0 and
+// warps kP2CodeWarp + 1 ..): one warp keeps only about one TMA box in
+// flight per few hundred ns, so several warps shorten the A-tile latency.
+#ifndef NF4_P2_A_WARPS
+#define NF4_P2_A_WARPS 2
+#endif
+constexpr int kP2AWarps = NF4_P2_A_WARPS;
+#ifndef NF4_P2_ROT_MUL
+#define NF4_P2_ROT_MUL 13
+#endif
+constexpr int kP2ARows = 256 / kP2AWarps;               // A rows per producer box
+constexpr int kP2Threads = 64 + kP2DeqWarps * 32 + 32 * kP2AWarps;
+constexpr uint32_t kP2ABytes = 2 * kHalfABytes;        // 256 A rows (two 128-row blocks)
 constexpr uint32_t kP2BBytes = 128 * 128;              // this CTA's 128 W' rows
-constexpr uint32_t kP2CBytes = 128 * 32;               // their codes
-constexpr uint32_t kP2StageBytes = kP2ABytes + kP2BBytes + kP2CBytes;
-constexpr size_t kP2Smem = size_t(kP2Stages) * kP2StageBytes + 1024 + 256;
+constexpr uint32_t kP2StageBytes = kP2ABytes + kP2BBytes;
+// NF4 codes arrive in their own ring, four K steps per TMA box: forward,
+// 128 W rows x 128 code bytes (128-byte swizzle); dx, 256 W rows x 64 code
+// bytes (64-byte swizzle).  Either way 16 KB per box and a conflict-free
+// 16-byte read per thread.
+constexpr int kP2CodeSteps = 4;
+constexpr int kP2CodeSlots = 2;
+constexpr uint32_t kP2CodeBytes = 128 * 128;
+constexpr size_t kP2Smem =
+    size_t(kP2Stages) * kP2StageBytes + size_t(kP2CodeSlots) * kP2CodeBytes + 1024 + 256;
 constexpr int kP2TileM = 512;
 
 struct PairShared {
-  uint64_t afull[kP2Stages];   // leader: A (+ adapter B) bytes of both CTAs landed
-  uint64_t cfull[kP2Stages];   // each CTA: its code tile landed
-  uint64_t bready[kP2Stages];  // leader: both CTAs' W' halves written (16 warp arrivals)
-  uint64_t empty[kP2Stages];   // each CTA: the MMAs reading the stage finished
+  uint64_t afull[kP2Stages];     // leader: A (+ adapter B) bytes of both CTAs landed
+  uint64_t bready[kP2Stages];    // leader: both CTAs' W' halves written (16 warp arrivals)
+  uint64_t empty[kP2Stages];     // each CTA: the MMAs reading the stage finished
+  uint64_t cfull[kP2CodeSlots];  // each CTA: a code box landed
+  uint64_t cempty[kP2CodeSlots]; // each CTA: its 8 dequant warps finished a code box
   uint64_t accum;
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
+
+// Byte offset in a code slot of the 16 code bytes that thread (row, half)
+// dequantizes at step j (0..3) of the slot's four: 128-byte swizzle of
+// 128-byte rows (forward) or 64-byte swizzle of 64-byte rows (dx, where tile
+// row `row` is W row j * 64 + (row & 63) and code column group row >> 6).
+template <int MODE>
+__device__ __forceinline__ uint32_t code_offset(uint32_t row, uint32_t half, uint32_t j) {
+  if (MODE == kFwd) return row * 128u + ((((2u * j + half) ^ (row & 7u))) << 4);
+  const uint32_t R = j * 64u + (row & 63u);
+  const uint32_t c = 2u * (row >> 6) + half;
+  return R * 64u + ((c ^ ((R >> 1) & 3u)) << 4);
+}
 
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
@@ -416,10 +450,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
                         const __grid_constant__ CUtensorMap tm_codes, const FusedParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  PairShared* sh = reinterpret_cast<PairShared*>(smem + kP2Stages * kP2StageBytes);
+  uint8_t* code_base = smem + kP2Stages * kP2StageBytes;
+  PairShared* sh = reinterpret_cast<PairShared*>(code_base + kP2CodeSlots * kP2CodeBytes);
   auto stage_a = [&](int s) { return smem + s * kP2StageBytes; };
   auto stage_b = [&](int s) { return smem + s * kP2StageBytes + kP2ABytes; };
-  auto stage_c = [&](int s) { return smem + s * kP2StageBytes + kP2ABytes + kP2BBytes; };
+  auto code_slot = [&](int c) { return code_base + c * kP2CodeBytes; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -429,14 +464,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
   const int m0 = blockIdx.y * kP2TileM;
   const int total_steps = p.main_steps + p.adapter_steps;
   volatile uint32_t* abort_flag = &sh->abort_flag;
+  // The pairs of one M tile run at the same time and read the same A rows;
+  // each starts its reduction at a different whole code box (rotation by
+  // kstep_rot steps), so they do not all request the same lines at once.
+  const int code_groups = p.main_steps / kP2CodeSteps;
+  const int kstep_rot = (p.main_steps % kP2CodeSteps == 0 && NF4_P2_ROT_MUL > 0)
+                            ? kP2CodeSteps * int(((blockIdx.x >> 1) * NF4_P2_ROT_MUL) % code_groups)
+                            : 0;
+  auto kstep = [&](int it) { return it + kstep_rot < p.main_steps ? it + kstep_rot : it + kstep_rot - p.main_steps; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kP2Stages; ++s) {
       mbar_init(&sh->afull[s], 1);
-      mbar_init(&sh->cfull[s], 1);
       // leader: its own 8 dequant warps + one forwarded arrival from the peer
       mbar_init(&sh->bready[s], rank == 0 ? kP2DeqWarps + 1 : kP2DeqWarps);
       mbar_init(&sh->empty[s], 1);
+    }
+    for (int c = 0; c < kP2CodeSlots; ++c) {
+      mbar_init(&sh->cfull[c], 1);
+      mbar_init(&sh->cempty[c], kP2DeqWarps);
     }
     mbar_init(&sh->accum, 1);
     mbar_init(&sh->drain, 1);
@@ -457,36 +503,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
 
-  if (warp == 0) {
-    // ---------------- TMA producer (both CTAs)
+  const int a_part = warp == 0 ? 0 : (warp > kP2CodeWarp ? warp - kP2CodeWarp : -1);
+  if (a_part >= 0) {
+    // ---------------- A (and adapter B) TMA producers (both CTAs): producer
+    // a_part loads A rows a_part * kP2ARows .. + kP2ARows - 1 of this CTA's 256
     if (lane == 0) {
-      int issued = 0;
+      const int arow = a_part * kP2ARows;
       for (int it = 0; it < total_steps; ++it) {
         const int s = it % kP2Stages;
         const uint32_t ph = (it / kP2Stages) & 1;
         if (!mbar_wait_cluster(&sh->empty[s], ph ^ 1, abort_flag, p.status)) break;
         const uint32_t afull_leader = mapa_shared(smem_u32(&sh->afull[s]), 0);
-        uint8_t* a = stage_a(s);
+        uint8_t* a = stage_a(s) + arow * 128;
         if (it < p.main_steps) {
-          if (rank == 0) mbar_arrive_expect_tx(&sh->afull[s], 2 * kP2ABytes);
-          mbar_arrive_expect_tx(&sh->cfull[s], kP2CBytes);
-          const int k0 = it * kTileK;
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d_pair(a + h * kHalfABytes, &tm_a, afull_leader, k0, m0 + 256 * h + 128 * int(rank));
-          if (MODE == kFwd) {
-            tma_load_2d(stage_c(s), &tm_codes, &sh->cfull[s], k0 / 2, my_n0);
-          } else {
-#pragma unroll
-            for (int g = 0; g < 2; ++g)
-              tma_load_2d(stage_c(s) + g * 2048, &tm_codes, &sh->cfull[s], (my_n0 + 64 * g) / 2, k0);
-          }
+          if (rank == 0 && a_part == 0) mbar_arrive_expect_tx(&sh->afull[s], 2 * kP2ABytes);
+          tma_load_2d_pair(a, &tm_a, afull_leader, kstep(it) * kTileK, m0 + 256 * int(rank) + arow);
         } else {
           const int r0 = (it - p.main_steps) * kTileK;
-          if (rank == 0) mbar_arrive_expect_tx(&sh->afull[s], 2 * (kP2ABytes + kP2BBytes));
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d_pair(a + h * kHalfABytes, &tm_a2, afull_leader, r0, m0 + 256 * h + 128 * int(rank));
+          if (rank == 0 && a_part == 0) mbar_arrive_expect_tx(&sh->afull[s], 2 * (kP2ABytes + kP2BBytes));
+          tma_load_2d_pair(a, &tm_a2, afull_leader, r0, m0 + 256 * int(rank) + arow);
+          if (a_part != 0) continue;
           if (MODE == kFwd) {
             tma_load_2d_pair(stage_b(s), &tm_b2, afull_leader, r0, my_n0);
           } else {
@@ -495,14 +531,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
               tma_load_2d_pair(stage_b(s) + g * 8192, &tm_b2, afull_leader, my_n0 + 64 * g, r0);
           }
         }
+      }
+    }
+  } else if (warp == kP2CodeWarp) {
+    // ---------------- code producer: one box per four K steps into a two-slot ring
+    if (lane == 0) {
+      const int groups = int((p.main_steps + kP2CodeSteps - 1) / kP2CodeSteps);
+      int issued = 0;
+      for (int g = 0; g < groups; ++g) {
+        const int c = g % kP2CodeSlots;
+        const uint32_t ph = (g / kP2CodeSlots) & 1;
+        if (!mbar_wait(&sh->cempty[c], ph ^ 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&sh->cfull[c], kP2CodeBytes);
+        const int kg = kstep(g * kP2CodeSteps) / kP2CodeSteps;   // code box of this group
+        if (MODE == kFwd)   // code bytes kg*128 .. +127 of W rows my_n0 .. +127
+          tma_load_2d(code_slot(c), &tm_codes, &sh->cfull[c], kg * 128, my_n0);
+        else                // code bytes my_n0/2 .. +63 of W rows kg*256 .. +255
+          tma_load_2d(code_slot(c), &tm_codes, &sh->cfull[c], my_n0 / 2, kg * 256);
         ++issued;
       }
       if (*abort_flag) {
-        // Unwind: wait (bounded) for this CTA's code copies still in flight.
-        for (int it = issued - 1; it >= 0 && it >= issued - kP2Stages; --it) {
-          if (it >= p.main_steps) continue;
+        // Unwind: wait (bounded) for the code copies still in flight.
+        for (int g = issued - 1; g >= 0 && g >= issued - kP2CodeSlots; --g) {
           uint32_t dummy_abort = 0;
-          mbar_wait(&sh->cfull[it % kP2Stages], (it / kP2Stages) & 1, &dummy_abort, nullptr);
+          mbar_wait(&sh->cfull[g % kP2CodeSlots], (g / kP2CodeSlots) & 1, &dummy_abort, nullptr);
         }
       }
     }
@@ -557,10 +609,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       }
     }
   } else {
-    // ---------------- dequant warps: thread pair per W' row (one NF4 block)
-    const int t = threadIdx.x - 64;                   // 0..255
-    const int row = t >> 1;                           // 0..127 tile row
-    const uint32_t half = uint32_t(t & 1);
+    // ---------------- dequant warps: thread pair per W' row (one NF4 block);
+    // a warp covers 16 rows, lanes 0-15 the first half of each block and
+    // lanes 16-31 the second, so each quarter-warp touches 8 consecutive rows.
+    const int row = (warp - 2) * 16 + (lane & 15);    // 0..127 tile row
+    const uint32_t half = uint32_t(lane >> 4);
     const bool dq = p.double_quant != 0;
     const float s_g = dq ? __ldg(p.absmax_scale) : 0.0f;
     int64_t w_row;
@@ -575,9 +628,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       row_step = 64;
     }
     auto scale_at = [&](int it) -> float {
-      const int64_t wr = w_row + int64_t(row_step) * it;
+      const int ks = kstep(it);
+      const int64_t wr = w_row + int64_t(row_step) * ks;
       if (wr >= p.N) return 0.0f;
-      const int bcol = (MODE == kFwd) ? it : block_col0;
+      const int bcol = (MODE == kFwd) ? ks : block_col0;
       if (MODE == kDx && bcol >= p.kb_per_row) return 0.0f;
       return load_scale(p.absmax_q, p.absmax, s_g, dq, wr * p.kb_per_row + bcol);
     };
@@ -593,11 +647,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       sc[1] = sc[2];
       sc[2] = sc[3];
       sc[3] = (it + 4 < p.main_steps) ? scale_at(it + 4) : 0.0f;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sh->cfull[s], ph, abort_flag, p.status))) break;
-      dequant_half_row(stage_c(s) + row * 32 + half * 16, scale, stage_b(s), uint32_t(row), half);
+      const int g = it / kP2CodeSteps;
+      const int j = it % kP2CodeSteps;
+      const int c = g % kP2CodeSlots;
+      // the W' half of stage s is free once the MMAs of step it - kP2Stages
+      // finished (the first round passes at once), and the codes of group g landed
+      bool ok = mbar_wait_cluster(&sh->empty[s], ph ^ 1, abort_flag, p.status);
+      if (ok && j == 0) ok = mbar_wait(&sh->cfull[c], (g / kP2CodeSlots) & 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      dequant_half_row(code_slot(c) + code_offset<MODE>(uint32_t(row), half, uint32_t(j)), scale,
+                       stage_b(s), uint32_t(row), half);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->bready[s]);
+      if (lane == 0) {
+        mbar_arrive(&sh->bready[s]);
+        if (j == kP2CodeSteps - 1 || it == p.main_steps - 1) mbar_arrive(&sh->cempty[c]);
+      }
     }
 
     // ---------------- epilogue: this CTA's 128 rows of both accumulators
@@ -606,7 +671,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     if (ok) {
       const int quad = warp & 3;
       const int h = (warp - 2) >> 2;
-      const int grow = m0 + 256 * h + 128 * int(rank) + quad * 32 + lane;
+      const int grow = m0 + 256 * int(rank) + 128 * h + quad * 32 + lane;
       for (int c = 0; c < kTileN / 32; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + h * kTileN + c * 32, v);
@@ -902,7 +967,7 @@ EncodeTiledFn encode_fn() {
 
 // 2-D map over a row-major matrix: `inner` elements per row, `outer` rows.
 bool make_map(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
-              uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+              uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const uint32_t esize = bf16 ? 2 : 1;
@@ -913,9 +978,14 @@ bool make_map(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uin
   CUresult res = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                     const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return res == CUDA_SUCCESS;
+}
+
+bool make_map(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+              uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  return make_map(map, base, bf16, inner, outer, box_inner, box_outer,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -1091,10 +1161,12 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   const bool pair = use_pair(a.M);
   const uint32_t brows = pair ? 128 : 256;     // W' rows per CTA
   CUtensorMap ta, ta2, tb2, tc;
-  bool ok = make_map(&ta, a.x, true, a.K, a.M, 64, 128, true);
-  ok = ok && make_map(&ta2, T, true, a.r, a.M, 64, 128, true);
+  const uint32_t arows = pair ? uint32_t(kP2ARows) : 256u;   // A rows per TMA box
+  bool ok = make_map(&ta, a.x, true, a.K, a.M, 64, arows, true);
+  ok = ok && make_map(&ta2, T, true, a.r, a.M, 64, arows, true);
   ok = ok && make_map(&tb2, a.B, true, a.r, a.N, 64, brows, true);
-  ok = ok && make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, brows, false);
+  ok = ok && (pair ? make_map(&tc, a.w->codes, false, a.K / 2, a.N, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)
+                   : make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, brows, false));
   if (!ok) return cudaErrorInvalidValue;
   const FusedParams p = fused_params(a, kFwd);
   NF4_PROF_BEGIN(st, kKFusedFwd);
@@ -1154,14 +1226,17 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
   if (a.dx == nullptr) return cudaSuccess;
   // dx = dy W' + U A
   CUtensorMap ta, ta2, tb2, tc;
-  bool ok = make_map(&ta, a.dy, true, a.N, a.M, 64, 128, true);
-  ok = ok && make_map(&ta2, U, true, a.r, a.M, 64, 128, true);
+  const bool pair = use_pair(a.M);
+  const uint32_t arows = pair ? uint32_t(kP2ARows) : 256u;   // A rows per TMA box
+  bool ok = make_map(&ta, a.dy, true, a.N, a.M, 64, arows, true);
+  ok = ok && make_map(&ta2, U, true, a.r, a.M, 64, arows, true);
   ok = ok && make_map(&tb2, a.A, true, a.K, a.r, 64, 64, true);
-  ok = ok && make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, 64, false);
+  ok = ok && (pair ? make_map(&tc, a.w->codes, false, a.K / 2, a.N, 64, 256, CU_TENSOR_MAP_SWIZZLE_64B)
+                   : make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, 64, false));
   if (!ok) return cudaErrorInvalidValue;
   const FusedParams p = fused_params(a, kDx);
   NF4_PROF_BEGIN(st, kKFusedDx);
-  if (use_pair(a.M)) {
+  if (pair) {
     dim3 grid(unsigned(2 * cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kP2TileM)));
     fused_nf4_gemm_pair<kDx><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, p);
   } else {
