@@ -39,7 +39,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the dominant kernel from an ncu capture, keyed by
 # the hash of the kernel source it was taken on (see profiles/); reported as
 # null once the source changes.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/fused_nf4_gemm_pair_11008x4096_M4096.md: forward 112.3 MB, dx 179.8 MB per launch
+    "d2a3cb6c72ac6ec4": {"fwd": 112_319_000, "dx": 179_838_720},
+}
 
 
 def linear_flops(m, n, k, r):
@@ -287,11 +290,14 @@ def run_ours(args):
                 if fused_launches else None)
     peak = pk.get("bf16_tflops_sustained") or pk.get("bf16_tflops")
     src = source_hash()
-    traffic = NCU_TRAFFIC.get(src)
+    tr = NCU_TRAFFIC.get(src)
+    # bytes per launch, averaged over the step's forward and dx launches
+    traffic = (tr["fwd"] + tr["dx"]) / 2 if tr else None
     roofline = {
         "kernel": "fused_nf4_gemm (fwd + dx launches)",
         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
         "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+        "traffic_per_launch": tr,
         "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside a long step)",
         "flops_per_launch": {"fwd": fwd_flops, "dx": dx_flops},
         "share_of_step_kernel_time": (fwd_ms + dx_ms) / total_kernel_ms if total_kernel_ms else None,
