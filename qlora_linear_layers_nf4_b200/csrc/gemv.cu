@@ -36,6 +36,7 @@ constexpr int kGvAWarps = 4;                        // up to 64 adapter rows of 
 constexpr int kGvThreads = (kGvWWarps + kGvAWarps) * 32;
 constexpr int kGvRows = 128;                        // W rows per CTA
 constexpr int kGvMaxBlocks = 16;                    // 64-wide K blocks per CTA
+static_assert(kGvWWarps + kGvAWarps > kGvMaxBlocks, "one issuing warp per K block plus one for B");
 constexpr int kGvMaxR = 16 * kGvAWarps;
 constexpr int kGvLutBytes = 0;                      // the table is a static array
 
@@ -161,24 +162,23 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   const uint32_t abytes = uint32_t(p.r_pad) * 128u;
 
   // Every byte this CTA reads is requested before anything else, one barrier
-  // per 64-wide K block (one lane of warp 0 each, so the copies issue in
-  // parallel) so compute starts on the first block to land.
-  if (warp == 0) {
-    if (lane == 0) abort_flag = 0;
-    if (lane <= kGvMaxBlocks) {
-      mbar_init(&bar[lane], 1);
-      fence_barrier_init();
-      fence_proxy_async_smem();
-      if (lane == kGvMaxBlocks) {
-        mbar_arrive_expect_tx(&bar[kGvMaxBlocks], uint32_t(kGvRows) * uint32_t(p.r) * 2u);
-        tma_load_2d(smem + L.bs, &tm_b, &bar[kGvMaxBlocks], 0, n0);
-      } else if (lane < nblk) {
-        const int b = lane, kb = kb0 + b;
-        mbar_arrive_expect_tx(&bar[b], 4096u + xbytes + abytes);
-        tma_load_2d(codes + b * 4096, &tm_codes, &bar[b], kb * 32, n0);
-        tma_load_2d(xs + b * xbytes, &tm_x, &bar[b], kb * 64, 0);
-        tma_load_2d(as + b * abytes, &tm_a, &bar[b], kb * 64, 0);
-      }
+  // per 64-wide K block so compute starts on the first block to land.  Warp b
+  // issues block b's copies (and warp kGvMaxBlocks the B tile): one warp keeps
+  // only a few TMA copies going per microsecond, so the issue is spread.
+  if (threadIdx.x == 0) abort_flag = 0;
+  if (lane == 0 && warp <= kGvMaxBlocks) {
+    mbar_init(&bar[warp], 1);
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    if (warp == kGvMaxBlocks) {
+      mbar_arrive_expect_tx(&bar[kGvMaxBlocks], uint32_t(kGvRows) * uint32_t(p.r) * 2u);
+      tma_load_2d(smem + L.bs, &tm_b, &bar[kGvMaxBlocks], 0, n0);
+    } else if (warp < nblk) {
+      const int b = warp, kb = kb0 + b;
+      mbar_arrive_expect_tx(&bar[b], 4096u + xbytes + abytes);
+      tma_load_2d(codes + b * 4096, &tm_codes, &bar[b], kb * 32, n0);
+      tma_load_2d(xs + b * xbytes, &tm_x, &bar[b], kb * 64, 0);
+      tma_load_2d(as + b * abytes, &tm_a, &bar[b], kb * 64, 0);
     }
   }
   // Block scales: independent loads issued up front (row = t & 127).

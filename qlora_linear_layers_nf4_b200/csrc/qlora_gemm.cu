@@ -158,7 +158,6 @@ struct FusedShared {
   uint64_t bready[kStages];  // dequantized B tile written (8 warp arrivals)
   uint64_t empty[kStages];   // MMAs reading the stage finished (umma_commit)
   uint64_t accum;            // all MMAs finished
-  uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
@@ -189,7 +188,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       mbar_init(&sh->empty[s], 1);
     }
     mbar_init(&sh->accum, 1);
-    mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -254,6 +252,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, kTileN, false, MODE == kDx);
       bool ok = true;
+      int issued = 0;
       for (int it = 0; it < total_steps && ok; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
@@ -278,15 +277,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             umma_f16(tmem + h * kTileN, adesc, bdesc, idesc, (it > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&sh->empty[s]);
+        // The last step's commit goes to accum (nobody waits on its stage);
+        // MMAs finish in order, so it covers the whole accumulation.
+        umma_commit(it + 1 < total_steps ? &sh->empty[s] : &sh->accum);
+        ++issued;
       }
-      if (ok) {
-        umma_commit(&sh->accum);
-      } else {
-        umma_commit(&sh->drain);
-        uint32_t dummy_abort = 0;
-        mbar_wait(&sh->drain, 0, &dummy_abort, nullptr);
-      }
+      if (!ok) drain_issued(sh->empty, issued, kStages);
     }
   } else {
     // ---------------- dequant warps (one NF4 block = one tile row per thread)
@@ -425,7 +421,6 @@ struct PairShared {
   uint64_t cfull[kP2CodeSlots];  // each CTA: a code box landed
   uint64_t cempty[kP2CodeSlots]; // each CTA: its 8 dequant warps finished a code box
   uint64_t accum;
-  uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
@@ -485,7 +480,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       mbar_init(&sh->cempty[c], kP2DeqWarps);
     }
     mbar_init(&sh->accum, 1);
-    mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -512,7 +506,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       for (int it = 0; it < total_steps; ++it) {
         const int s = it % kP2Stages;
         const uint32_t ph = (it / kP2Stages) & 1;
-        if (!mbar_wait_cluster(&sh->empty[s], ph ^ 1, abort_flag, p.status)) break;
+        if (!mbar_wait(&sh->empty[s], ph ^ 1, abort_flag, p.status)) break;
         const uint32_t afull_leader = mapa_shared(smem_u32(&sh->afull[s]), 0);
         uint8_t* a = stage_a(s) + arow * 128;
         if (it < p.main_steps) {
@@ -574,11 +568,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     if (lane == 0 && rank == 0) {
       const uint32_t idesc = idesc_bf16_f32(256, kTileN, false, MODE == kDx);
       bool ok = true;
+      int issued = 0;
       for (int it = 0; it < total_steps && ok; ++it) {
         const int s = it % kP2Stages;
         const uint32_t ph = (it / kP2Stages) & 1;
         const bool adapter = it >= p.main_steps;
-        ok = mbar_wait_cluster(&sh->afull[s], ph, abort_flag, p.status);
+        // afull completes by TMA transactions (and empty / accum by
+        // tcgen05.commit): a CTA-scope acquire is enough there.  bready is
+        // arrived by the peer's thread, so its wait acquires at cluster scope.
+        ok = mbar_wait(&sh->afull[s], ph, abort_flag, p.status);
         if (ok && !adapter) ok = mbar_wait_cluster(&sh->bready[s], ph, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
@@ -598,15 +596,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
             umma_f16_pair(tmem + h * kTileN, adesc, bdesc, idesc, (it > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit_pair_mc(&sh->empty[s], 0x3);
+        // One commit per step, multicast to both CTAs.  The last step's
+        // commit goes to accum instead (nobody waits on its stage); MMAs
+        // finish in order, so it covers the whole accumulation.  (A second
+        // commit issued right behind the first was seen to arrive before the
+        // MMAs had finished reading their operands.)
+        umma_commit_pair_mc(it + 1 < total_steps ? &sh->empty[s] : &sh->accum, 0x3);
+        ++issued;
       }
-      if (ok) {
-        umma_commit_pair_mc(&sh->accum, 0x3);
-      } else {
-        umma_commit_pair_mc(&sh->drain, 0x1);
-        uint32_t dummy_abort = 0;
-        mbar_wait_cluster(&sh->drain, 0, &dummy_abort, nullptr);
-      }
+      if (!ok) drain_issued(sh->empty, issued, kP2Stages);
     }
   } else {
     // ---------------- dequant warps: thread pair per W' row (one NF4 block);
@@ -652,7 +650,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       const int c = g % kP2CodeSlots;
       // the W' half of stage s is free once the MMAs of step it - kP2Stages
       // finished (the first round passes at once), and the codes of group g landed
-      bool ok = mbar_wait_cluster(&sh->empty[s], ph ^ 1, abort_flag, p.status);
+      bool ok = mbar_wait(&sh->empty[s], ph ^ 1, abort_flag, p.status);
       if (ok && j == 0) ok = mbar_wait(&sh->cfull[c], (g / kP2CodeSlots) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       dequant_half_row(code_slot(c) + code_offset<MODE>(uint32_t(row), half, uint32_t(j)), scale,
@@ -666,7 +664,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     }
 
     // ---------------- epilogue: this CTA's 128 rows of both accumulators
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_cluster(&sh->accum, 0, abort_flag, p.status));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&sh->accum, 0, abort_flag, p.status));
     tc_fence_after();
     if (ok) {
       const int quad = warp & 3;
@@ -763,7 +761,6 @@ struct AdapterShared {
   uint64_t full[kAdStages];
   uint64_t empty[kAdStages];
   uint64_t accum;
-  uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
@@ -786,11 +783,10 @@ __global__ void __launch_bounds__(kAdThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAdStages; ++s) {
-      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->full[s], 2);     // the A copies' issuer and the B copies' issuer
       mbar_init(&sh->empty[s], 1);
     }
     mbar_init(&sh->accum, 1);
-    mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -806,41 +802,52 @@ __global__ void __launch_bounds__(kAdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nsteps; ++i) {
-        const int s = i % kAdStages;
-        const uint32_t ph = (i / kAdStages) & 1;
-        if (!mbar_wait(&sh->empty[s], ph ^ 1, abort_flag, p.status)) break;
-        uint8_t* a = smem + s * stage_bytes;
-        uint8_t* b = a + kAdABytes;
-        const int red0 = (step0 + i) * 64;
-        mbar_arrive_expect_tx(&sh->full[s], stage_bytes);
+  // TMA copies: the A tile from warp 0 and the B tile from warp 2 (one warp
+  // keeps only a few TMA copies going per microsecond); each arrives on the
+  // stage's full barrier with its own byte count.
+  const bool a_issuer = warp == 0 && lane == 0;
+  const bool b_issuer = warp == 2 && lane == 0;
+  if (a_issuer || b_issuer) {
+    int issued = 0;
+    for (int i = 0; i < nsteps; ++i) {
+      const int s = i % kAdStages;
+      const uint32_t ph = (i / kAdStages) & 1;
+      if (!mbar_wait(&sh->empty[s], ph ^ 1, abort_flag, p.status)) break;
+      uint8_t* a = smem + s * stage_bytes;
+      uint8_t* b = a + kAdABytes;
+      const int red0 = (step0 + i) * 64;
+      if (a_issuer) {
+        mbar_arrive_expect_tx(&sh->full[s], kAdABytes);
         if (p.a_mn) {
           tma_load_2d(a, &tm_a, &sh->full[s], mo0, red0);
           tma_load_2d(a + 8192, &tm_a, &sh->full[s], mo0 + 64, red0);
         } else {
           tma_load_2d(a, &tm_a, &sh->full[s], red0, mo0);
         }
+      } else {
+        mbar_arrive_expect_tx(&sh->full[s], b_bytes);
         if (p.b_mn) {
           for (int g = 0; g < p.NP / 64; ++g) tma_load_2d(b + g * 8192, &tm_b, &sh->full[s], 64 * g, red0);
         } else {
           tma_load_2d(b, &tm_b, &sh->full[s], red0, 0);
         }
-        ++issued;
       }
-      if (*abort_flag) {
-        for (int i = issued - 1; i >= 0 && i >= issued - kAdStages; --i) {
-          uint32_t dummy_abort = 0;
-          mbar_wait(&sh->full[i % kAdStages], (i / kAdStages) & 1, &dummy_abort, nullptr);
-        }
+      ++issued;
+    }
+    if (*abort_flag) {
+      // Unwind: wait (bounded) for this issuer's copies still in flight.
+      for (int i = issued - 1; i >= 0 && i >= issued - kAdStages; --i) {
+        uint32_t dummy_abort = 0;
+        mbar_wait(&sh->full[i % kAdStages], (i / kAdStages) & 1, &dummy_abort, nullptr);
       }
     }
+  }
+  if (warp == 0) {
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, p.NP, p.a_mn != 0, p.b_mn != 0);
       bool ok = true;
+      int issued = 0;
       for (int i = 0; i < nsteps; ++i) {
         const int s = i % kAdStages;
         const uint32_t ph = (i / kAdStages) & 1;
@@ -857,14 +864,14 @@ __global__ void __launch_bounds__(kAdThreads, 1)
                                         : smem_desc_sw128(b_base + kk * 32, 16, 1024);
           umma_f16(tmem, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&sh->empty[s]);
+        // the last step's commit goes to accum (nobody waits on its stage)
+        umma_commit(i + 1 < nsteps ? &sh->empty[s] : &sh->accum);
+        ++issued;
       }
-      if (ok) {
-        umma_commit(&sh->accum);
-      } else {
-        umma_commit(&sh->drain);
-        uint32_t dummy_abort = 0;
-        mbar_wait(&sh->drain, 0, &dummy_abort, nullptr);
+      if (!ok) {
+        drain_issued(sh->empty, issued, kAdStages);
+      } else if (nsteps == 0) {
+        mbar_arrive(&sh->accum);   // an empty slice: no MMAs to wait for
       }
     }
   } else {

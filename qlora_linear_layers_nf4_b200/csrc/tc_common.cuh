@@ -260,6 +260,16 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// After an abort, wait (bounded) until the MMAs of the steps still in flight
+// finished: step j (of `issued`) released ring stage j % stages with one
+// commit, and every step before issued - stages is known to be complete.
+__device__ __forceinline__ void drain_issued(uint64_t* empty, int issued, int stages) {
+  for (int j = issued > stages ? issued - stages : 0; j < issued; ++j) {
+    uint32_t no_abort = 0;
+    mbar_wait(&empty[j % stages], uint32_t(j / stages) & 1u, &no_abort, nullptr);
+  }
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives row
 // (lane base + i), columns [col, col + 32).
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {

@@ -56,10 +56,13 @@ class Run:
             bb = WL.to_bf16_bits(rng.standard_normal(case.n).astype(np.float32) * np.float32(0.1))
             self.bias = _bf(dev, bb)
             self.bias_np = WL.bf16_bits_to_f32(bb).astype(np.float64)
-        self.y, self.T = Q.linear_fwd(self.q, self.x, self.A, self.B, case.alpha, bias=self.bias)
+        ws = Q.Workspace(dev)
+        self.y, self.T = Q.linear_fwd(self.q, self.x, self.A, self.B, case.alpha, bias=self.bias,
+                                      workspace=ws)
         self.dA, self.dB, self.dx = Q.linear_bwd(self.q, self.x, self.A, self.B, case.alpha, self.dy,
-                                                 t=self.T if pass_t else None)
+                                                 t=self.T if pass_t else None, workspace=ws)
         torch.cuda.synchronize()
+        assert ws.read_status() == 0, "device status word reports an error"
         self.w_hat = O.bf16_to_f32(O.dequantize(self.ref_q, "bf16")).astype(np.float64)
         f = WL.bf16_bits_to_f32
         self.xn, self.an, self.bn, self.dyn = (f(v).astype(np.float64) for v in (inp.x, inp.a, inp.b, inp.dy))
