@@ -6,6 +6,8 @@
 // the frozen base").  Each thread owns 8 consecutive elements (32 bytes in,
 // one u32 of packed codes out); the absmax of a block of bs elements is a
 // shuffle-xor reduction over the bs/8 lanes that hold it.
+#include <algorithm>
+
 #include "nf4_common.cuh"
 #include "kernels.h"
 
@@ -120,34 +122,48 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
   float cta_max = 0.0f;
   bool bad = false;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  // Iterate in whole warps so every lane takes part in the shuffles.
-  for (int64_t base = int64_t(blockIdx.x) * blockDim.x; base < n_words; base += stride) {
-    const int64_t i = base + threadIdx.x;
-    const bool valid = i < n_words;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    if (valid) {
-      a = __ldcs(w + 2 * i);
-      b = __ldcs(w + 2 * i + 1);
-      bad |= !finite8(a, b);
+  // Encode one word (8 elements) whose block max over the G lanes is known.
+  auto encode_word = [&](int64_t i, bool valid, const float4& a, const float4& b, float m) {
+    if (!valid) return;
+    uint32_t word;
+    if (fast_scale(m)) {
+      const float y = __frcp_rn(m);
+      word = pair_byte_fast(a.x, a.y, m, y, buckets) | (pair_byte_fast(a.z, a.w, m, y, buckets) << 8) |
+             (pair_byte_fast(b.x, b.y, m, y, buckets) << 16) |
+             (pair_byte_fast(b.z, b.w, m, y, buckets) << 24);
+    } else {
+      word = pair_byte(a.x, a.y, m) | (pair_byte(a.z, a.w, m) << 8) |
+             (pair_byte(b.x, b.y, m) << 16) | (pair_byte(b.z, b.w, m) << 24);
     }
-    float m = max_abs8(a, b);
+    __stcs(codes + i, word);
+    if ((threadIdx.x & (G - 1)) == 0 && absmax != nullptr) absmax[i / G] = m;
+  };
+  // Two words per thread per iteration, a grid-stride apart, both loaded before
+  // either is encoded (64 bytes in flight per thread).  The loop runs in whole
+  // warps so every lane takes part in the shuffles.
+  for (int64_t base = int64_t(blockIdx.x) * blockDim.x; base < n_words; base += 2 * stride) {
+    const int64_t i0 = base + threadIdx.x;
+    const int64_t i1 = i0 + stride;
+    const bool v0 = i0 < n_words, v1 = i1 < n_words;
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), b0 = a0, a1 = a0, b1 = a0;
+    if (v0) {
+      a0 = __ldcs(w + 2 * i0);
+      b0 = __ldcs(w + 2 * i0 + 1);
+    }
+    if (v1) {
+      a1 = __ldcs(w + 2 * i1);
+      b1 = __ldcs(w + 2 * i1 + 1);
+    }
+    bad |= (v0 && !finite8(a0, b0)) || (v1 && !finite8(a1, b1));
+    float m0 = max_abs8(a0, b0), m1 = max_abs8(a1, b1);
 #pragma unroll
-    for (int o = G / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (valid) {
-      uint32_t word;
-      if (fast_scale(m)) {
-        const float y = __frcp_rn(m);
-        word = pair_byte_fast(a.x, a.y, m, y, buckets) | (pair_byte_fast(a.z, a.w, m, y, buckets) << 8) |
-               (pair_byte_fast(b.x, b.y, m, y, buckets) << 16) |
-               (pair_byte_fast(b.z, b.w, m, y, buckets) << 24);
-      } else {
-        word = pair_byte(a.x, a.y, m) | (pair_byte(a.z, a.w, m) << 8) |
-               (pair_byte(b.x, b.y, m) << 16) | (pair_byte(b.z, b.w, m) << 24);
-      }
-      __stcs(codes + i, word);
-      if ((threadIdx.x & (G - 1)) == 0 && absmax != nullptr) absmax[i / G] = m;
+    for (int o = G / 2; o > 0; o >>= 1) {
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
     }
-    cta_max = fmaxf(cta_max, m);
+    encode_word(i0, v0, a0, b0, m0);
+    encode_word(i1, v1, a1, b1, m1);
+    cta_max = fmaxf(cta_max, fmaxf(m0, m1));
   }
   if (bad) report(status, NF4_ERR_NONFINITE);
   if (gmax != nullptr) cta_global_max(cta_max, gmax);
@@ -186,25 +202,36 @@ __global__ void __launch_bounds__(256) quantize_generic_kernel(
 // Launched as a programmatic dependent of the quantize kernel: it starts
 // early and waits (griddepcontrol.wait) until the quantize grid has finished
 // and its writes are visible.
+// Four scales per thread (one 16-byte load, one 4-byte store), the loads
+// issued before the global maximum is read; the grid covers every group of
+// four once, and the first threads take the n_blocks % 4 tail.
+__device__ __forceinline__ uint32_t dq_code(float a, float g, float s_g, bool fast, float y) {
+  if (!(g > 0.0f)) return 0u;
+  const float ratio = fast ? div_corrected(a, s_g, y) : __fdiv_rn(a, s_g);
+  return uint32_t(min(max(__float2int_rn(ratio), 0), 255));
+}
+
 __global__ void __launch_bounds__(256) double_quant_kernel(
     const float* __restrict__ absmax, int64_t n_blocks, const uint32_t* __restrict__ gmax,
     uint8_t* __restrict__ absmax_q, float* __restrict__ absmax_scale) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t n4 = n_blocks / 4;
+  const int64_t i4 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (i4 < n4) a4 = reinterpret_cast<const float4*>(absmax)[i4];
+  const int64_t tail = n4 * 4 + i4;
+  const float at = (tail < n_blocks) ? absmax[tail] : 0.0f;
   const float g = __uint_as_float(*gmax);
   const float s_g = __fdiv_rn(g, 255.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *absmax_scale = s_g;
   const bool fast = fast_scale(s_g);
   const float y = fast ? __frcp_rn(s_g) : 0.0f;
-  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n_blocks; i += stride) {
-    uint32_t q = 0;
-    if (g > 0.0f) {
-      const float a = absmax[i];
-      const float ratio = fast ? div_corrected(a, s_g, y) : __fdiv_rn(a, s_g);
-      q = uint32_t(min(max(__float2int_rn(ratio), 0), 255));
-    }
-    absmax_q[i] = uint8_t(q);
+  if (i4 < n4) {
+    const uint32_t q = dq_code(a4.x, g, s_g, fast, y) | (dq_code(a4.y, g, s_g, fast, y) << 8) |
+                       (dq_code(a4.z, g, s_g, fast, y) << 16) | (dq_code(a4.w, g, s_g, fast, y) << 24);
+    reinterpret_cast<uint32_t*>(absmax_q)[i4] = q;
   }
+  if (tail < n_blocks) absmax_q[tail] = uint8_t(dq_code(at, g, s_g, fast, y));
 }
 
 // ------------------------------------------------------------------ dequant
@@ -341,7 +368,10 @@ cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uin
                                 uint8_t* absmax_q, float* absmax_scale, int sms,
                                 cudaStream_t stream, int* launches) {
   const int threads = 256;
-  const int grid = grid_for(n_blocks, threads, sms, 4);
+  (void)sms;
+  // one thread per four scales, at least one thread for the tail
+  const int64_t groups = std::max<int64_t>(n_blocks / 4, 1);
+  const int grid = int((groups + threads - 1) / threads);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(grid), 1, 1);
   cfg.blockDim = dim3(unsigned(threads), 1, 1);
