@@ -49,6 +49,9 @@ Readings of points the pages leave open (each is also listed in the design doc):
       bf16 inputs.
   R9  Backward of L = sum(dy * y) with W frozen: dB = s dy^T (x A^T),
       dA = s (dy B)^T x, dx = dy W' + s (dy B) A.
+  R16 Merge: W_merged = w' + s B A from the fp32 dequant w' (not the bf16
+      one), the sum taken exactly and rounded to fp32, then (for a bf16
+      result) to bf16 with ties to even.
 """
 from __future__ import annotations
 
@@ -70,6 +73,7 @@ __all__ = [
     "bf16_to_f32",
     "qlora_forward",
     "qlora_backward",
+    "merge",
     "matmul_bruteforce",
 ]
 
@@ -294,6 +298,33 @@ def qlora_backward(x, w_hat, a, b, alpha: float, dy):
     d_a = s * (u.T @ x)
     d_x = dy @ w_hat + s * (u @ a)
     return d_a, d_b, d_x
+
+
+# ---------------------------------------------------------------------------
+# Merge  ([P3] merge_and_export_gguf: W_merged = W_base + (B @ A) * scale;
+#         [P4] "The merge math", equation 6.3.6; reading R16)
+# ---------------------------------------------------------------------------
+
+def merge(q: dict, a, b, alpha: float, out_dtype: str = "bf16") -> np.ndarray:
+    """Dense merged weight W' + (alpha/r) B A of a quantized base.
+
+    W' is the fp32 dequant; B A and the sum are exact in fp64.  out_dtype
+    "f64" returns that sum, "f32" its round to fp32, "bf16" the uint16 bits of
+    the fp32 value rounded to bf16 (R16).
+    """
+    w = dequantize(q, "f32").astype(np.float64)
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    s = float(alpha) / float(a.shape[0])
+    merged = w + s * (b @ a)
+    if out_dtype == "f64":
+        return merged
+    m32 = merged.astype(np.float32)
+    if out_dtype == "f32":
+        return m32
+    if out_dtype == "bf16":
+        return bf16_round(m32).reshape(merged.shape)
+    raise ValueError(out_dtype)
 
 
 def matmul_bruteforce(p, q):

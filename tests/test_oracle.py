@@ -354,3 +354,59 @@ def test_finite_difference_gradients():
         xm[i, j] -= h
         fd = (loss(xp, a, b) - loss(xm, a, b)) / (2 * h)
         assert abs(fd - d_x[i, j]) <= 1e-8 * max(1.0, abs(d_x[i, j]))
+
+
+# --------------------------------------------------------------------------- merge
+
+def _tiny_q():
+    inp, w_hat, x, a, b, dy = _tiny()
+    q = O.quantize(inp.w, 64, double=inp.case.double_quant)
+    return inp, q, x, a, b
+
+
+def test_merge_equals_forward_on_the_fp32_base():
+    # Equation 6.3.6 with the fp32 dequant as the base: the merged weight
+    # applied to x equals the adapter-on-base forward (an independent path).
+    inp, q, x, a, b = _tiny_q()
+    m = O.merge(q, a, b, inp.case.alpha, "f64")
+    w32 = O.dequantize(q, "f32")
+    y, _ = O.qlora_forward(x, w32, a, b, inp.case.alpha)
+    y2 = O.matmul_bruteforce(x, m.T)
+    assert np.max(np.abs(y - y2)) <= 1e-11 * np.max(np.abs(y))
+
+
+def test_merge_matches_bruteforce_and_rounds_once():
+    inp, q, x, a, b = _tiny_q()
+    s = inp.case.alpha / inp.case.r
+    want = O.dequantize(q, "f32").astype(np.float64) + s * O.matmul_bruteforce(b, a)
+    m = O.merge(q, a, b, inp.case.alpha, "f64")
+    assert np.max(np.abs(m - want)) <= 1e-13 * np.max(np.abs(want))
+    # f32: the nearest fp32 of the exact sum (checked with exact rationals on a sample)
+    m32 = O.merge(q, a, b, inp.case.alpha, "f32")
+    rng = np.random.default_rng(0)
+    for idx in rng.integers(0, m32.size, 64):
+        exact = Fraction(float(want.flat[idx]))
+        got = Fraction(float(m32.flat[idx]))
+        lo = np.nextafter(m32.flat[idx], np.float32(-np.inf))
+        hi = np.nextafter(m32.flat[idx], np.float32(np.inf))
+        assert abs(got - exact) <= abs(Fraction(float(lo)) - exact)
+        assert abs(got - exact) <= abs(Fraction(float(hi)) - exact)
+    # bf16: the fp32 value rounded to bf16 (torch's rounding as the independent routine)
+    import torch
+    mb = O.merge(q, a, b, inp.case.alpha, "bf16")
+    tb = torch.from_numpy(m32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(mb, tb)
+
+
+def test_merge_special_cases():
+    inp, q, x, a, b = _tiny_q()
+    # B = 0: the merge is the plain dequant, bit for bit in both dtypes
+    assert np.array_equal(O.merge(q, a, np.zeros_like(b), inp.case.alpha, "bf16"),
+                          O.dequantize(q, "bf16"))
+    assert np.array_equal(O.merge(q, a, np.zeros_like(b), inp.case.alpha, "f32").view(np.uint32),
+                          O.dequantize(q, "f32").view(np.uint32))
+    # zero base: only the low-rank update remains
+    q0 = O.quantize(np.zeros_like(inp.w), 64)
+    s = inp.case.alpha / inp.case.r
+    assert np.allclose(O.merge(q0, a, b, inp.case.alpha, "f64"), s * O.matmul_bruteforce(b, a),
+                       rtol=1e-13, atol=0)
