@@ -533,6 +533,30 @@ def measure_rows(args, dev, flush, pk, pk_kind, barrier):
     del qws
     torch.cuda.empty_cache()
 
+    # ---- dense merge of the 11008x4096 layer with its r = 64 adapter (bf16 out),
+    # 3 rotating outputs (270 MB)
+    case = WL.PREFILL
+    inp = WL.draw_linear(case)
+    qm = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True)
+    Am, Bm = bf16_dev(inp.a, dev), bf16_dev(inp.b, dev)
+    outs_m = [torch.empty((case.n, case.k), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    wsm = Q.Workspace(dev)
+    bufm = wsm.get(Q.workspace_bytes(Q.OP_MERGE, 0, case.n, case.k, case.r, 64, True))
+    cwm = qm.c_struct()
+
+    def mcall(o):
+        def f():
+            st = L.nf4_merge(ctypes.byref(cwm), ptr(Am), ptr(Bm), case.r, float(case.alpha), Q.NF4_BF16,
+                             ptr(o), ptr(bufm), bufm.numel(), stream())
+            assert st == 0, st
+        return f
+
+    mbytes = (case.n * case.k // 2 + case.n * case.k // 64 + 4 + 2 * case.r * (case.n + case.k)
+              + 2 * case.n * case.k)
+    row("merge_11008x4096_r64_bf16", [mcall(o) for o in outs_m], mbytes)
+    del outs_m, qm
+    torch.cuda.empty_cache()
+
     # ---- the seven targets of one decoder block, fwd + bwd each (long kernels: eager)
     if not args.no_block:
         ws_q = Q.Workspace(dev)
@@ -606,6 +630,13 @@ def profile_row(args):
                 for q in qs:
                     Q.dequantize(q, "f32")
                     Q.dequantize(q, "bf16")
+    elif args.profile_row == "merge":
+        case = WL.PREFILL
+        inp = WL.draw_linear(case)
+        q = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True)
+        A, B = bf16_dev(inp.a, dev), bf16_dev(inp.b, dev)
+        for _ in range(n):
+            Q.merge(q, A, B, case.alpha, "bf16", workspace=ws)
     elif args.profile_row == "decode":
         base = WL.DECODE[0]
         q = Q.quantize(torch.from_numpy(WL.draw_weight((base.n, base.k), seed=200)).to(dev), 64, True)
@@ -668,7 +699,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-row", choices=["quantize", "dequantize", "decode"],
+    ap.add_argument("--profile-row", choices=["quantize", "dequantize", "decode", "merge"],
                     help="only launch one secondary row eagerly (for ncu); no bench line")
     args = ap.parse_args()
     if args.warmup < 3:

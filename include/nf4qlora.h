@@ -73,7 +73,8 @@ typedef enum {
   NF4_OP_QUANTIZE = 0,
   NF4_OP_DEQUANTIZE = 1,
   NF4_OP_LINEAR_FWD = 2,
-  NF4_OP_LINEAR_BWD = 3
+  NF4_OP_LINEAR_BWD = 3,
+  NF4_OP_MERGE = 4
 } nf4_op;
 
 /*
@@ -258,6 +259,26 @@ NF4_API nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t 
                             const void* B, int r, float alpha, int compute_dtype,
                             const void* dy, const void* t, float* dA, float* dB, void* dx,
                             void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Merge of the quantized base with its trained adapter into one dense weight
+ * (qlora-rs src/export.rs, merge_and_export_gguf: W_merged = W_base +
+ * (B @ A) * scale; "LoRA and QLoRA, mathematically", "The merge math",
+ * equation 6.3.6 -- the merged weight stays in BF16, it is not requantized):
+ *   out[n, k] = w'[n, k] + s (B A)[n, k],  s = alpha / r,
+ * w' = fp32(L[code] * scale) the fp32 dequant, B A accumulated in fp32, the sum
+ * rounded once to fp32 (one FMA) and then, for NF4_BF16, to bf16 (nearest,
+ * ties to even).
+ *   w          block_size 64; cols % 64 == 0, rows % 8 == 0.
+ *   A, B       [r, K] and [N, r] bf16; 8 <= r <= 256, r % 8 == 0.
+ *   out_dtype  NF4_BF16 or NF4_F32; out has rows * cols elements, written.
+ *   workspace  >= nf4_workspace_bytes(NF4_OP_MERGE, 0, N, K, r, 64, dq): the
+ *              status word only.
+ * Same validation, ownership and error rules as the linear entry points.
+ */
+NF4_API nf4_status nf4_merge(const nf4_weight* w, const void* A, const void* B, int r, float alpha,
+                             int out_dtype, void* out, void* workspace, size_t ws_bytes,
+                             void* stream);
 
 #ifdef __cplusplus
 }

@@ -83,7 +83,7 @@ double g_prof_ms[nf4::kNumKernelIds];
 
 const char* const kKernelNames[nf4::kNumKernelIds] = {
     "nf4_quantize", "nf4_double_quant", "nf4_dequantize", "adapter_gemm",
-    "adapter_finalize", "fused_nf4_gemm_fwd", "fused_nf4_gemm_dx", "nf4_gemv", "nf4_gemv_reduce"};
+    "fused_nf4_gemm_fwd", "fused_nf4_gemm_dx", "nf4_gemv", "nf4_merge"};
 
 cudaEvent_t prof_event() {
   if (!g_prof_free.empty()) {
@@ -197,6 +197,7 @@ size_t nf4_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r, int b
     case NF4_OP_DEQUANTIZE: return 0;
     case NF4_OP_LINEAR_FWD: return nf4::kWsHeader + nf4::linear_workspace_bytes(false, M, N, K, r);
     case NF4_OP_LINEAR_BWD: return nf4::kWsHeader + nf4::linear_workspace_bytes(true, M, N, K, r);
+    case NF4_OP_MERGE: return nf4::kWsHeader;
     default: return 0;
   }
 }
@@ -355,6 +356,26 @@ nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const
   cudaError_t e = nf4::launch_linear_bwd(a, sm_count(), static_cast<cudaStream_t>(stream),
                                          &launches);
   if (e == cudaErrorNotSupported) { g_launches += launches; return NF4_ERR_UNSUPPORTED; }
+  return finish(e, launches);
+}
+
+nf4_status nf4_merge(const nf4_weight* w, const void* A, const void* B, int r, float alpha,
+                     int out_dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  // the linear checks with a stand-in x (the merge has no activations)
+  nf4_status s = check_linear(w, A, 1, A, B, r, alpha, NF4_BF16);
+  if (s != NF4_OK) return s;
+  if (out_dtype != NF4_BF16 && out_dtype != NF4_F32) {
+    return out_dtype == NF4_F16 ? NF4_ERR_UNSUPPORTED : NF4_ERR_INVALID_ARG;
+  }
+  if (out == nullptr) return NF4_ERR_INVALID_ARG;
+  if (!aligned16(out)) return NF4_ERR_ALIGNMENT;
+  if (workspace == nullptr || !aligned16(workspace)) return NF4_ERR_WORKSPACE;
+  if (ws_bytes < nf4_workspace_bytes(NF4_OP_MERGE, 0, w->rows, w->cols, r, 64, w->double_quant))
+    return NF4_ERR_WORKSPACE;
+  uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + nf4::kWsStatus);
+  int launches = 0;
+  const cudaError_t e = nf4::launch_merge(*w, A, B, r, alpha, out_dtype == NF4_F32 ? 1 : 0, out,
+                                          status, static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches);
 }
 

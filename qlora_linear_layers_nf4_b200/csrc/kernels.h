@@ -50,12 +50,21 @@ size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, in
 // rows; bf16 or u8), optional 128-byte swizzle.  False if it cannot be encoded.
 bool make_map_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
                  uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+// The same for fp32 and bf16 elements with any swizzle mode.
+bool make_map_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                     uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+bool make_map_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                      uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 // Decode-shape forward (gemv.cu): one kernel for M <= 32 tokens.
 bool decode_supported(int64_t M, int64_t N, int64_t K, int r);
 cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
+
+// Dense merge W' + s B A (merge.cu).
+cudaError_t launch_merge(const nf4_weight& w, const void* A, const void* B, int r, float alpha,
+                         int out_f32, void* out, uint32_t* status, cudaStream_t st, int* launches);
 
 }  // namespace nf4
 
@@ -67,11 +76,10 @@ enum KernelId {
   kKDoubleQuant,
   kKDequantize,
   kKAdapterGemm,
-  kKAdapterFinalize,
   kKFusedFwd,
   kKFusedDx,
   kKGemv,
-  kKGemvReduce,
+  kKMerge,
   kNumKernelIds
 };
 

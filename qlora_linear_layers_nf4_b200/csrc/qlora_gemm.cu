@@ -1146,6 +1146,24 @@ bool make_map_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, 
   return make_map(map, base, bf16, inner, outer, box_inner, box_outer, swizzle128);
 }
 
+bool make_map_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                     uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 4};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                      uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  return make_map(map, base, true, inner, outer, box_inner, box_outer, swizzle);
+}
+
 size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, int r) {
   (void)N;
   (void)K;

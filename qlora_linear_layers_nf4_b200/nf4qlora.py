@@ -21,13 +21,14 @@ STATUS_NAMES = {
     7: "NF4_ERR_NONFINITE", 8: "NF4_ERR_TIMEOUT",
 }
 NF4_F32, NF4_BF16, NF4_F16 = 0, 1, 2
-OP_QUANTIZE, OP_DEQUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD = 0, 1, 2, 3
+OP_QUANTIZE, OP_DEQUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD, OP_MERGE = 0, 1, 2, 3, 4
 
 EXPORTED = (
     "nf4_status_string", "nf4_version", "nf4_codebook", "nf4_launch_count",
     "nf4_profile_begin", "nf4_profile_end", "nf4_profile_kernel_count", "nf4_kernel_name",
     "nf4_profile_get", "nf4_workspace_bytes", "nf4_read_status", "nf4_quantize",
     "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "nf4_quantize_noalloc",
+    "nf4_merge",
 )
 
 
@@ -95,6 +96,8 @@ def lib() -> ctypes.CDLL:
     L.qlora_linear_bwd.argtypes = [ctypes.POINTER(CWeight), vp, i64, vp, vp, i32, f32, i32, vp, vp,
                                    vp, vp, vp, vp, sz, vp]
     L.qlora_linear_bwd.restype = i32
+    L.nf4_merge.argtypes = [ctypes.POINTER(CWeight), vp, vp, i32, f32, i32, vp, vp, sz, vp]
+    L.nf4_merge.restype = i32
     _lib = L
     return L
 
@@ -242,6 +245,23 @@ def dequantize(q: QuantizedWeight, out_dtype: str = "f32", stream=None):
     out = torch.empty((q.rows, q.cols), dtype=dt[1], device=q.device)
     cw = q.c_struct()
     _check(lib().nf4_dequantize(ctypes.byref(cw), dt[0], _ptr(out), _stream(stream)), "nf4_dequantize")
+    return out
+
+
+def merge(q: QuantizedWeight, A, B, alpha: float, out_dtype: str = "bf16", out=None,
+          workspace: Workspace | None = None, stream=None):
+    """Dense merged weight dequant(W) + (alpha/r) B A, [rows, cols] in bf16 or f32."""
+    import torch
+    dt = {"f32": (NF4_F32, torch.float32), "bf16": (NF4_BF16, torch.bfloat16)}[out_dtype]
+    r = A.shape[0]
+    if out is None:
+        out = torch.empty((q.rows, q.cols), dtype=dt[1], device=q.device)
+    ws = workspace if workspace is not None else Workspace(q.device)
+    need = lib().nf4_workspace_bytes(OP_MERGE, 0, q.rows, q.cols, r, q.block_size, int(q.double_quant))
+    buf = ws.get(need)
+    cw = q.c_struct()
+    _check(lib().nf4_merge(ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha), dt[0], _ptr(out),
+                           _ptr(buf), buf.numel(), _stream(stream)), "nf4_merge")
     return out
 
 
