@@ -229,7 +229,7 @@ NF4_API nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out,
  *                  K % 64 == 0, N % 8 == 0.
  *   x              [M, K] compute_dtype; M >= 1.
  *   A, B           [r, K] and [N, r] compute_dtype; 8 <= r <= 256, r % 8 == 0.
- *   compute_dtype  NF4_BF16 (NF4_F16 / NF4_F32 give NF4_ERR_UNSUPPORTED).
+ *   compute_dtype  NF4_BF16 or NF4_F16 (NF4_F32 gives NF4_ERR_UNSUPPORTED).
  *   bias           [N] compute_dtype, or NULL.
  *   y              [M, N] compute_dtype, written.
  *   t_out          [M, r] compute_dtype, or NULL: when given, receives

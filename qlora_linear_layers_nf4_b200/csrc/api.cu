@@ -49,8 +49,8 @@ nf4_status check_linear(const nf4_weight* w, const void* x, int64_t M, const voi
     return NF4_ERR_INVALID_ARG;
   }
   if (!(alpha == alpha) || r < 8 || r > 256 || (r % 8) != 0) return NF4_ERR_INVALID_ARG;
-  if (compute_dtype != NF4_BF16) {
-    if (compute_dtype == NF4_F16 || compute_dtype == NF4_F32) return NF4_ERR_UNSUPPORTED;
+  if (compute_dtype != NF4_BF16 && compute_dtype != NF4_F16) {
+    if (compute_dtype == NF4_F32) return NF4_ERR_UNSUPPORTED;
     return NF4_ERR_INVALID_ARG;
   }
   if (M < 1 || w->rows < 1 || w->cols < 1) return NF4_ERR_SHAPE;
@@ -304,6 +304,7 @@ nf4_status qlora_linear_fwd(const nf4_weight* w, const void* x, int64_t M, const
   a.K = w->cols;
   a.r = r;
   a.s = alpha / float(r);
+  a.f16 = compute_dtype == NF4_F16 ? 1 : 0;
   a.x = x;
   a.A = A;
   a.B = B;
@@ -341,6 +342,7 @@ nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const
   a.K = w->cols;
   a.r = r;
   a.s = alpha / float(r);
+  a.f16 = compute_dtype == NF4_F16 ? 1 : 0;
   a.x = x;
   a.A = A;
   a.B = B;

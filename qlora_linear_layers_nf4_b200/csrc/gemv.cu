@@ -21,6 +21,7 @@
 //     term, bias and bf16 rounding are applied in that reduction.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kernels.h"
 #include "nf4_common.cuh"
@@ -86,13 +87,37 @@ __host__ __device__ inline GemvLayout gemv_layout(int bps, int np, int r_pad, in
   return L;
 }
 
+template <bool F16>
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                           uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  if (F16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+// One 2-byte element of the compute type (f16 or bf16) to and from fp32.
+template <bool F16>
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) {
+  if (F16) return __half2float(*reinterpret_cast<const __half*>(&v));
+  return __bfloat162float(v);
+}
+template <bool F16>
+__device__ __forceinline__ __nv_bfloat16 from_f32(float v) {
+  if (F16) {
+    const __half h = __float2half_rn(v);
+    return *reinterpret_cast<const __nv_bfloat16*>(&h);
+  }
+  return __float2bfloat16_rn(v);
 }
 
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
@@ -130,7 +155,7 @@ __device__ __forceinline__ void frag_pair(const uint4& lo, const uint4& hi, int 
   }
 }
 
-template <int NT8>
+template <int NT8, bool F16>
 __global__ void __launch_bounds__(kGvThreads, 1)
     nf4_gemv(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
              const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -204,8 +229,13 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   // unscaled levels, one copy per lane so 32 lanes never share a bank.
   for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
     const int e = i >> 5;
-    const __nv_bfloat162 h = __floats2bfloat162_rn(level(e >> 4), level(e & 15));
-    lut[i] = *reinterpret_cast<const uint32_t*>(&h);
+    if (F16) {
+      const __half2 h = __floats2half2_rn(level(e >> 4), level(e & 15));
+      lut[i] = *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(level(e >> 4), level(e & 15));
+      lut[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
   }
   {
     const int row = threadIdx.x & (kGvRows - 1);
@@ -257,7 +287,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         for (int i = 0; i < 4; ++i) {
           uint32_t b0, b1;
           frag_pair(xl, xh, i, b0, b1);
-          mma_16816(blk, afr[i], b0, b1);
+          mma_16816<F16>(blk, afr[i], b0, b1);
         }
         acc[t][0] = fmaf(s0, blk[0], acc[t][0]);
         acc[t][1] = fmaf(s0, blk[1], acc[t][1]);
@@ -291,7 +321,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
           for (int i = 0; i < 4; ++i) {
             uint32_t b0, b1;
             frag_pair(xl, xh, i, b0, b1);
-            mma_16816(acc[t], afr[i], b0, b1);
+            mma_16816<F16>(acc[t], afr[i], b0, b1);
           }
         }
       }
@@ -334,8 +364,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       const __nv_bfloat16* b0row = bs + r0 * p.r;
       const __nv_bfloat16* b8row = bs + (r0 + 8) * p.r;
       for (int j = 0; j < p.r; ++j) {
-        const float bv0 = p.s * __bfloat162float(b0row[j]);
-        const float bv8 = p.s * __bfloat162float(b8row[j]);
+        const float bv0 = p.s * to_f32<F16>(b0row[j]);
+        const float bv8 = p.s * to_f32<F16>(b8row[j]);
 #pragma unroll
         for (int t = 0; t < NT8; ++t) {
           const float t0 = tpart[j * NP + 8 * t + 2 * q];
@@ -366,7 +396,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       const uint32_t off = uint32_t((j * NP + m) * 4);
       float v = 0.0f;
       for (int sl = 0; sl < p.slices; ++sl) v += ld_shared_cluster_f32(mapa_shared(tbase + off, uint32_t(sl)));
-      p.t_out[i] = __float2bfloat16_rn(p.s * v);
+      p.t_out[i] = from_f32<F16>(p.s * v);
     }
   }
 
@@ -389,12 +419,12 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       v.z += w.z;
       v.w += w.w;
     }
-    const float bias = p.bias != nullptr ? __bfloat162float(p.bias[n]) : 0.0f;
+    const float bias = p.bias != nullptr ? to_f32<F16>(p.bias[n]) : 0.0f;
     const float vals[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int m = 4 * mq + e;
-      if (m < p.M) p.y[int64_t(m) * p.N + n] = __float2bfloat16_rn(vals[e] + bias);
+      if (m < p.M) p.y[int64_t(m) * p.N + n] = from_f32<F16>(vals[e] + bias);
     }
   }
   cluster_sync();
@@ -467,23 +497,22 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   cfg.numAttrs = 1;
   // The shared-memory opt-in is set once per instantiation (the maximum the
   // decode path can ask for), not on every call.
-  static bool attr_done[3] = {false, false, false};
-  const int slot = nt8 == 1 ? 0 : (nt8 == 2 ? 1 : 2);
+  auto kernel_for = [](int n8, bool f16) {
+    if (f16) return n8 == 1 ? nf4_gemv<1, true> : (n8 == 2 ? nf4_gemv<2, true> : nf4_gemv<4, true>);
+    return n8 == 1 ? nf4_gemv<1, false> : (n8 == 2 ? nf4_gemv<2, false> : nf4_gemv<4, false>);
+  };
+  static bool attr_done[6] = {false, false, false, false, false, false};
+  const int slot = (nt8 == 1 ? 0 : (nt8 == 2 ? 1 : 2)) + (a.f16 ? 3 : 0);
+  auto* kernel = kernel_for(nt8, a.f16 != 0);
   cudaError_t e = cudaSuccess;
   if (!attr_done[slot]) {
     const int max_smem = 190 * 1024;   // + the 32 KB static lookup table
-    e = slot == 0 ? cudaFuncSetAttribute(nf4_gemv<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem)
-      : slot == 1 ? cudaFuncSetAttribute(nf4_gemv<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem)
-                  : cudaFuncSetAttribute(nf4_gemv<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     if (e != cudaSuccess) return e;
     attr_done[slot] = true;
   }
   NF4_PROF_BEGIN(st, kKGemv);
-  switch (nt8) {
-    case 1: e = cudaLaunchKernelEx(&cfg, nf4_gemv<1>, tc, tx, ta, tb, p); break;
-    case 2: e = cudaLaunchKernelEx(&cfg, nf4_gemv<2>, tc, tx, ta, tb, p); break;
-    default: e = cudaLaunchKernelEx(&cfg, nf4_gemv<4>, tc, tx, ta, tb, p); break;
-  }
+  e = cudaLaunchKernelEx(&cfg, kernel, tc, tx, ta, tb, p);
   NF4_PROF_END(st, kKGemv);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;

@@ -28,7 +28,8 @@ struct LinearArgs {
   int64_t M, N, K;
   int r;
   float s;                 // alpha / r
-  const void* x;           // [M, K] bf16
+  int f16;                 // compute type f16 (else bf16): x, A, B, bias, dy, y, dx, T, U
+  const void* x;           // [M, K] bf16 / f16
   const void* A;           // [r, K] bf16
   const void* B;           // [N, r] bf16
   const void* bias;        // [N] bf16 or null

@@ -44,22 +44,34 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+__device__ __forceinline__ uint32_t f16x2_rn(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// Two values rounded (nearest, ties to even) to the compute type: f16 or bf16.
+__device__ __forceinline__ uint32_t pack2(bool f16, float lo, float hi) {
+  return f16 ? f16x2_rn(lo, hi) : bf16x2_rn(lo, hi);
+}
+__device__ __forceinline__ float2 unpack2(bool f16, uint32_t w) {
+  return f16 ? __half22float2(*reinterpret_cast<const __half2*>(&w))
+             : __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+}
 
-// The sixteen dequantized values of one block, bf16(L[c] * scale) with the
-// fp32 product rounded to nearest even, split into byte planes so a lookup is
-// a register byte-permute: lo[q] holds the low bytes of entries 4q..4q+3,
-// hi[q] their high bytes.
+// The sixteen dequantized values of one block, bf16(L[c] * scale) (or f16)
+// with the fp32 product rounded to nearest even, split into byte planes so a
+// lookup is a register byte-permute: lo[q] holds the low bytes of entries
+// 4q..4q+3, hi[q] their high bytes.
 struct BlockTable {
   uint32_t lo[4];
   uint32_t hi[4];
 };
 
-__device__ __forceinline__ BlockTable make_table(float scale) {
+__device__ __forceinline__ BlockTable make_table(float scale, bool f16) {
   uint32_t p[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    p[j] = bf16x2_rn(__fmul_rn(__uint_as_float(level_bits(2 * j)), scale),
-                     __fmul_rn(__uint_as_float(level_bits(2 * j + 1)), scale));
+    p[j] = pack2(f16, __fmul_rn(__uint_as_float(level_bits(2 * j)), scale),
+                 __fmul_rn(__uint_as_float(level_bits(2 * j + 1)), scale));
   }
   BlockTable t;
 #pragma unroll
@@ -84,10 +96,10 @@ __device__ __forceinline__ uint2 decode4(uint32_t w, const BlockTable& t) {
 // Dequantize one 64-element block (32 code bytes at `codes`, smem) into row
 // `row` of a 128-byte-swizzled bf16 tile at `tile` (smem).
 __device__ __forceinline__ void dequant_row(const uint8_t* codes, float scale, uint8_t* tile,
-                                            uint32_t row) {
+                                            uint32_t row, bool f16) {
   const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
   const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
-  const BlockTable t = make_table(scale);
+  const BlockTable t = make_table(scale, f16);
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -100,9 +112,9 @@ __device__ __forceinline__ void dequant_row(const uint8_t* codes, float scale, u
 // Half a block (32 elements, 16 code bytes at `codes`, smem) into 16-byte
 // chunks 4*half .. 4*half+3 of row `row` of a 128-byte-swizzled bf16 tile.
 __device__ __forceinline__ void dequant_half_row(const uint8_t* codes, float scale, uint8_t* tile,
-                                                 uint32_t row, uint32_t half) {
+                                                 uint32_t row, uint32_t half, bool f16) {
   const uint4 c = *reinterpret_cast<const uint4*>(codes);
-  const BlockTable t = make_table(scale);
+  const BlockTable t = make_table(scale, f16);
   const uint32_t words[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -145,10 +157,11 @@ struct FusedParams {
   int out_cols;      // N (fwd) or K (dx)
   int kb_per_row;    // K / 64 NF4 blocks per W row
   int double_quant;
+  int f16;           // operands and outputs in f16 (else bf16)
   const uint8_t* absmax_q;
   const float* absmax;
   const float* absmax_scale;
-  const __nv_bfloat16* bias;
+  const __nv_bfloat16* bias;   // 2-byte elements of the compute type
   __nv_bfloat16* out;
   uint32_t* status;
 };
@@ -250,7 +263,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, kTileN, false, MODE == kDx);
+      const uint32_t idesc = idesc_f32acc(128, kTileN, false, MODE == kDx, p.f16 != 0);
       bool ok = true;
       int issued = 0;
       for (int it = 0; it < total_steps && ok; ++it) {
@@ -316,7 +329,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const float scale = next_scale;
       if (it + 1 < p.main_steps) next_scale = scale_at(it + 1);
       if (!__all_sync(0xffffffffu, mbar_wait(&sh->full[s], ph, abort_flag, p.status))) break;
-      dequant_row(stage_c(s) + t * 32, scale, stage_b(s), uint32_t(t));
+      dequant_row(stage_c(s) + t * 32, scale, stage_b(s), uint32_t(t), p.f16 != 0);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->bready[s]);
@@ -342,18 +355,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
               float f[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
+              const bool f16 = p.f16 != 0;
               if (MODE == kFwd && p.bias != nullptr) {
                 const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
-                const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
+                const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                  const float2 bf = __bfloat1622float2(b2[e]);
+                  const float2 bf = unpack2(f16, bw[e]);
                   f[2 * e] += bf.x;
                   f[2 * e + 1] += bf.y;
                 }
               }
-              const uint4 o = make_uint4(bf16x2_rn(f[0], f[1]), bf16x2_rn(f[2], f[3]),
-                                         bf16x2_rn(f[4], f[5]), bf16x2_rn(f[6], f[7]));
+              const uint4 o = make_uint4(pack2(f16, f[0], f[1]), pack2(f16, f[2], f[3]),
+                                         pack2(f16, f[4], f[5]), pack2(f16, f[6], f[7]));
               *reinterpret_cast<uint4*>(p.out + int64_t(row) * p.out_cols + col) = o;
             }
           }
@@ -566,7 +580,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     }
     // ---------------- MMA issuer (leader CTA only)
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_bf16_f32(256, kTileN, false, MODE == kDx);
+      const uint32_t idesc = idesc_f32acc(256, kTileN, false, MODE == kDx, p.f16 != 0);
       bool ok = true;
       int issued = 0;
       for (int it = 0; it < total_steps && ok; ++it) {
@@ -654,7 +668,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       if (ok && j == 0) ok = mbar_wait(&sh->cfull[c], (g / kP2CodeSlots) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       dequant_half_row(code_slot(c) + code_offset<MODE>(uint32_t(row), half, uint32_t(j)), scale,
-                       stage_b(s), uint32_t(row), half);
+                       stage_b(s), uint32_t(row), half, p.f16 != 0);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -683,18 +697,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
               float f[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
+              const bool f16 = p.f16 != 0;
               if (MODE == kFwd && p.bias != nullptr) {
                 const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
-                const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
+                const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                  const float2 bf = __bfloat1622float2(b2[e]);
+                  const float2 bf = unpack2(f16, bw[e]);
                   f[2 * e] += bf.x;
                   f[2 * e + 1] += bf.y;
                 }
               }
-              const uint4 o = make_uint4(bf16x2_rn(f[0], f[1]), bf16x2_rn(f[2], f[3]),
-                                         bf16x2_rn(f[4], f[5]), bf16x2_rn(f[6], f[7]));
+              const uint4 o = make_uint4(pack2(f16, f[0], f[1]), pack2(f16, f[2], f[3]),
+                                         pack2(f16, f[4], f[5]), pack2(f16, f[6], f[7]));
               *reinterpret_cast<uint4*>(p.out + int64_t(grow) * p.out_cols + col) = o;
             }
           }
@@ -733,7 +748,8 @@ struct AdapterParams {
   int slices;
   int a_mn;          // A operand MN-major
   int b_mn;          // B operand MN-major
-  int kind;          // 0: bf16(scale * D) [Mo][r]; 1: fp32 D [Mo][r]; 2: fp32 D^T [r][Mo]
+  int kind;          // 0: bf16/f16(scale * D) [Mo][r]; 1: fp32 D [Mo][r]; 2: fp32 D^T [r][Mo]
+  int f16;           // operands and the kind-0 output in f16 (else bf16)
   float scale;
   __nv_bfloat16* out_bf16;
   float* out_f32;
@@ -743,8 +759,8 @@ struct AdapterParams {
 // Write 4 consecutive output columns (col .. col+3 < r) of one row.
 __device__ __forceinline__ void adapter_store4(const AdapterParams& p, int row, int col, float4 v) {
   if (p.kind == 0) {
-    const uint2 o = make_uint2(bf16x2_rn(v.x * p.scale, v.y * p.scale),
-                               bf16x2_rn(v.z * p.scale, v.w * p.scale));
+    const uint2 o = make_uint2(pack2(p.f16 != 0, v.x * p.scale, v.y * p.scale),
+                               pack2(p.f16 != 0, v.z * p.scale, v.w * p.scale));
     *reinterpret_cast<uint2*>(p.out_bf16 + int64_t(row) * p.r + col) = o;
   } else if (p.kind == 1) {
     *reinterpret_cast<float4*>(p.out_f32 + int64_t(row) * p.r + col) = v;
@@ -845,7 +861,7 @@ __global__ void __launch_bounds__(kAdThreads, 1)
   if (warp == 0) {
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, p.NP, p.a_mn != 0, p.b_mn != 0);
+      const uint32_t idesc = idesc_f32acc(128, p.NP, p.a_mn != 0, p.b_mn != 0, p.f16 != 0);
       bool ok = true;
       int issued = 0;
       for (int i = 0; i < nsteps; ++i) {
@@ -1043,14 +1059,15 @@ cudaError_t set_attrs() {
   return e;
 }
 
-// One rank-r product through adapter_gemm + adapter_finalize.
+// One rank-r product through adapter_gemm.
 //   a_mn/b_mn: operand majorness; a_base/b_base: matrices as [outer][inner].
 struct AdapterJob {
   const void* a; uint64_t a_inner, a_outer; bool a_mn;
   const void* b; uint64_t b_inner, b_outer; bool b_mn;
   int64_t Mo, red;
   int r;
-  int kind;          // see adapter_finalize
+  int kind;          // see AdapterParams::kind
+  int f16;           // operands (and the kind-0 output) in f16
   float scale;
   __nv_bfloat16* out_bf16;
   float* out_f32;
@@ -1076,6 +1093,7 @@ cudaError_t run_adapter(const AdapterJob& j, uint32_t* status, int sms, cudaStre
   p.a_mn = j.a_mn;
   p.b_mn = j.b_mn;
   p.kind = j.kind;
+  p.f16 = j.f16;
   p.scale = j.scale;
   p.out_bf16 = j.out_bf16;
   p.out_f32 = j.out_f32;
@@ -1116,6 +1134,7 @@ FusedParams fused_params(const LinearArgs& a, int mode) {
   p.out_cols = mode == kFwd ? int(a.N) : int(a.K);
   p.kb_per_row = int(a.K / 64);
   p.double_quant = a.w->double_quant;
+  p.f16 = a.f16;
   p.absmax_q = a.w->absmax_q;
   p.absmax = a.w->absmax;
   p.absmax_scale = a.w->absmax_scale;
@@ -1135,7 +1154,7 @@ cudaError_t forward_adapter_T(const LinearArgs& a, __nv_bfloat16* T, int sms, cu
   AdapterJob j{};
   j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = false;
   j.b = a.A; j.b_inner = a.K; j.b_outer = a.r; j.b_mn = false;
-  j.Mo = a.M; j.red = a.K; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = T;
+  j.Mo = a.M; j.red = a.K; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = T; j.f16 = a.f16;
   return run_adapter(j, a.status, sms, st, launches);
 }
 
@@ -1226,7 +1245,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     AdapterJob j{};
     j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = false;
     j.b = a.B; j.b_inner = a.r; j.b_outer = a.N; j.b_mn = true;
-    j.Mo = a.M; j.red = a.N; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = U;
+    j.Mo = a.M; j.red = a.N; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = U; j.f16 = a.f16;
     e = run_adapter(j, a.status, sms, st, launches);
     if (e != cudaSuccess) return e;
   }
@@ -1235,7 +1254,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     AdapterJob j{};
     j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = true;
     j.b = T; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
-    j.Mo = a.N; j.red = a.M; j.r = a.r; j.kind = 1; j.scale = 1.0f; j.out_f32 = a.dB;
+    j.Mo = a.N; j.red = a.M; j.r = a.r; j.kind = 1; j.scale = 1.0f; j.out_f32 = a.dB; j.f16 = a.f16;
     e = run_adapter(j, a.status, sms, st, launches);
     if (e != cudaSuccess) return e;
   }
@@ -1244,7 +1263,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     AdapterJob j{};
     j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = true;
     j.b = U; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
-    j.Mo = a.K; j.red = a.M; j.r = a.r; j.kind = 2; j.scale = 1.0f; j.out_f32 = a.dA;
+    j.Mo = a.K; j.red = a.M; j.r = a.r; j.kind = 2; j.scale = 1.0f; j.out_f32 = a.dA; j.f16 = a.f16;
     e = run_adapter(j, a.status, sms, st, launches);
     if (e != cudaSuccess) return e;
   }

@@ -344,14 +344,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor for kind::f16: bf16 x bf16 -> fp32, M x N, majors.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
-                                                       bool b_mn_major) {
-  return (1u << 4)                      // D format: f32
-         | (1u << 7)                    // A format: bf16
-         | (1u << 10)                   // B format: bf16
+// Instruction descriptor for kind::f16 with fp32 accumulation, M x N, operand
+// majors; A and B are both bf16 (format 1) or both f16 (format 0).
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                     bool f16_operands) {
+  return (1u << 4)                                     // D format: f32
+         | (uint32_t(f16_operands ? 0u : 1u) << 7)     // A format
+         | (uint32_t(f16_operands ? 0u : 1u) << 10)    // B format
          | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) |
          (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
+                                                       bool b_mn_major) {
+  return idesc_f32acc(M, N, a_mn_major, b_mn_major, false);
 }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` inside a 128-byte-swizzled

@@ -265,20 +265,34 @@ def merge(q: QuantizedWeight, A, B, alpha: float, out_dtype: str = "bf16", out=N
     return out
 
 
+def _compute_dtype(x):
+    """The C ABI's compute type for activations of x's dtype (bf16 or f16)."""
+    import torch
+    if x.dtype == torch.bfloat16:
+        return NF4_BF16
+    if x.dtype == torch.float16:
+        return NF4_F16
+    raise TypeError(f"compute dtype must be bfloat16 or float16, got {x.dtype}")
+
+
 def linear_fwd(q: QuantizedWeight, x, A, B, alpha: float, bias=None, want_t: bool = True,
                out=None, t_out=None, workspace: Workspace | None = None, stream=None):
-    """y = x W'^T + (alpha/r) (x A^T) B^T (+ bias); returns (y, T or None)."""
+    """y = x W'^T + (alpha/r) (x A^T) B^T (+ bias); returns (y, T or None).
+
+    x, A, B (and bias) share one compute dtype, bfloat16 or float16; y and T
+    come back in it."""
     import torch
+    dt = _compute_dtype(x)
     M = x.shape[0]
     r = A.shape[0]
-    y = out if out is not None else torch.empty((M, q.rows), dtype=torch.bfloat16, device=x.device)
+    y = out if out is not None else torch.empty((M, q.rows), dtype=x.dtype, device=x.device)
     if want_t and t_out is None:
-        t_out = torch.empty((M, r), dtype=torch.bfloat16, device=x.device)
+        t_out = torch.empty((M, r), dtype=x.dtype, device=x.device)
     ws = workspace or default_workspace(x.device)
     buf = ws.get(workspace_bytes(OP_LINEAR_FWD, M, q.rows, q.cols, r, q.block_size, q.double_quant))
     cw = q.c_struct()
     st = lib().qlora_linear_fwd(ctypes.byref(cw), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
-                                NF4_BF16, _ptr(bias), _ptr(y), _ptr(t_out), _ptr(buf), buf.numel(),
+                                dt, _ptr(bias), _ptr(y), _ptr(t_out), _ptr(buf), buf.numel(),
                                 _stream(stream))
     _check(st, "qlora_linear_fwd")
     return y, t_out
@@ -286,19 +300,20 @@ def linear_fwd(q: QuantizedWeight, x, A, B, alpha: float, bias=None, want_t: boo
 
 def linear_bwd(q: QuantizedWeight, x, A, B, alpha: float, dy, t=None, want_dx: bool = True,
                dA=None, dB=None, dx=None, workspace: Workspace | None = None, stream=None):
-    """Adapter backward; returns (dA fp32 [r,K], dB fp32 [N,r], dx bf16 [M,K] or None)."""
+    """Adapter backward; returns (dA fp32 [r,K], dB fp32 [N,r], dx [M,K] in x's dtype or None)."""
     import torch
+    dt = _compute_dtype(x)
     M = x.shape[0]
     r = A.shape[0]
     dA = dA if dA is not None else torch.empty((r, q.cols), dtype=torch.float32, device=x.device)
     dB = dB if dB is not None else torch.empty((q.rows, r), dtype=torch.float32, device=x.device)
     if want_dx and dx is None:
-        dx = torch.empty((M, q.cols), dtype=torch.bfloat16, device=x.device)
+        dx = torch.empty((M, q.cols), dtype=x.dtype, device=x.device)
     ws = workspace or default_workspace(x.device)
     buf = ws.get(workspace_bytes(OP_LINEAR_BWD, M, q.rows, q.cols, r, q.block_size, q.double_quant))
     cw = q.c_struct()
     st = lib().qlora_linear_bwd(ctypes.byref(cw), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
-                                NF4_BF16, _ptr(dy), _ptr(t), _ptr(dA), _ptr(dB), _ptr(dx),
+                                dt, _ptr(dy), _ptr(t), _ptr(dA), _ptr(dB), _ptr(dx),
                                 _ptr(buf), buf.numel(), _stream(stream))
     _check(st, "qlora_linear_bwd")
     return dA, dB, dx

@@ -102,8 +102,11 @@ def draw_linear(case: LinearCase, m: int | None = None) -> LinearInputs:
     bias = None
     if case.with_bias:
         bias = to_bf16_bits(rng.standard_normal(case.n, dtype=np.float32) * np.float32(0.1))
-    return LinearInputs(case, w.astype(np.float32), to_bf16_bits(x), to_bf16_bits(a),
-                        to_bf16_bits(b), to_bf16_bits(dy), bias)
+    out = LinearInputs(case, w.astype(np.float32), to_bf16_bits(x), to_bf16_bits(a),
+                       to_bf16_bits(b), to_bf16_bits(dy), bias)
+    # the fp32 draws themselves, for rounding to another compute dtype (f16)
+    out.extra["f32"] = {"x": x, "a": a, "b": b, "dy": dy}
+    return out
 
 
 def draw_weight(shape, seed: int, sigma: float = W_SIGMA) -> np.ndarray:

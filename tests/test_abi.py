@@ -111,7 +111,7 @@ def test_linear_host_validation():
     assert _fwd(_cw(), r=4) == 1                  # r < 8
     assert _fwd(_cw(), r=12) == 1                 # r % 8
     assert _fwd(_cw(), r=512) == 1
-    assert _fwd(_cw(), dtype=2) == 4              # F16 compute: not in this build
+    assert _fwd(_cw(), dtype=2, wsb=0) == 5       # F16 compute passes the dtype check
     assert _fwd(_cw(), dtype=0) == 4              # F32 compute: not in this build
     assert _fwd(_cw(), dtype=9) == 1
     assert _fwd(_cw(), M=0) == 2
@@ -125,6 +125,21 @@ def test_linear_host_validation():
     st = L.qlora_linear_bwd(ctypes.byref(_cw()), FAKE, 16, FAKE, FAKE, 16, 32.0, 1, None, None,
                             FAKE, FAKE, None, FAKE, 1 << 40, None)
     assert st == 1                                # dy required
+
+
+def test_merge_host_validation():
+    L = Q.lib()
+    m = lambda cw, r=16, dt=1, out=FAKE, wsb=1 << 40: L.nf4_merge(
+        ctypes.byref(cw), FAKE, FAKE, r, 32.0, dt, out, FAKE, wsb, None)
+    assert m(_cw(), r=4) == 1                     # r < 8
+    assert m(_cw(), r=264) == 1                   # r > 256
+    assert m(_cw(), dt=2) == 4                    # f16 output: not in this build
+    assert m(_cw(), dt=7) == 1
+    assert m(_cw(), out=None) == 1
+    assert m(_cw(), out=FAKE + 2) == 3
+    assert m(_cw(cols=4000)) == 2                 # K % 64
+    assert m(_cw(bs=128)) == 4                    # block 64 only
+    assert m(_cw(), wsb=0) == 5
 
 
 def test_bucket_encoding_conditions():
