@@ -533,6 +533,36 @@ def measure_rows(args, dev, flush, pk, pk_kind, barrier):
     del qws
     torch.cuda.empty_cache()
 
+    # ---- the headline layer in the F16 compute dtype (same draws rounded to f16)
+    case = WL.PREFILL
+    inp = WL.draw_linear(case)
+    qf = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True)
+    d32 = inp.extra["f32"]
+    xf, Af, Bf, dyf = (torch.from_numpy(d32[k]).to(dev).half() for k in ("x", "a", "b", "dy"))
+    yf = torch.empty((case.m, case.n), dtype=torch.float16, device=dev)
+    Tf = torch.empty((case.m, case.r), dtype=torch.float16, device=dev)
+    dxf = torch.empty((case.m, case.k), dtype=torch.float16, device=dev)
+    dAf = torch.empty((case.r, case.k), dtype=torch.float32, device=dev)
+    dBf = torch.empty((case.n, case.r), dtype=torch.float32, device=dev)
+    wsf = Q.Workspace(dev)
+
+    def f16_step():
+        Q.linear_fwd(qf, xf, Af, Bf, case.alpha, out=yf, t_out=Tf, workspace=wsf)
+        Q.linear_bwd(qf, xf, Af, Bf, case.alpha, dyf, t=Tf, dA=dAf, dB=dBf, dx=dxf, workspace=wsf)
+
+    fsteps = max(3, min(args.steps, 20))
+    ms = time_steps(f16_step, fsteps, 3, flush=flush, barrier=barrier)
+    fl = linear_flops(case.m, case.n, case.k, case.r)
+    tf = fl * fsteps / (ms * 1e-3) / 1e12
+    out["prefill_11008x4096_M4096_f16_fwd_bwd"] = {
+        "TFLOP/s": tf, "ms_per_step": ms / fsteps,
+        "frac_f16_sustained": tf / (pk.get("bf16_tflops_sustained") or pk.get("bf16_tflops")),
+        "method": "eager steps, L2 flushed before each; the f16 dense peak equals the bf16 one"}
+    if wsf.read_status() != 0:
+        raise RuntimeError("device status reported an error in the f16 row")
+    del qf, xf, dyf, yf, dxf
+    torch.cuda.empty_cache()
+
     # ---- dense merge of the 11008x4096 layer with its r = 64 adapter (bf16 out),
     # 3 rotating outputs (270 MB)
     case = WL.PREFILL

@@ -211,6 +211,20 @@ NF4_API nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t co
                                         void* stream);
 
 /*
+ * nf4_quantize for a weight held in another element type: in_dtype NF4_F32
+ * (identical to nf4_quantize), NF4_BF16 or NF4_F16.  Each element is widened
+ * to fp32 exactly and quantized as nf4_quantize would quantize that fp32
+ * value (the pages' quantize_nf4 takes any tensor; a bf16 model's weights
+ * are quantized without an fp32 copy).  w is rows*cols elements of in_dtype,
+ * 16-byte aligned; every other argument, result and error as nf4_quantize.
+ * NF4_ERR_INVALID_ARG for any other in_dtype.
+ */
+NF4_API nf4_status nf4_quantize_typed(const void* w, int in_dtype, int64_t rows, int64_t cols,
+                                      int block_size, int double_quant, uint8_t* codes,
+                                      float* absmax, uint8_t* absmax_q, float* absmax_scale,
+                                      void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Dequantization (qlora-rs dequantize_nf4; "Honor compute_dtype
  * (BF16/F16/F32) in forward dequant").  out[e] = fp32(L[code_e] * scale_b)
  * as one fp32 product; NF4_BF16 / NF4_F16 store its round-to-nearest-even.

@@ -214,9 +214,13 @@ nf4_status nf4_read_status(void* workspace, void* stream) {
   return static_cast<nf4_status>(host);
 }
 
-nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int block_size,
-                        int double_quant, uint8_t* codes, float* absmax, uint8_t* absmax_q,
-                        float* absmax_scale, void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+nf4_status quantize_impl(const void* w, int in_dtype, int64_t rows, int64_t cols, int block_size,
+                         int double_quant, uint8_t* codes, float* absmax, uint8_t* absmax_q,
+                         float* absmax_scale, void* workspace, size_t ws_bytes, void* stream) {
   if (rows < 0 || cols < 0) return NF4_ERR_SHAPE;
   if (block_size <= 0 || (block_size % 2) != 0) return NF4_ERR_SHAPE;
   if (double_quant != 0 && double_quant != 1) return NF4_ERR_INVALID_ARG;
@@ -252,12 +256,32 @@ nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int block_si
     e = cudaMemsetAsync(gmax, 0, sizeof(uint32_t), st);
   }
   if (e == cudaSuccess)
-    e = nf4::launch_quantize(w, numel, block_size, codes, amax, status,
+    e = nf4::launch_quantize(w, in_dtype, numel, block_size, codes, amax, status,
                              double_quant ? gmax : nullptr, sms, st, &launches);
   if (e == cudaSuccess && double_quant)
     e = nf4::launch_double_quant(amax, numel / block_size, gmax, absmax_q, absmax_scale, sms, st,
                                  &launches);
   return finish(e, launches);
+}
+
+}  // namespace
+
+extern "C" {
+
+nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int block_size,
+                        int double_quant, uint8_t* codes, float* absmax, uint8_t* absmax_q,
+                        float* absmax_scale, void* workspace, size_t ws_bytes, void* stream) {
+  return quantize_impl(w, NF4_F32, rows, cols, block_size, double_quant, codes, absmax, absmax_q,
+                       absmax_scale, workspace, ws_bytes, stream);
+}
+
+nf4_status nf4_quantize_typed(const void* w, int in_dtype, int64_t rows, int64_t cols,
+                              int block_size, int double_quant, uint8_t* codes, float* absmax,
+                              uint8_t* absmax_q, float* absmax_scale, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  if (in_dtype != NF4_F32 && in_dtype != NF4_BF16 && in_dtype != NF4_F16) return NF4_ERR_INVALID_ARG;
+  return quantize_impl(w, in_dtype, rows, cols, block_size, double_quant, codes, absmax, absmax_q,
+                       absmax_scale, workspace, ws_bytes, stream);
 }
 
 nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out, void* stream) {

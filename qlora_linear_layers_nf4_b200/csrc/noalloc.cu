@@ -108,7 +108,7 @@ extern "C" nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t
     e = cudaMemsetAsync(gmax, 0, sizeof(uint32_t), st);   // the array keeps the last call's max
   }
   if (e == cudaSuccess)
-    e = launch_quantize(w, numel, block_size, codes, amax, /*status=*/nullptr,
+    e = launch_quantize(w, NF4_F32, numel, block_size, codes, amax, /*status=*/nullptr,
                         double_quant ? gmax : nullptr, sms, st, &launches);
   if (e == cudaSuccess && double_quant)
     e = launch_double_quant(amax, n_blocks, gmax, absmax_q, absmax_scale, sms, st, &launches);

@@ -175,7 +175,7 @@ struct FusedShared {
   uint32_t abort_flag;
 };
 
-template <int MODE>
+template <int MODE, bool F16>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a2,
                    const __grid_constant__ CUtensorMap tm_b2,
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_f32acc(128, kTileN, false, MODE == kDx, p.f16 != 0);
+      const uint32_t idesc = idesc_f32acc(128, kTileN, false, MODE == kDx, F16);
       bool ok = true;
       int issued = 0;
       for (int it = 0; it < total_steps && ok; ++it) {
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const float scale = next_scale;
       if (it + 1 < p.main_steps) next_scale = scale_at(it + 1);
       if (!__all_sync(0xffffffffu, mbar_wait(&sh->full[s], ph, abort_flag, p.status))) break;
-      dequant_row(stage_c(s) + t * 32, scale, stage_b(s), uint32_t(t), p.f16 != 0);
+      dequant_row(stage_c(s) + t * 32, scale, stage_b(s), uint32_t(t), F16);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->bready[s]);
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
               float f[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
-              const bool f16 = p.f16 != 0;
+              constexpr bool f16 = F16;
               if (MODE == kFwd && p.bias != nullptr) {
                 const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
                 const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
@@ -451,7 +451,7 @@ __device__ __forceinline__ uint32_t code_offset(uint32_t row, uint32_t half, uin
   return R * 64u + ((c ^ ((R >> 1) & 3u)) << 4);
 }
 
-template <int MODE>
+template <int MODE, bool F16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     fused_nf4_gemm_pair(const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_a2,
@@ -580,7 +580,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
     }
     // ---------------- MMA issuer (leader CTA only)
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_f32acc(256, kTileN, false, MODE == kDx, p.f16 != 0);
+      const uint32_t idesc = idesc_f32acc(256, kTileN, false, MODE == kDx, F16);
       bool ok = true;
       int issued = 0;
       for (int it = 0; it < total_steps && ok; ++it) {
@@ -668,7 +668,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       if (ok && j == 0) ok = mbar_wait(&sh->cfull[c], (g / kP2CodeSlots) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       dequant_half_row(code_slot(c) + code_offset<MODE>(uint32_t(row), half, uint32_t(j)), scale,
-                       stage_b(s), uint32_t(row), half, p.f16 != 0);
+                       stage_b(s), uint32_t(row), half, F16);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -697,7 +697,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
               float f[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
-              const bool f16 = p.f16 != 0;
+              constexpr bool f16 = F16;
               if (MODE == kFwd && p.bias != nullptr) {
                 const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
                 const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
@@ -1041,17 +1041,15 @@ bool g_attr_done = false;
 
 cudaError_t set_attrs() {
   if (g_attr_done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm<kFwd>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(kFusedSmem));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fused_nf4_gemm<kDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(kFusedSmem));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fused_nf4_gemm_pair<kFwd>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kP2Smem));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fused_nf4_gemm_pair<kDx>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kP2Smem));
+  const void* single[4] = {(const void*)fused_nf4_gemm<kFwd, false>, (const void*)fused_nf4_gemm<kDx, false>,
+                           (const void*)fused_nf4_gemm<kFwd, true>, (const void*)fused_nf4_gemm<kDx, true>};
+  const void* pair[4] = {(const void*)fused_nf4_gemm_pair<kFwd, false>, (const void*)fused_nf4_gemm_pair<kDx, false>,
+                         (const void*)fused_nf4_gemm_pair<kFwd, true>, (const void*)fused_nf4_gemm_pair<kDx, true>};
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+    e = cudaFuncSetAttribute(single[i], cudaFuncAttributeMaxDynamicSharedMemorySize, int(kFusedSmem));
+  for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+    e = cudaFuncSetAttribute(pair[i], cudaFuncAttributeMaxDynamicSharedMemorySize, int(kP2Smem));
   const size_t ad_smem = kAdStages * (kAdABytes + 256 * 128) + 1024 + 256;
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(adapter_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, int(ad_smem));
@@ -1216,10 +1214,12 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   NF4_PROF_BEGIN(st, kKFusedFwd);
   if (pair) {
     dim3 grid(unsigned(2 * cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kP2TileM)));
-    fused_nf4_gemm_pair<kFwd><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, p);
+    if (a.f16) fused_nf4_gemm_pair<kFwd, true><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, p);
+    else fused_nf4_gemm_pair<kFwd, false><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, p);
   } else {
     dim3 grid(unsigned(cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kTileM)));
-    fused_nf4_gemm<kFwd><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+    if (a.f16) fused_nf4_gemm<kFwd, true><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+    else fused_nf4_gemm<kFwd, false><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
   }
   NF4_PROF_END(st, kKFusedFwd);
   e = cudaGetLastError();
@@ -1282,10 +1282,12 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
   NF4_PROF_BEGIN(st, kKFusedDx);
   if (pair) {
     dim3 grid(unsigned(2 * cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kP2TileM)));
-    fused_nf4_gemm_pair<kDx><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, p);
+    if (a.f16) fused_nf4_gemm_pair<kDx, true><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, p);
+    else fused_nf4_gemm_pair<kDx, false><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, p);
   } else {
     dim3 grid(unsigned(cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kTileM)));
-    fused_nf4_gemm<kDx><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+    if (a.f16) fused_nf4_gemm<kDx, true><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+    else fused_nf4_gemm<kDx, false><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
   }
   NF4_PROF_END(st, kKFusedDx);
   e = cudaGetLastError();

@@ -8,6 +8,9 @@
 // shuffle-xor reduction over the bs/8 lanes that hold it.
 #include <algorithm>
 
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
 #include "nf4_common.cuh"
 #include "kernels.h"
 
@@ -107,10 +110,43 @@ __device__ __forceinline__ void cta_global_max(float v, uint32_t* gmax) {
   }
 }
 
-// G = block_size / 8 lanes per block (1, 2, 4, 8, 16 or 32).
-template <int G>
+// Input element types: fp32, or bf16 / f16 widened exactly to fp32.
+constexpr int kInF32 = 0;
+constexpr int kInBF16 = 1;
+constexpr int kInF16 = 2;
+
+__device__ __forceinline__ float2 widen2(int in, uint32_t v) {
+  if (in == kInBF16) return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
+  return __half22float2(*reinterpret_cast<const __half2*>(&v));
+}
+
+// Elements 8i .. 8i+7 of the input as two float4 (streaming loads).
+template <int IN>
+__device__ __forceinline__ void load8(const void* w, int64_t i, float4& a, float4& b) {
+  if (IN == kInF32) {
+    const float4* p = static_cast<const float4*>(w) + 2 * i;
+    a = __ldcs(p);
+    b = __ldcs(p + 1);
+  } else {
+    const uint4 u = __ldcs(static_cast<const uint4*>(w) + i);
+    const float2 e0 = widen2(IN, u.x), e1 = widen2(IN, u.y), e2 = widen2(IN, u.z), e3 = widen2(IN, u.w);
+    a = make_float4(e0.x, e0.y, e1.x, e1.y);
+    b = make_float4(e2.x, e2.y, e3.x, e3.y);
+  }
+}
+
+// One element of the input as fp32.
+template <int IN>
+__device__ __forceinline__ float load1(const void* w, int64_t e) {
+  if (IN == kInF32) return static_cast<const float*>(w)[e];
+  if (IN == kInBF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(w)[e]);
+  return __half2float(static_cast<const __half*>(w)[e]);
+}
+
+// G = block_size / 8 lanes per block (1, 2, 4, 8, 16 or 32); IN the input type.
+template <int G, int IN>
 __global__ void __launch_bounds__(256) quantize_vec_kernel(
-    const float4* __restrict__ w, int64_t n_words, int64_t blocks_per_row_unused,
+    const void* __restrict__ w, int64_t n_words, int64_t blocks_per_row_unused,
     uint32_t* __restrict__ codes, float* __restrict__ absmax, uint32_t* __restrict__ status,
     uint32_t* __restrict__ gmax) {
   (void)blocks_per_row_unused;
@@ -146,14 +182,8 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
     const int64_t i1 = i0 + stride;
     const bool v0 = i0 < n_words, v1 = i1 < n_words;
     float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), b0 = a0, a1 = a0, b1 = a0;
-    if (v0) {
-      a0 = __ldcs(w + 2 * i0);
-      b0 = __ldcs(w + 2 * i0 + 1);
-    }
-    if (v1) {
-      a1 = __ldcs(w + 2 * i1);
-      b1 = __ldcs(w + 2 * i1 + 1);
-    }
+    if (v0) load8<IN>(w, i0, a0, b0);
+    if (v1) load8<IN>(w, i1, a1, b1);
     bad |= (v0 && !finite8(a0, b0)) || (v1 && !finite8(a1, b1));
     float m0 = max_abs8(a0, b0), m1 = max_abs8(a1, b1);
 #pragma unroll
@@ -170,8 +200,9 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
 }
 
 // Any even block size: one thread per block, two passes over its elements.
+template <int IN>
 __global__ void __launch_bounds__(256) quantize_generic_kernel(
-    const float* __restrict__ w, int64_t n_blocks, int bs, uint8_t* __restrict__ codes,
+    const void* __restrict__ w, int64_t n_blocks, int bs, uint8_t* __restrict__ codes,
     float* __restrict__ absmax, uint32_t* __restrict__ status, uint32_t* __restrict__ gmax) {
   asm volatile("griddepcontrol.launch_dependents;");
   float cta_max = 0.0f;
@@ -181,14 +212,15 @@ __global__ void __launch_bounds__(256) quantize_generic_kernel(
     const int64_t blk = base + threadIdx.x;
     float m = 0.0f;
     if (blk < n_blocks) {
-      const float* p = w + blk * bs;
+      const int64_t e0 = blk * bs;
       for (int e = 0; e < bs; ++e) {
-        const float v = p[e];
+        const float v = load1<IN>(w, e0 + e);
         bad |= !isfinite(v);
         m = fmaxf(m, fabsf(v));
       }
       uint8_t* c = codes + blk * (bs / 2);
-      for (int e = 0; e < bs; e += 2) c[e / 2] = uint8_t(pair_byte(p[e], p[e + 1], m));
+      for (int e = 0; e < bs; e += 2)
+        c[e / 2] = uint8_t(pair_byte(load1<IN>(w, e0 + e), load1<IN>(w, e0 + e + 1), m));
       if (absmax != nullptr) absmax[blk] = m;
     }
     cta_max = fmaxf(cta_max, m);
@@ -333,31 +365,41 @@ int log2_exact(int v) {
 
 }  // namespace
 
-cudaError_t launch_quantize(const float* w, int64_t numel, int bs, uint8_t* codes,
-                            float* absmax_out, uint32_t* status, uint32_t* gmax, int sms,
-                            cudaStream_t stream, int* launches) {
+template <int IN>
+void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes, float* absmax_out,
+                           uint32_t* status, uint32_t* gmax, int sms, cudaStream_t stream) {
   const int threads = 256;
   const bool vec = (bs % 8 == 0) && bs <= 256 && log2_exact(bs) >= 0;
-  NF4_PROF_BEGIN(stream, kKQuantize);
   if (vec) {
     const int64_t n_words = numel / 8;
     const int grid = grid_for(n_words, threads, sms, 8);
-    const float4* w4 = reinterpret_cast<const float4*>(w);
     uint32_t* c32 = reinterpret_cast<uint32_t*>(codes);
     switch (bs / 8) {
-      case 1: quantize_vec_kernel<1><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
-      case 2: quantize_vec_kernel<2><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
-      case 4: quantize_vec_kernel<4><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
-      case 8: quantize_vec_kernel<8><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
-      case 16: quantize_vec_kernel<16><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
-      default: quantize_vec_kernel<32><<<grid, threads, 0, stream>>>(w4, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 1: quantize_vec_kernel<1, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 2: quantize_vec_kernel<2, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 4: quantize_vec_kernel<4, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 8: quantize_vec_kernel<8, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 16: quantize_vec_kernel<16, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
+      default: quantize_vec_kernel<32, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
     }
   } else {
     const int64_t n_blocks = numel / bs;
     const int grid = grid_for(n_blocks, threads, sms, 8);
-    quantize_generic_kernel<<<grid, threads, 0, stream>>>(w, n_blocks, bs, codes, absmax_out,
-                                                          status, gmax);
+    quantize_generic_kernel<IN><<<grid, threads, 0, stream>>>(w, n_blocks, bs, codes, absmax_out,
+                                                              status, gmax);
   }
+}
+
+cudaError_t launch_quantize(const void* w, int in_dtype, int64_t numel, int bs, uint8_t* codes,
+                            float* absmax_out, uint32_t* status, uint32_t* gmax, int sms,
+                            cudaStream_t stream, int* launches) {
+  NF4_PROF_BEGIN(stream, kKQuantize);
+  if (in_dtype == NF4_BF16)
+    launch_quantize_typed<kInBF16>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream);
+  else if (in_dtype == NF4_F16)
+    launch_quantize_typed<kInF16>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream);
+  else
+    launch_quantize_typed<kInF32>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream);
   NF4_PROF_END(stream, kKQuantize);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;

@@ -28,7 +28,7 @@ EXPORTED = (
     "nf4_profile_begin", "nf4_profile_end", "nf4_profile_kernel_count", "nf4_kernel_name",
     "nf4_profile_get", "nf4_workspace_bytes", "nf4_read_status", "nf4_quantize",
     "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "nf4_quantize_noalloc",
-    "nf4_merge",
+    "nf4_merge", "nf4_quantize_typed",
 )
 
 
@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
     L.qlora_linear_bwd.restype = i32
     L.nf4_merge.argtypes = [ctypes.POINTER(CWeight), vp, vp, i32, f32, i32, vp, vp, sz, vp]
     L.nf4_merge.restype = i32
+    L.nf4_quantize_typed.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]
+    L.nf4_quantize_typed.restype = i32
     _lib = L
     return L
 
@@ -210,10 +212,12 @@ class QuantizedWeight:
 
 def quantize(w, block_size: int = 64, double_quant: bool = False, keep_absmax: bool | None = None,
              workspace: Workspace | None = None, stream=None, check_status: bool = False) -> QuantizedWeight:
-    """NF4-quantize an fp32 CUDA tensor (any shape; flattened row-major)."""
+    """NF4-quantize a float32, bfloat16 or float16 CUDA tensor (any shape;
+    flattened row-major).  bf16 / f16 elements are widened to fp32 exactly."""
     import torch
-    if w.dtype != torch.float32 or not w.is_cuda:
-        raise TypeError("quantize expects a float32 CUDA tensor")
+    in_dtype = {torch.float32: NF4_F32, torch.bfloat16: NF4_BF16, torch.float16: NF4_F16}.get(w.dtype)
+    if in_dtype is None or not w.is_cuda:
+        raise TypeError("quantize expects a float32, bfloat16 or float16 CUDA tensor")
     w = w.contiguous()
     rows = int(w.shape[0]) if w.dim() >= 1 else 1
     cols = 1
@@ -229,9 +233,14 @@ def quantize(w, block_size: int = 64, double_quant: bool = False, keep_absmax: b
     absmax_scale = torch.empty(1, dtype=torch.float32, device=dev) if double_quant else None
     ws = workspace or default_workspace(dev)
     buf = ws.get(workspace_bytes(OP_QUANTIZE, 0, rows, cols, 0, block_size, double_quant))
-    st = lib().nf4_quantize(_ptr(w), rows, cols, block_size, int(double_quant), _ptr(codes),
-                            _ptr(absmax), _ptr(absmax_q), _ptr(absmax_scale), _ptr(buf),
-                            buf.numel(), _stream(stream))
+    if in_dtype == NF4_F32:
+        st = lib().nf4_quantize(_ptr(w), rows, cols, block_size, int(double_quant), _ptr(codes),
+                                _ptr(absmax), _ptr(absmax_q), _ptr(absmax_scale), _ptr(buf),
+                                buf.numel(), _stream(stream))
+    else:
+        st = lib().nf4_quantize_typed(_ptr(w), in_dtype, rows, cols, block_size, int(double_quant),
+                                      _ptr(codes), _ptr(absmax), _ptr(absmax_q), _ptr(absmax_scale),
+                                      _ptr(buf), buf.numel(), _stream(stream))
     _check(st, "nf4_quantize")
     if check_status:
         _check(ws.read_status(stream), "nf4_quantize (device)")

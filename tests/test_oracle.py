@@ -410,3 +410,17 @@ def test_merge_special_cases():
     s = inp.case.alpha / inp.case.r
     assert np.allclose(O.merge(q0, a, b, inp.case.alpha, "f64"), s * O.matmul_bruteforce(b, a),
                        rtol=1e-13, atol=0)
+
+
+def test_bf16_and_f16_widening_is_exact():
+    # The typed quantizer's definition rests on widening bf16 / f16 to fp32
+    # exactly; checked against torch's conversions on every bf16 pattern and
+    # a sweep of f16 values.
+    import torch
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    mine = WL.bf16_bits_to_f32(bits)
+    theirs = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    same = (mine.view(np.uint32) == theirs.view(np.uint32)) | (np.isnan(mine) & np.isnan(theirs))
+    assert np.all(same)
+    h = bits.view(np.float16)
+    assert np.all((h.astype(np.float32) == torch.from_numpy(h).float().numpy()) | np.isnan(h))
