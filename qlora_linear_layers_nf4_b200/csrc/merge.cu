@@ -13,9 +13,9 @@
 // (MN-major straight from A's [r, K] storage) come by TMA, one tcgen05 MMA
 // chain accumulates the 128 x 256 fp32 product in TMEM, and eight epilogue
 // warps read it back, dequantize the matching NF4 codes (read once from HBM,
-// fetched while the MMAs run), stage each 128 x 32 piece of the merged tile in
-// swizzled shared memory and write it with a TMA tensor store, so every HBM
-// write is a whole line.  The kernel is bound by the output and code bytes;
+// fetched while the MMAs run), stage each warp's 32 x 32 piece of the merged
+// tile in swizzled shared memory and write it with a TMA tensor store, so
+// every HBM write is a whole line and no warp waits on another.  The kernel is bound by the output and code bytes;
 // the contraction is a small fraction of its time.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -35,9 +35,9 @@ constexpr int kMgEpiWarps = kMgCols / 32;    // 128 columns per epilogue thread
 constexpr int kMgThreads = 64 + 32 * kMgEpiWarps;
 constexpr int kMgCtasPerSm = 512 / kMgCols;  // as many as the TMEM columns allow
 // Output staging, after the MMAs are done, over the operand buffers: per
-// 128-column half two 128 x 32 buffers (16 KB each, sized for fp32 rows).
-constexpr uint32_t kMgStageBytes = 16384;
-constexpr uint32_t kMgStagingBytes = 2 * 2 * kMgStageBytes;
+// epilogue warp two 32 x 32 buffers (4 KB each, sized for fp32 rows).
+constexpr uint32_t kMgStageBytes = 4096;
+constexpr uint32_t kMgStagingBytes = kMgEpiWarps * 2 * kMgStageBytes;
 constexpr int kMgMaxChunks = 4;              // r <= 256 in 64-wide chunks
 constexpr uint32_t kMgBBytes = kMgRows * 128;            // B rows x 64 r (bf16)
 constexpr uint32_t kMgABytes = (kMgCols / 64) * 64 * 128; // 64 r x kMgCols k (bf16)
@@ -176,16 +176,13 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
         scale[j] = p.double_quant ? __fmul_rn(float(__ldg(p.absmax_q + blk)), s_g) : __ldg(p.absmax + blk);
       }
     }
-    // The 128 threads of a half agree on going ahead (a barrier with an AND),
-    // so their named barriers below always pair up.
-    const uint32_t bar_id = 1u + uint32_t(half);
-    const bool issuer = ((warp - 2) & 3) == 0 && lane == 0;
-    bool ok = mbar_wait(&sh->accum, 0, abort_flag, p.status);
-    ok = named_barrier_and(bar_id, 128, ok);
+    // Each warp stages and stores its own 32 rows, so the warps never wait on
+    // one another: two 32 x 32 buffers per warp, one TMA store per piece.
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&sh->accum, 0, abort_flag, p.status));
     tc_fence_after();
     if (ok) {
       const float* lut = sh->lut + lane;
-      uint8_t* stage = smem + half * 2 * kMgStageBytes;
+      uint8_t* stage = smem + (warp - 2) * 2 * kMgStageBytes;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
@@ -209,28 +206,28 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
         }
         // buffer c & 1 is free once the store issued two pieces ago has read it
         uint8_t* buf = stage + (c & 1) * kMgStageBytes;
-        if (issuer && c >= 2) bulk_wait_group_read<1>();
-        named_barrier(bar_id, 128);
-        if (p.out_f32) {       // 128-byte rows, 128-byte swizzle: chunk j at j ^ (row & 7)
+        if (lane == 0 && c >= 2) bulk_wait_group_read<1>();
+        __syncwarp();
+        if (p.out_f32) {       // 128-byte rows, 128-byte swizzle: chunk j at j ^ (lane & 7)
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<float4*>(buf + row * 128 + ((j ^ (row & 7)) << 4)) =
+            *reinterpret_cast<float4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
                 make_float4(m[4 * j], m[4 * j + 1], m[4 * j + 2], m[4 * j + 3]);
-        } else {               // 64-byte rows, 64-byte swizzle: chunk j at j ^ ((row >> 1) & 3)
+        } else {               // 64-byte rows, 64-byte swizzle: chunk j at j ^ ((lane >> 1) & 3)
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4)) =
+            *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
                 make_uint4(pack_bf16x2(m[8 * j], m[8 * j + 1]), pack_bf16x2(m[8 * j + 2], m[8 * j + 3]),
                            pack_bf16x2(m[8 * j + 4], m[8 * j + 5]), pack_bf16x2(m[8 * j + 6], m[8 * j + 7]));
         }
         fence_proxy_async_smem();
-        named_barrier(bar_id, 128);
-        if (issuer && k < p.K) {
-          tma_store_2d(&tm_out, buf, k, n0);   // rows past N are clipped by the tensor map
+        __syncwarp();
+        if (lane == 0 && k < p.K) {
+          tma_store_2d(&tm_out, buf, k, n0 + quad * 32);   // rows past N are clipped by the map
           bulk_commit_group();
         }
       }
-      if (issuer) bulk_wait_group_all();
+      if (lane == 0) bulk_wait_group_all();
     }
   }
 
@@ -269,8 +266,8 @@ cudaError_t launch_merge(const nf4_weight& w, const void* A, const void* B, int 
   // (MN-major); out [N, K]: 32 x 128 boxes in the staging layout.
   bool ok = make_map_2d(&tb, B, true, uint64_t(r), uint64_t(N), 64, kMgRows, true);
   ok = ok && make_map_2d(&ta, A, true, uint64_t(K), uint64_t(r), 64, 64, true);
-  ok = ok && (out_f32 ? make_map_2d_f32(&to, out, uint64_t(K), uint64_t(N), 32, kMgRows, CU_TENSOR_MAP_SWIZZLE_128B)
-                      : make_map_2d_bf16(&to, out, uint64_t(K), uint64_t(N), 32, kMgRows, CU_TENSOR_MAP_SWIZZLE_64B));
+  ok = ok && (out_f32 ? make_map_2d_f32(&to, out, uint64_t(K), uint64_t(N), 32, 32, CU_TENSOR_MAP_SWIZZLE_128B)
+                      : make_map_2d_bf16(&to, out, uint64_t(K), uint64_t(N), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
   if (!ok) return cudaErrorInvalidValue;
   MergeParams p;
   p.N = int(N);
