@@ -5,23 +5,26 @@
 //     y  = x W'^T + T B^T,          T = s x A^T,  s = alpha / r
 // and its backward for L = sum(dy * y) with W frozen is
 //     U  = s dy B,  dB = dy^T T,  dA = U^T x,  dx = dy W' + U A.
-// W' = bf16(L[code] * scale) is never written to HBM: the fused kernel
-// dequantizes each NF4 tile into shared memory, in the 128-byte-swizzled
-// layout the tensor core reads, right before the MMA that consumes it.  The
-// adapter product rides in the same TMEM accumulator as extra K steps
-// ([x | T] [W' | B]^T forward, [dy | U] [W' ; A] backward).
+// W' = bf16(L[code] * scale) (f16 in the F16 compute dtype) is never
+// written to HBM: the fused kernel dequantizes each NF4 tile into shared
+// memory, in the swizzled layout the tensor core reads, right before the MMA
+// that consumes it.  The adapter product rides in the same TMEM accumulator
+// as extra K steps ([x | T] [W' | B]^T forward, [dy | U] [W' ; A] backward).
 //
-// Kernels
-//   fused_nf4_gemm<kFwd>  y[M,N]  = x W'^T + T B^T (+ bias)   K-major W' tiles
-//   fused_nf4_gemm<kDx>   dx[M,K] = dy W' + U A                 MN-major W' tiles
-//   adapter_gemm          the rank-r products T, U, dB, dA^T, split along the
-//                         reduction over a thread-block cluster whose CTAs
-//                         sum their fp32 partials through distributed
-//                         shared memory
+// Kernels (each fused kernel in bf16 and f16 instantiations)
+//   fused_nf4_gemm_pair<kFwd>  y[M,N]  = x W'^T + T B^T (+ bias), M > 256:
+//                              a 2-CTA cluster, tcgen05 cta_group::2, 512 x 256 tiles
+//   fused_nf4_gemm_pair<kDx>   dx[M,K] = dy W' + U A (MN-major W' tiles)
+//   fused_nf4_gemm<kFwd/kDx>   the same on one CTA, 256 x 256 tiles, 32 < M <= 256
+//   adapter_gemm               the rank-r products T, U, dB, dA^T, split along
+//                              the reduction over a thread-block cluster whose
+//                              CTAs sum their fp32 partials through
+//                              distributed shared memory
 #include <algorithm>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kernels.h"
 #include "nf4_common.cuh"
