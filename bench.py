@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the hash of the kernel source it was taken on (see profiles/); reported as
 # null once the source changes.
 NCU_TRAFFIC = {
-    # profiles/fused_nf4_gemm_pair_11008x4096_M4096.md: forward 112.3 MB, dx 179.8 MB per launch
-    "d2a3cb6c72ac6ec4": {"fwd": 112_320_000, "dx": 179_838_720},
+    # profiles/fused_nf4_gemm_pair_11008x4096_M4096.md: forward 113.4 MB, dx 175.8 MB per launch
+    "04a914d3af56e147": {"fwd": 113_431_552, "dx": 175_750_912},
 }
 
 
