@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the hash of the kernel source it was taken on (see profiles/); reported as
 # null once the source changes.
 NCU_TRAFFIC = {
-    # profiles/fused_nf4_gemm_pair_11008x4096_M4096.md: forward 113.4 MB, dx 175.8 MB per launch
-    "04a914d3af56e147": {"fwd": 113_431_552, "dx": 175_750_912},
+    # profiles/fused_nf4_gemm_pair_11008x4096_M4096.md: forward 129.4 MB, dx 180.9 MB per launch
+    "a9f4025d149c808b": {"fwd": 129_385_472, "dx": 180_922_624},
 }
 
 
