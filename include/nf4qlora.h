@@ -225,6 +225,23 @@ NF4_API nf4_status nf4_quantize_typed(const void* w, int in_dtype, int64_t rows,
                                       void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Self-check of the bounded-wait path (no counterpart on the pages).  Every
+ * mbarrier wait in the library's kernels gives up after a time limit, records
+ * NF4_ERR_TIMEOUT in the workspace status word and raises its CTA's abort
+ * flag, on which the CTA's other roles unwind; a lost arrival therefore ends
+ * in an error status, never in a hung GPU.  This call runs that path on
+ * purpose: two CTAs each wait on an mbarrier that nothing arrives on, with a
+ * limit of limit_us microseconds (1 .. 1000000), while a second warp per CTA
+ * waits with a 100x longer limit and must be released by the abort flag.
+ * Synchronizes `stream`; returns the status word the kernel left (NF4_ERR_TIMEOUT
+ * when the path works), clears it, and stores in *released the number of CTAs
+ * whose second warp was released by the abort (2 when the path works).
+ *   workspace  >= 256 bytes, 16-byte aligned.
+ */
+NF4_API nf4_status nf4_check_wait_timeout(void* workspace, size_t ws_bytes, uint32_t limit_us,
+                                          uint32_t* released, void* stream);
+
+/*
  * Dequantization (qlora-rs dequantize_nf4; "Honor compute_dtype
  * (BF16/F16/F32) in forward dequant").  out[e] = fp32(L[code_e] * scale_b)
  * as one fp32 product; NF4_BF16 / NF4_F16 store its round-to-nearest-even.

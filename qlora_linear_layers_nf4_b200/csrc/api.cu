@@ -385,6 +385,29 @@ nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const
   return finish(e, launches);
 }
 
+nf4_status nf4_check_wait_timeout(void* workspace, size_t ws_bytes, uint32_t limit_us,
+                                  uint32_t* released, void* stream) {
+  if (workspace == nullptr || !aligned16(workspace) || ws_bytes < nf4::kWsHeader) return NF4_ERR_WORKSPACE;
+  if (released == nullptr || limit_us < 1 || limit_us > 1000000) return NF4_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + nf4::kWsStatus);
+  uint32_t* seen = reinterpret_cast<uint32_t*>(ws + nf4::kWsHeader - 4);   // last header word
+  if (cudaMemsetAsync(seen, 0, sizeof(uint32_t), st) != cudaSuccess) return NF4_ERR_CUDA;
+  int launches = 0;
+  if (nf4::launch_wait_timeout_check(status, uint64_t(limit_us) * 1000u, seen, st, &launches) != cudaSuccess)
+    return NF4_ERR_CUDA;
+  g_launches += launches;
+  uint32_t host[2] = {0, 0};
+  if (cudaMemcpyAsync(&host[0], status, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(&host[1], seen, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return NF4_ERR_CUDA;
+  *released = host[1];
+  return static_cast<nf4_status>(host[0]);
+}
+
 nf4_status nf4_merge(const nf4_weight* w, const void* A, const void* B, int r, float alpha,
                      int out_dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
   // the linear checks with a stand-in x (the merge has no activations)

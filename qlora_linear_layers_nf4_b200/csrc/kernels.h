@@ -64,6 +64,12 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t stream,
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 
+// Bounded-wait self-check (selfcheck.cu): waits that nothing completes give
+// up after limit_ns, record NF4_ERR_TIMEOUT in *status and raise the abort
+// flag, which the second role counts into *seen_abort (one per CTA).
+cudaError_t launch_wait_timeout_check(uint32_t* status, uint64_t limit_ns, uint32_t* seen_abort,
+                                      cudaStream_t st, int* launches);
+
 // Dense merge W' + s B A (merge.cu).
 cudaError_t launch_merge(const nf4_weight& w, const void* A, const void* B, int r, float alpha,
                          int out_f32, void* out, uint32_t* status, cudaStream_t st, int* launches);

@@ -182,7 +182,8 @@ template <int MODE, bool F16>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a2,
                    const __grid_constant__ CUtensorMap tm_b2,
-                   const __grid_constant__ CUtensorMap tm_codes, const FusedParams p) {
+                   const __grid_constant__ CUtensorMap tm_codes,
+                   const __grid_constant__ CUtensorMap tm_out, const FusedParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   FusedShared* sh = reinterpret_cast<FusedShared*>(smem + kStages * kStageBytes);
@@ -338,44 +339,59 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       if (lane == 0) mbar_arrive(&sh->bready[s]);
     }
 
-    // ---------------- epilogue: TMEM -> registers -> bf16 -> global
+    // ---------------- epilogue: TMEM -> registers -> bf16 / f16 -> shared
+    // staging -> TMA store.  Each warp owns 32 rows (its TMEM lanes) of one
+    // accumulator and writes 32 x 32 pieces through two 2 KB buffers over
+    // the idle stage ring, so the output leaves as whole lines.
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&sh->accum, 0, abort_flag, p.status));
     tc_fence_after();
     if (ok) {
       const int quad = warp & 3;                     // TMEM lanes 32*quad .. +31
       const int half = (warp - 2) >> 2;              // accumulator half
-      const int row = m0 + half * 128 + quad * 32 + lane;
+      const int row0 = m0 + half * 128 + quad * 32;  // this warp's first row
+      uint8_t* stage = smem + (warp - 2) * 4096;
+      constexpr bool f16 = F16;
+#pragma unroll 1
       for (int c = 0; c < kTileN / 32; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + half * kTileN + c * 32, v);
         tmem_ld_wait();
         const int col0 = tile_n0 + c * 32;
-        if (row < p.M) {
+        uint32_t packed[16];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int col = col0 + 8 * g;
-            if (col < p.out_cols) {
-              float f[8];
+        for (int g = 0; g < 4; ++g) {
+          float f[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
-              constexpr bool f16 = F16;
-              if (MODE == kFwd && p.bias != nullptr) {
-                const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
-                const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
+          const int col = col0 + 8 * g;
+          if (MODE == kFwd && p.bias != nullptr && col < p.out_cols) {
+            const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
+            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float2 bf = unpack2(f16, bw[e]);
-                  f[2 * e] += bf.x;
-                  f[2 * e + 1] += bf.y;
-                }
-              }
-              const uint4 o = make_uint4(pack2(f16, f[0], f[1]), pack2(f16, f[2], f[3]),
-                                         pack2(f16, f[4], f[5]), pack2(f16, f[6], f[7]));
-              *reinterpret_cast<uint4*>(p.out + int64_t(row) * p.out_cols + col) = o;
+            for (int e = 0; e < 4; ++e) {
+              const float2 bf = unpack2(f16, bw[e]);
+              f[2 * e] += bf.x;
+              f[2 * e + 1] += bf.y;
             }
           }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) packed[4 * g + e] = pack2(f16, f[2 * e], f[2 * e + 1]);
+        }
+        uint8_t* buf = stage + (c & 1) * 2048;
+        if (lane == 0 && c >= 2) bulk_wait_group_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 4; ++j)   // 64-byte rows, 64-byte swizzle: chunk j at j ^ ((row >> 1) & 3)
+          *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && col0 < p.out_cols && row0 < p.M) {
+          tma_store_2d(&tm_out, buf, col0, row0);   // rows past M, columns past the end: clipped
+          bulk_commit_group();
         }
       }
+      if (lane == 0) bulk_wait_group_all();
     }
   }
 
@@ -1230,8 +1246,8 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   ok = ok && make_map(&tb2, a.B, true, a.r, a.N, 64, brows, true);
   ok = ok && (pair ? make_map(&tc, a.w->codes, false, a.K / 2, a.N, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)
                    : make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, brows, false));
-  CUtensorMap to;   // y [M, N]: 32 x 32 boxes in the pair epilogue's staging layout
-  ok = ok && (!pair || make_map_2d_bf16(&to, a.y, uint64_t(a.N), uint64_t(a.M), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
+  CUtensorMap to;   // y [M, N]: 32 x 32 boxes in the epilogues' staging layout
+  ok = ok && make_map_2d_bf16(&to, a.y, uint64_t(a.N), uint64_t(a.M), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) return cudaErrorInvalidValue;
   const FusedParams p = fused_params(a, kFwd);
   NF4_PROF_BEGIN(st, kKFusedFwd);
@@ -1241,8 +1257,8 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
     else fused_nf4_gemm_pair<kFwd, false><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, to, p);
   } else {
     dim3 grid(unsigned(cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kTileM)));
-    if (a.f16) fused_nf4_gemm<kFwd, true><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
-    else fused_nf4_gemm<kFwd, false><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+    if (a.f16) fused_nf4_gemm<kFwd, true><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, to, p);
+    else fused_nf4_gemm<kFwd, false><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, to, p);
   }
   NF4_PROF_END(st, kKFusedFwd);
   e = cudaGetLastError();
@@ -1300,8 +1316,8 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
   ok = ok && make_map(&tb2, a.A, true, a.K, a.r, 64, 64, true);
   ok = ok && (pair ? make_map(&tc, a.w->codes, false, a.K / 2, a.N, 64, 256, CU_TENSOR_MAP_SWIZZLE_64B)
                    : make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, 64, false));
-  CUtensorMap to;   // dx [M, K]: 32 x 32 boxes in the pair epilogue's staging layout
-  ok = ok && (!pair || make_map_2d_bf16(&to, a.dx, uint64_t(a.K), uint64_t(a.M), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
+  CUtensorMap to;   // dx [M, K]: 32 x 32 boxes in the epilogues' staging layout
+  ok = ok && make_map_2d_bf16(&to, a.dx, uint64_t(a.K), uint64_t(a.M), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) return cudaErrorInvalidValue;
   const FusedParams p = fused_params(a, kDx);
   NF4_PROF_BEGIN(st, kKFusedDx);
@@ -1311,8 +1327,8 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     else fused_nf4_gemm_pair<kDx, false><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, to, p);
   } else {
     dim3 grid(unsigned(cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kTileM)));
-    if (a.f16) fused_nf4_gemm<kDx, true><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
-    else fused_nf4_gemm<kDx, false><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, p);
+    if (a.f16) fused_nf4_gemm<kDx, true><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, to, p);
+    else fused_nf4_gemm<kDx, false><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, to, p);
   }
   NF4_PROF_END(st, kKFusedDx);
   e = cudaGetLastError();

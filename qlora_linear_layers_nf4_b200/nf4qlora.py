@@ -28,7 +28,7 @@ EXPORTED = (
     "nf4_profile_begin", "nf4_profile_end", "nf4_profile_kernel_count", "nf4_kernel_name",
     "nf4_profile_get", "nf4_workspace_bytes", "nf4_read_status", "nf4_quantize",
     "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "nf4_quantize_noalloc",
-    "nf4_merge", "nf4_quantize_typed",
+    "nf4_merge", "nf4_quantize_typed", "nf4_check_wait_timeout",
 )
 
 
@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
     L.nf4_merge.restype = i32
     L.nf4_quantize_typed.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]
     L.nf4_quantize_typed.restype = i32
+    L.nf4_check_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, ctypes.POINTER(ctypes.c_uint32), vp]
+    L.nf4_check_wait_timeout.restype = i32
     _lib = L
     return L
 

@@ -142,6 +142,16 @@ def test_merge_host_validation():
     assert m(_cw(), wsb=0) == 5
 
 
+def test_wait_check_host_validation():
+    L = Q.lib()
+    rel = ctypes.c_uint32(0)
+    assert L.nf4_check_wait_timeout(None, 256, 1000, ctypes.byref(rel), None) == 5
+    assert L.nf4_check_wait_timeout(FAKE, 16, 1000, ctypes.byref(rel), None) == 5
+    assert L.nf4_check_wait_timeout(FAKE, 256, 0, ctypes.byref(rel), None) == 1
+    assert L.nf4_check_wait_timeout(FAKE, 256, 2000000, ctypes.byref(rel), None) == 1
+    assert L.nf4_check_wait_timeout(FAKE, 256, 1000, None, None) == 1
+
+
 def test_bucket_encoding_conditions():
     # The quantize kernel's fast encode indexes 64 buckets of width 1/32 over
     # [-1, 1] and compares with the single threshold inside the bucket.  It is
