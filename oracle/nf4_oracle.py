@@ -52,6 +52,9 @@ Readings of points the pages leave open (each is also listed in the design doc):
   R16 Merge: W_merged = w' + s B A from the fp32 dequant w' (not the bf16
       one), the sum taken exactly and rounded to fp32, then (for a bf16
       result) to bf16 with ties to even.
+  R19 A tensor whose size is not a multiple of the block: the last block holds
+      the remaining elements and its absmax is theirs alone; for an odd
+      element count the last byte's low nibble is 7 (the exact-zero level).
 """
 from __future__ import annotations
 
@@ -130,10 +133,11 @@ def nearest_code(v: np.ndarray) -> np.ndarray:
 
 
 def pack_codes(codes: np.ndarray) -> np.ndarray:
-    """Two 4-bit codes per byte, the even element in the high nibble (R5)."""
+    """Two 4-bit codes per byte, the even element in the high nibble (R5); an
+    odd count ends with a byte whose low nibble is 7 (R19)."""
     codes = np.asarray(codes, dtype=np.uint8).reshape(-1)
     if codes.size % 2:
-        raise ValueError("an even number of codes is needed to pack")
+        codes = np.concatenate([codes, np.array([7], dtype=np.uint8)])
     return ((codes[0::2] << 4) | codes[1::2]).astype(np.uint8)
 
 
@@ -173,11 +177,13 @@ def quantize(w: np.ndarray, block_size: int = 64, double: bool = False) -> dict:
     flat = w.reshape(-1)
     if block_size <= 0 or block_size % 2:
         raise ValueError("block_size must be a positive even number")
-    if flat.size % block_size:
-        raise ValueError("numel must be a multiple of block_size")
     if not np.all(np.isfinite(flat)):
         raise ValueError("non-finite input")
-    blocks = flat.reshape(-1, block_size)
+    # R19: a short last block; zero padding changes neither its absmax nor the
+    # codes of its elements, and the padding's own codes are dropped below.
+    n = flat.size
+    pad = (-n) % block_size
+    blocks = np.concatenate([flat, np.zeros(pad, dtype=np.float32)]).reshape(-1, block_size)
     absmax = np.abs(blocks).max(axis=1).astype(np.float32)
     codes = np.full(blocks.shape, 7, dtype=np.uint8)       # R3: absmax == 0
     nz = absmax > 0
@@ -185,7 +191,7 @@ def quantize(w: np.ndarray, block_size: int = 64, double: bool = False) -> dict:
         v = (blocks[nz] / absmax[nz][:, None]).astype(np.float32)  # R4
         codes[nz] = nearest_code(v)
     out = {
-        "codes": pack_codes(codes.reshape(-1)),
+        "codes": pack_codes(codes.reshape(-1)[:n]),
         "absmax": absmax,
         "shape": tuple(w.shape),
         "block_size": int(block_size),
@@ -238,10 +244,11 @@ def dequantize(q: dict, out_dtype: str = "f32") -> np.ndarray:
     RNE-rounded values, "f16" gives numpy float16 (RNE).
     """
     levels = nf4_levels()
-    codes = unpack_codes(q["codes"])
+    n = int(np.prod(q["shape"]))
+    codes = unpack_codes(q["codes"])[:n]
     scales = block_scales(q)
     bs = q["block_size"]
-    per_elem_scale = np.repeat(scales, bs)
+    per_elem_scale = np.repeat(scales, bs)[:n]
     w = (levels[codes] * per_elem_scale).astype(np.float32)   # one fp32 product
     w = w.reshape(q["shape"])
     if out_dtype == "f32":

@@ -199,8 +199,6 @@ def test_round_trip_error_bound():
 
 def test_refuses_bad_shapes_and_nonfinite():
     with pytest.raises(ValueError):
-        O.quantize(np.zeros(100, np.float32), 64)
-    with pytest.raises(ValueError):
         O.quantize(np.zeros(64, np.float32), 63)
     w = np.zeros(64, np.float32)
     w[3] = np.inf
@@ -424,3 +422,41 @@ def test_bf16_and_f16_widening_is_exact():
     assert np.all(same)
     h = bits.view(np.float16)
     assert np.all((h.astype(np.float32) == torch.from_numpy(h).float().numpy()) | np.isnan(h))
+
+
+# --------------------------------------------------------------------------- tail blocks (R19)
+
+def test_tail_block_is_its_own_quantization():
+    # The short last block must come out exactly as that block quantized on its
+    # own (a full-block quantization with block size = its length, an
+    # independent path), and the full blocks as before.
+    rng = np.random.default_rng(8)
+    for n, bs in [(100, 64), (1000, 64), (130, 32), (37, 8), (65, 64)]:
+        w = (rng.standard_normal(n) * 0.02).astype(np.float32)
+        q = O.quantize(w, bs)
+        full = (n // bs) * bs
+        t = n - full
+        codes = O.unpack_codes(q["codes"])[:n]
+        if full:
+            qf = O.quantize(w[:full], bs)
+            assert np.array_equal(codes[:full], O.unpack_codes(qf["codes"]))
+            assert np.array_equal(q["absmax"][:-1], qf["absmax"])
+        if t % 2 == 0:
+            qt = O.quantize(w[full:], t)
+            assert np.array_equal(codes[full:], O.unpack_codes(qt["codes"]))
+            assert q["absmax"][-1] == qt["absmax"][0]
+        assert q["absmax"][-1] == np.max(np.abs(w[full:]))       # its own elements only
+        assert q["codes"].size == (n + 1) // 2
+        if n % 2:
+            assert q["codes"][-1] & 0x0F == 7                      # the pad nibble
+        # round trip within the largest half gap of the block's absmax
+        d = O.dequantize(q, "f32")
+        scale = np.repeat(q["absmax"], bs)[:n]
+        assert np.all(np.abs(d - w) <= scale * 0.1519 + 1e-12)
+
+
+def test_tail_block_double_quant_counts_every_block():
+    w = WL.draw_weight((1, 1000), seed=12).reshape(-1)
+    q = O.quantize(w, 64, double=True)
+    assert q["absmax_q"].size == 16                   # 15 full blocks + the tail
+    assert q["absmax_q"].max() == 255
