@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the hash of the kernel source it was taken on (see profiles/); reported as
 # null once the source changes.
 NCU_TRAFFIC = {
-    # profiles/fused_nf4_gemm_pair_11008x4096_M4096.md: forward 129.4 MB, dx 180.9 MB per launch
-    "a9f4025d149c808b": {"fwd": 129_385_472, "dx": 180_922_624},
+    # profiles/fused_nf4_gemm_pair_11008x4096_M4096.md: forward 125.3 MB, dx 180.0 MB per launch
+    "971f40c8dc885c10": {"fwd": 125_310_464, "dx": 180_007_424},
 }
 
 

@@ -82,12 +82,15 @@ typedef enum {
  * src/export.rs page (data -> codes, scales -> absmax, scales_quantized ->
  * absmax_q, scales_scales -> absmax_scale, shape -> rows/cols).  Asymmetric
  * zero-points are not part of NF4 and are not represented.
- *   codes         rows*cols/2 bytes.  Element e of the row-major flattened
- *                 tensor has a 4-bit code in byte e/2: the HIGH nibble for
- *                 even e, the LOW nibble for odd e.
- *   absmax        fp32 per block (rows*cols/block_size), block b covering
- *                 elements [b*block_size, (b+1)*block_size).  Used when
- *                 double_quant == 0.  May be NULL when double_quant != 0.
+ *   codes         ceil(rows*cols/2) bytes.  Element e of the row-major
+ *                 flattened tensor has a 4-bit code in byte e/2: the HIGH
+ *                 nibble for even e, the LOW nibble for odd e.  For an odd
+ *                 element count the last byte's low nibble is 7 (level 0.0).
+ *   absmax        fp32 per block (nblocks = ceil(rows*cols/block_size)), block
+ *                 b covering elements [b*block_size, (b+1)*block_size); the
+ *                 last block may be short and covers the elements that
+ *                 remain.  Used when double_quant == 0.  May be NULL when
+ *                 double_quant != 0.
  *   absmax_q      u8 per block, used when double_quant != 0.
  *   absmax_scale  one fp32 (the scale of the scales), used when
  *                 double_quant != 0.  Block b decodes with
@@ -163,13 +166,16 @@ NF4_API nf4_status nf4_read_status(void* workspace, void* stream);
  * "NF4 pack/unpack + block absmax scales" and "Double quant (simplified
  * global u8 scales)").
  *   w            fp32 [rows, cols], read only.
- *   block_size   positive and even; rows*cols must be a multiple of it.
- *                Multiples of 8 up to 256 that are powers of two take the
- *                vectorized path; other even sizes a per-block path.
+ *   block_size   positive and even.  Multiples of 8 up to 256 that are
+ *                powers of two take the vectorized path; other even sizes a
+ *                per-block path.  rows*cols need not be a multiple of it: the
+ *                last block then holds the remaining elements, its absmax is
+ *                the max over those alone, and a small extra kernel encodes
+ *                it (the pages' quantize_nf4 takes tensors of any size).
  *   For each block: absmax = max |w|; v = w / absmax (IEEE fp32 division);
  *   code = index of the nearest NF4 level (lower code on an exact tie);
  *   absmax == 0 gives code 7 for the whole block.
- *   codes        u8 [rows*cols/2], written (packing as in nf4_weight).
+ *   codes        u8 [ceil(rows*cols/2)], written (packing as in nf4_weight).
  *   absmax       fp32 [nblocks]; written when non-NULL.  Required when
  *                double_quant == 0.
  *   double_quant 0 or 1.  When 1: G = max absmax, absmax_scale[0] =
@@ -245,8 +251,10 @@ NF4_API nf4_status nf4_check_wait_timeout(void* workspace, size_t ws_bytes, uint
  * Dequantization (qlora-rs dequantize_nf4; "Honor compute_dtype
  * (BF16/F16/F32) in forward dequant").  out[e] = fp32(L[code_e] * scale_b)
  * as one fp32 product; NF4_BF16 / NF4_F16 store its round-to-nearest-even.
- *   w->block_size must be a positive multiple of 8; out has rows*cols
- *   elements of out_dtype.
+ *   w->block_size must be positive and even (multiples of 8 take the
+ *   vectorized path); rows*cols need not be a multiple of it (a short last
+ *   block decodes with its own scale).  out has rows*cols elements of
+ *   out_dtype.
  */
 NF4_API nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out, void* stream);
 

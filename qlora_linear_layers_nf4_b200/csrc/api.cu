@@ -34,7 +34,7 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 size_t quantize_ws(int64_t numel, int bs, int dq) {
   size_t bytes = nf4::kWsHeader;
-  if (dq && bs > 0 && numel > 0) bytes += round_up(size_t(numel / bs) * sizeof(float), 256);
+  if (dq && bs > 0 && numel > 0) bytes += round_up(size_t((numel + bs - 1) / bs) * sizeof(float), 256);
   return bytes;
 }
 
@@ -225,8 +225,7 @@ nf4_status quantize_impl(const void* w, int in_dtype, int64_t rows, int64_t cols
   if (block_size <= 0 || (block_size % 2) != 0) return NF4_ERR_SHAPE;
   if (double_quant != 0 && double_quant != 1) return NF4_ERR_INVALID_ARG;
   if (rows != 0 && cols > INT64_MAX / rows) return NF4_ERR_SHAPE;
-  const int64_t numel = rows * cols;
-  if (numel % block_size != 0) return NF4_ERR_SHAPE;
+  const int64_t numel = rows * cols;  // a short last block is allowed
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (numel == 0) {  // empty tensor: nothing to encode; the scale of no scales is 0
     if (double_quant && absmax_scale != nullptr) {
@@ -259,7 +258,7 @@ nf4_status quantize_impl(const void* w, int in_dtype, int64_t rows, int64_t cols
     e = nf4::launch_quantize(w, in_dtype, numel, block_size, codes, amax, status,
                              double_quant ? gmax : nullptr, sms, st, &launches);
   if (e == cudaSuccess && double_quant)
-    e = nf4::launch_double_quant(amax, numel / block_size, gmax, absmax_q, absmax_scale, sms, st,
+    e = nf4::launch_double_quant(amax, (numel + block_size - 1) / block_size, gmax, absmax_q, absmax_scale, sms, st,
                                  &launches);
   return finish(e, launches);
 }
@@ -289,10 +288,9 @@ nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out, void* s
   if (out_dtype != NF4_F32 && out_dtype != NF4_BF16 && out_dtype != NF4_F16)
     return NF4_ERR_INVALID_ARG;
   if (w->rows < 0 || w->cols < 0) return NF4_ERR_SHAPE;
-  if (w->block_size <= 0 || (w->block_size % 8) != 0) return NF4_ERR_SHAPE;
+  if (w->block_size <= 0 || (w->block_size % 2) != 0) return NF4_ERR_SHAPE;
   if (w->rows != 0 && w->cols > INT64_MAX / w->rows) return NF4_ERR_SHAPE;
-  const int64_t numel = w->rows * w->cols;
-  if (numel % w->block_size != 0) return NF4_ERR_SHAPE;
+  const int64_t numel = w->rows * w->cols;  // a short last block is allowed
   if (w->double_quant) {
     if (w->absmax_q == nullptr || w->absmax_scale == nullptr) return NF4_ERR_INVALID_ARG;
     if (!aligned16(w->absmax_q) || !aligned4(w->absmax_scale)) return NF4_ERR_ALIGNMENT;

@@ -70,8 +70,7 @@ extern "C" nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t
   if (double_quant != 0 && double_quant != 1) return NF4_ERR_INVALID_ARG;
   if (rows != 0 && cols > INT64_MAX / rows) return NF4_ERR_SHAPE;
   const int64_t numel = rows * cols;
-  if (numel % block_size != 0) return NF4_ERR_SHAPE;
-  const int64_t n_blocks = numel / block_size;
+  const int64_t n_blocks = (numel + block_size - 1) / block_size;  // the last may be short
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (numel == 0) {  // empty tensor: nothing to encode; the scale of no scales is 0
     if (double_quant && absmax_scale != nullptr) {

@@ -229,6 +229,45 @@ __global__ void __launch_bounds__(256) quantize_generic_kernel(
   if (gmax != nullptr) cta_global_max(cta_max, gmax);
 }
 
+// The short last block of a tensor whose size is not a multiple of the block
+// size: t (1 <= t < bs) elements starting at element e0 (a multiple of bs, so
+// at byte e0 / 2 of the codes).  One CTA: block max over the t elements, then
+// one byte per pair; an odd t leaves the last byte's low nibble as code 7
+// (level 0.0), which is what encoding a zero gives.
+template <int IN>
+__global__ void __launch_bounds__(256) quantize_tail_kernel(
+    const void* __restrict__ w, int64_t e0, int t, uint8_t* __restrict__ codes,
+    float* __restrict__ absmax, int64_t blk, uint32_t* __restrict__ status,
+    uint32_t* __restrict__ gmax) {
+  __shared__ float red[8];
+  float m = 0.0f;
+  bool bad = false;
+  for (int i = threadIdx.x; i < t; i += blockDim.x) {
+    const float v = load1<IN>(w, e0 + i);
+    bad |= !isfinite(v);
+    m = fmaxf(m, fabsf(v));
+  }
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = red[0];
+  for (int k = 1; k < int(blockDim.x >> 5); ++k) m = fmaxf(m, red[k]);
+  if (bad) report(status, NF4_ERR_NONFINITE);
+  uint8_t* c = codes + e0 / 2;
+  for (int p = threadIdx.x; 2 * p < t; p += blockDim.x) {
+    const float w0 = load1<IN>(w, e0 + 2 * p);
+    if (2 * p + 1 < t) {
+      c[p] = uint8_t(pair_byte(w0, load1<IN>(w, e0 + 2 * p + 1), m));
+    } else {
+      c[p] = uint8_t((pair_byte(w0, 0.0f, m) & 0xf0u) | 0x7u);
+    }
+  }
+  if (threadIdx.x == 0) {
+    if (absmax != nullptr) absmax[blk] = m;
+    if (gmax != nullptr && m > 0.0f) atomicMax(gmax, __float_as_uint(m));
+  }
+}
+
 // Simplified double quant of the block scales: one global scale G / 255 and a
 // u8 per block, rint(absmax / s_g) with ties to even.
 // Launched as a programmatic dependent of the quantize kernel: it starts
@@ -348,6 +387,37 @@ __global__ void __launch_bounds__(256) dequant_x4_kernel(
   }
 }
 
+// One fp32 value as the output type, rounded to nearest even.
+template <typename OutT>
+__device__ __forceinline__ OutT round_out(float v);
+template <>
+__device__ __forceinline__ float round_out<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 round_out<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <>
+__device__ __forceinline__ __half round_out<__half>(float v) { return __float2half_rn(v); }
+
+// Any even block size, and the short last block: one code byte (two
+// elements; bs is even, so both lie in one block) per thread, bytes
+// [byte0, byte1).  numel is the tensor's element count; a last byte that holds
+// one element writes only that one.
+template <typename OutT, bool kDouble>
+__global__ void __launch_bounds__(256) dequant_bytes_kernel(
+    const uint8_t* __restrict__ codes, int64_t byte0, int64_t byte1, int64_t numel, int bs,
+    const float* __restrict__ absmax, const uint8_t* __restrict__ absmax_q,
+    const float* __restrict__ absmax_scale, OutT* __restrict__ out) {
+  const float s_g = kDouble ? *absmax_scale : 0.0f;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = byte0 + int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < byte1; i += stride) {
+    const uint32_t byte = codes[i];
+    const int64_t e = 2 * i;
+    const int64_t blk = e / bs;
+    const float scale = kDouble ? __fmul_rn(float(absmax_q[blk]), s_g) : absmax[blk];
+    out[e] = round_out<OutT>(__fmul_rn(level(byte >> 4), scale));
+    if (e + 1 < numel) out[e + 1] = round_out<OutT>(__fmul_rn(level(byte & 15u), scale));
+  }
+}
+
 int grid_for(int64_t work_items, int threads, int sms, int per_sm) {
   int64_t g = (work_items + threads - 1) / threads;
   const int64_t cap = int64_t(sms) * per_sm;
@@ -367,11 +437,14 @@ int log2_exact(int v) {
 
 template <int IN>
 void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes, float* absmax_out,
-                           uint32_t* status, uint32_t* gmax, int sms, cudaStream_t stream) {
+                           uint32_t* status, uint32_t* gmax, int sms, cudaStream_t stream,
+                           int* launches) {
   const int threads = 256;
+  const int64_t n_full = numel / bs;          // whole blocks
+  const int tail = int(numel - n_full * bs);  // elements of the short last block
   const bool vec = (bs % 8 == 0) && bs <= 256 && log2_exact(bs) >= 0;
-  if (vec) {
-    const int64_t n_words = numel / 8;
+  if (n_full > 0 && vec) {
+    const int64_t n_words = n_full * bs / 8;
     const int grid = grid_for(n_words, threads, sms, 8);
     uint32_t* c32 = reinterpret_cast<uint32_t*>(codes);
     switch (bs / 8) {
@@ -382,27 +455,35 @@ void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes,
       case 16: quantize_vec_kernel<16, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
       default: quantize_vec_kernel<32, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
     }
-  } else {
-    const int64_t n_blocks = numel / bs;
-    const int grid = grid_for(n_blocks, threads, sms, 8);
-    quantize_generic_kernel<IN><<<grid, threads, 0, stream>>>(w, n_blocks, bs, codes, absmax_out,
+    ++*launches;
+  } else if (n_full > 0) {
+    const int grid = grid_for(n_full, threads, sms, 8);
+    quantize_generic_kernel<IN><<<grid, threads, 0, stream>>>(w, n_full, bs, codes, absmax_out,
                                                               status, gmax);
+    ++*launches;
+  }
+  if (tail > 0) {
+    // an ordinary launch: it starts once the full-block kernel has finished
+    quantize_tail_kernel<IN><<<1, threads, 0, stream>>>(w, n_full * bs, tail, codes, absmax_out,
+                                                        n_full, status, gmax);
+    ++*launches;
   }
 }
 
 cudaError_t launch_quantize(const void* w, int in_dtype, int64_t numel, int bs, uint8_t* codes,
                             float* absmax_out, uint32_t* status, uint32_t* gmax, int sms,
                             cudaStream_t stream, int* launches) {
+  int n = 0;
   NF4_PROF_BEGIN(stream, kKQuantize);
   if (in_dtype == NF4_BF16)
-    launch_quantize_typed<kInBF16>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream);
+    launch_quantize_typed<kInBF16>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream, &n);
   else if (in_dtype == NF4_F16)
-    launch_quantize_typed<kInF16>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream);
+    launch_quantize_typed<kInF16>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream, &n);
   else
-    launch_quantize_typed<kInF32>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream);
+    launch_quantize_typed<kInF32>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream, &n);
   NF4_PROF_END(stream, kKQuantize);
   cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) ++*launches;
+  if (e == cudaSuccess) *launches += n;
   return e;
 }
 
@@ -435,19 +516,25 @@ cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uin
 cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int sms,
                               cudaStream_t stream, int* launches) {
   const int64_t numel = w.rows * w.cols;
-  const int64_t n_words = numel / 8;
-  const int bs_words = w.block_size / 8;
-  const int shift = log2_exact(bs_words);
+  const int bs = w.block_size;
   const int threads = 256;
   const bool dq = w.double_quant != 0;
-  {
+  // Whole 8-element words of whole blocks go through the word kernel when the
+  // block size is a multiple of 8; every other code byte (a block size that is
+  // not, or the short last block) through the byte kernel.
+  const int64_t n_words = (bs % 8 == 0) ? (numel / bs) * bs / 8 : 0;
+  const int64_t byte0 = n_words * 4, byte1 = (numel + 1) / 2;
+  int n = 0;
+  NF4_PROF_BEGIN(stream, kKDequantize);
+  if (n_words > 0) {
+    const int bs_words = bs / 8;
+    const int shift = log2_exact(bs_words);
     const int grid = grid_for((n_words + 3) / 4, threads, sms, 8);
     const uint32_t* c = reinterpret_cast<const uint32_t*>(w.codes);
 #define NF4_DQ4_LAUNCH(T, D)                                                                    \
   dequant_x4_kernel<T, D><<<grid, threads, 0, stream>>>(c, n_words, shift, bs_words, w.absmax, \
                                                         w.absmax_q, w.absmax_scale,            \
                                                         reinterpret_cast<T*>(out))
-    NF4_PROF_BEGIN(stream, kKDequantize);
     if (out_dtype == NF4_F32) {
       if (dq) NF4_DQ4_LAUNCH(float, true); else NF4_DQ4_LAUNCH(float, false);
     } else if (out_dtype == NF4_BF16) {
@@ -456,11 +543,29 @@ cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int
       if (dq) NF4_DQ4_LAUNCH(__half, true); else NF4_DQ4_LAUNCH(__half, false);
     }
 #undef NF4_DQ4_LAUNCH
-    NF4_PROF_END(stream, kKDequantize);
-    cudaError_t e = cudaGetLastError();
-    if (e == cudaSuccess) ++*launches;
-    return e;
+    ++n;
   }
+  if (byte1 > byte0) {
+    const int grid = grid_for(byte1 - byte0, threads, sms, 8);
+#define NF4_DQB_LAUNCH(T, D)                                                               \
+  dequant_bytes_kernel<T, D><<<grid, threads, 0, stream>>>(w.codes, byte0, byte1, numel, bs, \
+                                                           w.absmax, w.absmax_q,            \
+                                                           w.absmax_scale,                  \
+                                                           reinterpret_cast<T*>(out))
+    if (out_dtype == NF4_F32) {
+      if (dq) NF4_DQB_LAUNCH(float, true); else NF4_DQB_LAUNCH(float, false);
+    } else if (out_dtype == NF4_BF16) {
+      if (dq) NF4_DQB_LAUNCH(__nv_bfloat16, true); else NF4_DQB_LAUNCH(__nv_bfloat16, false);
+    } else {
+      if (dq) NF4_DQB_LAUNCH(__half, true); else NF4_DQB_LAUNCH(__half, false);
+    }
+#undef NF4_DQB_LAUNCH
+    ++n;
+  }
+  NF4_PROF_END(stream, kKDequantize);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) *launches += n;
+  return e;
 }
 
 }  // namespace nf4

@@ -189,8 +189,8 @@ def default_workspace(device) -> Workspace:
 @dataclass
 class QuantizedWeight:
     """Device tensors of one NF4 weight (fields as in `nf4_weight`)."""
-    codes: object                    # uint8 [numel/2]
-    absmax: object | None            # fp32 [nblocks]
+    codes: object                    # uint8 [ceil(numel/2)]
+    absmax: object | None            # fp32 [nblocks = ceil(numel/block_size)]
     absmax_q: object | None          # uint8 [nblocks]
     absmax_scale: object | None      # fp32 [1]
     rows: int
@@ -227,9 +227,9 @@ def quantize(w, block_size: int = 64, double_quant: bool = False, keep_absmax: b
         cols *= int(d)
     numel = w.numel()
     dev = w.device
-    nblocks = numel // block_size if block_size > 0 else 0
+    nblocks = -(-numel // block_size) if block_size > 0 else 0   # the last block may be short
     keep_absmax = (not double_quant) if keep_absmax is None else keep_absmax
-    codes = torch.empty(max(numel // 2, 1), dtype=torch.uint8, device=dev)
+    codes = torch.empty(max((numel + 1) // 2, 1), dtype=torch.uint8, device=dev)
     absmax = torch.empty(max(nblocks, 1), dtype=torch.float32, device=dev) if keep_absmax else None
     absmax_q = torch.empty(max(nblocks, 1), dtype=torch.uint8, device=dev) if double_quant else None
     absmax_scale = torch.empty(1, dtype=torch.float32, device=dev) if double_quant else None

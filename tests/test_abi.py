@@ -65,6 +65,8 @@ def test_workspace_sizes():
     assert Q.workspace_bytes(Q.OP_DEQUANTIZE, 0, 4096, 4096, 0, 64, False) == 0
     assert Q.workspace_bytes(Q.OP_QUANTIZE, 0, 4096, 4096, 0, 64, False) >= 256
     assert Q.workspace_bytes(Q.OP_QUANTIZE, 0, 4096, 4096, 0, 64, True) >= 256 + 4096 * 64 * 4
+    # a short last block is a block of its own: 3 blocks for 130 elements
+    assert Q.workspace_bytes(Q.OP_QUANTIZE, 0, 13, 10, 0, 64, True) >= 256 + 3 * 4
     assert Q.workspace_bytes(Q.OP_LINEAR_FWD, 4096, 11008, 4096, 64, 64, True) >= 256
     assert Q.workspace_bytes(Q.OP_LINEAR_BWD, 4096, 11008, 4096, 64, 64, True) >= 256
 
@@ -76,7 +78,9 @@ def _quant(rows, cols, bs, dq, w=FAKE, codes=FAKE, absmax=FAKE, aq=FAKE, asc=FAK
 def test_quantize_host_validation():
     assert _quant(4, 64, 63, 0) == 2          # odd block size
     assert _quant(4, 64, 0, 0) == 2
-    assert _quant(3, 10, 64, 0) == 2          # numel not a multiple of the block
+    # a short last block (30 elements, block 64) passes the shape checks and
+    # reaches the workspace check
+    assert _quant(3, 10, 64, 1, wsb=16) == 5
     assert _quant(4, 64, 64, 2) == 1          # double_quant must be 0/1
     assert _quant(4, 64, 64, 0, w=None) == 1
     assert _quant(4, 64, 64, 0, absmax=None) == 1
@@ -95,8 +99,12 @@ def _cw(rows=4096, cols=4096, bs=64, dq=1, codes=FAKE):
 
 def test_dequantize_host_validation():
     L = Q.lib()
-    assert L.nf4_dequantize(ctypes.byref(_cw(bs=6)), 0, FAKE, None) == 2
-    assert L.nf4_dequantize(ctypes.byref(_cw(rows=3, cols=8, bs=16)), 0, FAKE, None) == 2
+    assert L.nf4_dequantize(ctypes.byref(_cw(bs=7)), 0, FAKE, None) == 2        # odd block size
+    assert L.nf4_dequantize(ctypes.byref(_cw(bs=0)), 0, FAKE, None) == 2
+    # any even block size and a short last block pass the shape checks and
+    # reach the alignment check of `out`
+    assert L.nf4_dequantize(ctypes.byref(_cw(bs=6)), 0, FAKE + 2, None) == 3
+    assert L.nf4_dequantize(ctypes.byref(_cw(rows=3, cols=8, bs=16)), 0, FAKE + 2, None) == 3
     assert L.nf4_dequantize(ctypes.byref(_cw()), 7, FAKE, None) == 1
     assert L.nf4_dequantize(ctypes.byref(_cw(codes=None)), 0, FAKE, None) == 1
     assert L.nf4_dequantize(ctypes.byref(_cw()), 0, FAKE + 2, None) == 3

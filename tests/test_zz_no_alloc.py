@@ -19,9 +19,9 @@ pytestmark = pytest.mark.gpu
 def _noalloc(L, w, bs, dq, use_own_absmax):
     import torch
     numel = w.numel()
-    nb = numel // bs
+    nb = -(-numel // bs)                  # the last block may be short
     dev = w.device
-    codes = torch.empty(numel // 2, dtype=torch.uint8, device=dev)
+    codes = torch.empty((numel + 1) // 2, dtype=torch.uint8, device=dev)
     absmax = torch.empty(nb, dtype=torch.float32, device=dev) if (use_own_absmax or not dq) else None
     aq = torch.empty(nb, dtype=torch.uint8, device=dev) if dq else None
     asc = torch.empty(1, dtype=torch.float32, device=dev) if dq else None
@@ -37,7 +37,8 @@ def test_noalloc_matches_quantize_two_calls(cuda_device):
     from qlora_linear_layers_nf4_b200 import nf4qlora as Q
     L = Q.lib()
     weights = [WL.draw_weight((4096, 4096), seed=1, sigma=0.02),      # the 4096x4096 matrix
-               WL.draw_weight((768, 1024), seed=5, sigma=0.005)]      # smaller max: stale max would show
+               WL.draw_weight((768, 1024), seed=5, sigma=0.005),      # smaller max: stale max would show
+               WL.draw_weight((97, 45), seed=6, sigma=0.001)]         # a short, odd-sized last block
     for call, wn in enumerate(weights):
         w = torch.from_numpy(wn).to(cuda_device)
         for dq, own in ((True, False), (True, True), (False, True)):
