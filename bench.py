@@ -560,7 +560,33 @@ def measure_rows(args, dev, flush, pk, pk_kind, barrier):
         "method": "eager steps, L2 flushed before each; the f16 dense peak equals the bf16 one"}
     if wsf.read_status() != 0:
         raise RuntimeError("device status reported an error in the f16 row")
-    del qf, xf, dyf, yf, dxf
+    del xf, dyf, yf, dxf
+    torch.cuda.empty_cache()
+
+    # ---- the same layer in the F32 compute dtype (fp32 FMAs on the CUDA cores),
+    # against the fp32 ALU peak: SMs x 128 FP32 lanes x 2 FLOP x the max SM clock
+    xs, As_, Bs_, dys = (torch.from_numpy(np.ascontiguousarray(d32[k])).to(dev) for k in ("x", "a", "b", "dy"))
+    ys = torch.empty((case.m, case.n), dtype=torch.float32, device=dev)
+    Ts = torch.empty((case.m, case.r), dtype=torch.float32, device=dev)
+    dxs = torch.empty((case.m, case.k), dtype=torch.float32, device=dev)
+
+    def f32_step():
+        Q.linear_fwd(qf, xs, As_, Bs_, case.alpha, out=ys, t_out=Ts, workspace=wsf)
+        Q.linear_bwd(qf, xs, As_, Bs_, case.alpha, dys, t=Ts, dA=dAf, dB=dBf, dx=dxs, workspace=wsf)
+
+    ssteps = 3
+    ms = time_steps(f32_step, ssteps, 3, flush=flush, barrier=barrier)
+    tf = fl * ssteps / (ms * 1e-3) / 1e12
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    alu_peak = sms * 128 * 2 * 1.965e9 / 1e12
+    out["prefill_11008x4096_M4096_f32_fwd_bwd"] = {
+        "TFLOP/s": tf, "ms_per_step": ms / ssteps, "bound": "alu",
+        "peak_tflops": alu_peak, "frac_fp32_alu": tf / alu_peak,
+        "peak_source": f"derived: {sms} SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz (max SM clock)",
+        "method": "eager steps, L2 flushed before each"}
+    if wsf.read_status() != 0:
+        raise RuntimeError("device status reported an error in the f32 row")
+    del qf, xs, dys, ys, dxs, Ts
     torch.cuda.empty_cache()
 
     # ---- dense merge of the 11008x4096 layer with its r = 64 adapter (bf16 out),
@@ -667,6 +693,17 @@ def profile_row(args):
         A, B = bf16_dev(inp.a, dev), bf16_dev(inp.b, dev)
         for _ in range(n):
             Q.merge(q, A, B, case.alpha, "bf16", workspace=ws)
+    elif args.profile_row == "f32":
+        # the 11008x4096 layer, M = 4096, fwd + bwd in the F32 compute dtype:
+        # per step six gemm_f32 launches (T, y, U, dB, dA, dx)
+        case = WL.PREFILL
+        inp = WL.draw_linear(case)
+        q = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True)
+        d32 = inp.extra["f32"]
+        x, A, B, dy = (torch.from_numpy(d32[k]).to(dev) for k in ("x", "a", "b", "dy"))
+        for _ in range(n):
+            y, T = Q.linear_fwd(q, x, A, B, case.alpha, workspace=ws)
+            Q.linear_bwd(q, x, A, B, case.alpha, dy, t=T, workspace=ws)
     elif args.profile_row == "decode":
         base = WL.DECODE[0]
         q = Q.quantize(torch.from_numpy(WL.draw_weight((base.n, base.k), seed=200)).to(dev), 64, True)
@@ -729,7 +766,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-row", choices=["quantize", "dequantize", "decode", "merge"],
+    ap.add_argument("--profile-row", choices=["quantize", "dequantize", "decode", "merge", "f32"],
                     help="only launch one secondary row eagerly (for ncu); no bench line")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -268,15 +268,23 @@ NF4_API nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out,
  *                  K % 64 == 0, N % 8 == 0.
  *   x              [M, K] compute_dtype; M >= 1.
  *   A, B           [r, K] and [N, r] compute_dtype; 8 <= r <= 256, r % 8 == 0.
- *   compute_dtype  NF4_BF16 or NF4_F16 (NF4_F32 gives NF4_ERR_UNSUPPORTED).
+ *   compute_dtype  NF4_BF16, NF4_F16 or NF4_F32.  NF4_F32 is the pages'
+ *                  debugging mode (rust-ai-core QLoraConfig, "Compute
+ *                  Dtype"): x, A, B, bias, y, T (and dy, dx) fp32, W' the
+ *                  fp32 dequant itself (not rounded further), every product
+ *                  and sum an IEEE fp32 operation on the CUDA cores (no tf32
+ *                  rounding of the operands), s applied as one fp32 multiply.
+ *                  It is a reference mode: about 33x slower than BF16 on an
+ *                  11008 x 4096 layer with 4096 tokens.
  *   bias           [N] compute_dtype, or NULL.
  *   y              [M, N] compute_dtype, written.
  *   t_out          [M, r] compute_dtype, or NULL: when given, receives
  *                  T = s (x A^T) rounded to compute_dtype, which
  *                  qlora_linear_bwd accepts as `t`.
- *   workspace      >= nf4_workspace_bytes(NF4_OP_LINEAR_FWD, M, N, K, r, 64, dq).
- * M <= 32 uses the weight-streaming decode path, larger M the fused
- * dequantize + tensor-core GEMM; both compute the same function.
+ *   workspace      >= nf4_workspace_bytes(NF4_OP_LINEAR_FWD, M, N, K, r, 64, dq)
+ *                  (the same size serves every compute dtype).
+ * BF16 / F16: M <= 32 uses the weight-streaming decode path, larger M the
+ * fused dequantize + tensor-core GEMM; both compute the same function.
  */
 NF4_API nf4_status qlora_linear_fwd(const nf4_weight* w, const void* x, int64_t M, const void* A,
                             const void* B, int r, float alpha, int compute_dtype,

@@ -49,10 +49,8 @@ nf4_status check_linear(const nf4_weight* w, const void* x, int64_t M, const voi
     return NF4_ERR_INVALID_ARG;
   }
   if (!(alpha == alpha) || r < 8 || r > 256 || (r % 8) != 0) return NF4_ERR_INVALID_ARG;
-  if (compute_dtype != NF4_BF16 && compute_dtype != NF4_F16) {
-    if (compute_dtype == NF4_F32) return NF4_ERR_UNSUPPORTED;
+  if (compute_dtype != NF4_BF16 && compute_dtype != NF4_F16 && compute_dtype != NF4_F32)
     return NF4_ERR_INVALID_ARG;
-  }
   if (M < 1 || w->rows < 1 || w->cols < 1) return NF4_ERR_SHAPE;
   if (w->block_size != 64) return NF4_ERR_UNSUPPORTED;
   if (w->cols % 64 != 0 || w->rows % 8 != 0) return NF4_ERR_SHAPE;
@@ -83,7 +81,7 @@ double g_prof_ms[nf4::kNumKernelIds];
 
 const char* const kKernelNames[nf4::kNumKernelIds] = {
     "nf4_quantize", "nf4_double_quant", "nf4_dequantize", "adapter_gemm",
-    "fused_nf4_gemm_fwd", "fused_nf4_gemm_dx", "nf4_gemv", "nf4_merge"};
+    "fused_nf4_gemm_fwd", "fused_nf4_gemm_dx", "nf4_gemv", "nf4_merge", "gemm_f32"};
 
 cudaEvent_t prof_event() {
   if (!g_prof_free.empty()) {
@@ -327,6 +325,7 @@ nf4_status qlora_linear_fwd(const nf4_weight* w, const void* x, int64_t M, const
   a.r = r;
   a.s = alpha / float(r);
   a.f16 = compute_dtype == NF4_F16 ? 1 : 0;
+  a.f32 = compute_dtype == NF4_F32 ? 1 : 0;
   a.x = x;
   a.A = A;
   a.B = B;
@@ -337,8 +336,9 @@ nf4_status qlora_linear_fwd(const nf4_weight* w, const void* x, int64_t M, const
   a.ws_bytes = ws_bytes;
   a.status = reinterpret_cast<uint32_t*>(a.ws + nf4::kWsStatus);
   int launches = 0;
-  cudaError_t e = nf4::launch_linear_fwd(a, sm_count(), static_cast<cudaStream_t>(stream),
-                                         &launches);
+  cudaError_t e = a.f32 ? nf4::launch_linear_fwd_f32(a, static_cast<cudaStream_t>(stream), &launches)
+                        : nf4::launch_linear_fwd(a, sm_count(), static_cast<cudaStream_t>(stream),
+                                                 &launches);
   if (e == cudaErrorNotSupported) { g_launches += launches; return NF4_ERR_UNSUPPORTED; }
   return finish(e, launches);
 }
@@ -365,6 +365,7 @@ nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const
   a.r = r;
   a.s = alpha / float(r);
   a.f16 = compute_dtype == NF4_F16 ? 1 : 0;
+  a.f32 = compute_dtype == NF4_F32 ? 1 : 0;
   a.x = x;
   a.A = A;
   a.B = B;
@@ -377,8 +378,9 @@ nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const
   a.ws_bytes = ws_bytes;
   a.status = reinterpret_cast<uint32_t*>(a.ws + nf4::kWsStatus);
   int launches = 0;
-  cudaError_t e = nf4::launch_linear_bwd(a, sm_count(), static_cast<cudaStream_t>(stream),
-                                         &launches);
+  cudaError_t e = a.f32 ? nf4::launch_linear_bwd_f32(a, static_cast<cudaStream_t>(stream), &launches)
+                        : nf4::launch_linear_bwd(a, sm_count(), static_cast<cudaStream_t>(stream),
+                                                 &launches);
   if (e == cudaErrorNotSupported) { g_launches += launches; return NF4_ERR_UNSUPPORTED; }
   return finish(e, launches);
 }

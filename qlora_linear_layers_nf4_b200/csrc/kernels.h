@@ -30,6 +30,7 @@ struct LinearArgs {
   int r;
   float s;                 // alpha / r
   int f16;                 // compute type f16 (else bf16): x, A, B, bias, dy, y, dx, T, U
+  int f32;                 // compute type fp32 (the CUDA-core path); f16 is then 0
   const void* x;           // [M, K] bf16 / f16
   const void* A;           // [r, K] bf16
   const void* B;           // [N, r] bf16
@@ -63,6 +64,9 @@ bool decode_supported(int64_t M, int64_t N, int64_t K, int r);
 cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
+// The F32 compute dtype (f32_gemm.cu): fp32 operands and outputs, CUDA-core fp32 FMAs.
+cudaError_t launch_linear_fwd_f32(const LinearArgs& a, cudaStream_t stream, int* launches);
+cudaError_t launch_linear_bwd_f32(const LinearArgs& a, cudaStream_t stream, int* launches);
 
 // Bounded-wait self-check (selfcheck.cu): waits that nothing completes give
 // up after limit_ns, record NF4_ERR_TIMEOUT in *status and raise the abort
@@ -88,6 +92,7 @@ enum KernelId {
   kKFusedDx,
   kKGemv,
   kKMerge,
+  kKGemmF32,
   kNumKernelIds
 };
 

@@ -1182,7 +1182,9 @@ FusedParams fused_params(const LinearArgs& a, int mode) {
 // Workspace regions after the header (256-byte aligned):
 //   fwd: [T bf16 M x r (when t_out is null)]
 //   bwd: [T bf16 M x r (when t is null)] [U bf16 M x r]
-size_t mr_bytes(int64_t M, int r) { return align256(size_t(M) * size_t(r) * 2); }
+// One [M, r] scratch matrix (T or U), sized for 4-byte elements so that the
+// same workspace serves every compute dtype (the F32 path keeps them in fp32).
+size_t mr_bytes(int64_t M, int r) { return align256(size_t(M) * size_t(r) * 4); }
 
 cudaError_t forward_adapter_T(const LinearArgs& a, __nv_bfloat16* T, int sms, cudaStream_t st,
                               int* launches) {

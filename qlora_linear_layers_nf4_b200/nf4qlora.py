@@ -277,21 +277,24 @@ def merge(q: QuantizedWeight, A, B, alpha: float, out_dtype: str = "bf16", out=N
 
 
 def _compute_dtype(x):
-    """The C ABI's compute type for activations of x's dtype (bf16 or f16)."""
+    """The C ABI's compute type for activations of x's dtype: bf16, f16, or
+    fp32 (the CUDA-core fp32 reference mode)."""
     import torch
     if x.dtype == torch.bfloat16:
         return NF4_BF16
     if x.dtype == torch.float16:
         return NF4_F16
-    raise TypeError(f"compute dtype must be bfloat16 or float16, got {x.dtype}")
+    if x.dtype == torch.float32:
+        return NF4_F32
+    raise TypeError(f"compute dtype must be bfloat16, float16 or float32, got {x.dtype}")
 
 
 def linear_fwd(q: QuantizedWeight, x, A, B, alpha: float, bias=None, want_t: bool = True,
                out=None, t_out=None, workspace: Workspace | None = None, stream=None):
     """y = x W'^T + (alpha/r) (x A^T) B^T (+ bias); returns (y, T or None).
 
-    x, A, B (and bias) share one compute dtype, bfloat16 or float16; y and T
-    come back in it."""
+    x, A, B (and bias) share one compute dtype, bfloat16, float16 or float32
+    (the fp32 reference mode); y and T come back in it."""
     import torch
     dt = _compute_dtype(x)
     M = x.shape[0]

@@ -120,7 +120,8 @@ def test_linear_host_validation():
     assert _fwd(_cw(), r=12) == 1                 # r % 8
     assert _fwd(_cw(), r=512) == 1
     assert _fwd(_cw(), dtype=2, wsb=0) == 5       # F16 compute passes the dtype check
-    assert _fwd(_cw(), dtype=0) == 4              # F32 compute: not in this build
+    assert _fwd(_cw(), dtype=0, wsb=0) == 5       # F32 compute accepted: reaches the workspace check
+    assert _fwd(_cw(), dtype=3) == 1              # no such dtype
     assert _fwd(_cw(), dtype=9) == 1
     assert _fwd(_cw(), M=0) == 2
     assert _fwd(_cw(cols=4000)) == 2              # K % 64
