@@ -231,6 +231,34 @@ NF4_API nf4_status nf4_quantize_typed(const void* w, int in_dtype, int64_t rows,
                                       void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * The two halves of the simplified double quant, for a tensor whose rows are
+ * quantized on several ranks (data parallel): each rank quantizes its shard
+ * with double_quant = 0 and keeps its fp32 block scales, takes their max with
+ * nf4_absmax_max, the ranks all-reduce that float with MAX (the one exchange;
+ * NCCL over NVLink), and each rank then encodes its scales against the global
+ * max with nf4_double_quant.  With shards that start on block boundaries the
+ * result is bit for bit the rows of a single-device nf4_quantize with
+ * double_quant = 1 (qlora-rs README, "Double quantization (simplified)": one
+ * scale of scales for the whole tensor).
+ *
+ * nf4_absmax_max: gmax[0] = max over absmax[0 .. n_blocks) (all >= 0; 0 for
+ *   n_blocks == 0).  absmax fp32 [n_blocks] and gmax fp32 [1] are device
+ *   memory, 4-byte aligned; gmax is overwritten.  Enqueued on `stream`.
+ */
+NF4_API nf4_status nf4_absmax_max(const float* absmax, int64_t n_blocks, float* gmax, void* stream);
+
+/*
+ * nf4_double_quant: with G = gmax[0] (device, >= 0, normally the global max
+ *   of the block scales), absmax_scale[0] = fp32(G / 255) and absmax_q[b] =
+ *   clamp(rint(absmax[b] / absmax_scale[0]), 0, 255), ties to even; G == 0
+ *   gives 0 and 0 -- exactly the double-quant stage of nf4_quantize.
+ *   absmax fp32 [n_blocks] and absmax_q u8 [n_blocks] 16-byte aligned;
+ *   absmax_scale fp32 [1] and gmax 4-byte aligned.  Enqueued on `stream`.
+ */
+NF4_API nf4_status nf4_double_quant(const float* absmax, int64_t n_blocks, const float* gmax,
+                                    uint8_t* absmax_q, float* absmax_scale, void* stream);
+
+/*
  * Self-check of the bounded-wait path (no counterpart on the pages).  Every
  * mbarrier wait in the library's kernels gives up after a time limit, records
  * NF4_ERR_TIMEOUT in the workspace status word and raises its CTA's abort

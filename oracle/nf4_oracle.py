@@ -149,15 +149,20 @@ def unpack_codes(packed: np.ndarray) -> np.ndarray:
     return out
 
 
-def double_quant(absmax: np.ndarray):
+def double_quant(absmax: np.ndarray, g=None):
     """Simplified double quant of the block scales (reading R6).
 
     [P1] "Double quantization (simplified)": the block scales become u8 codes
     with one scale-of-scales; [P3] stores them as scales_quantized (u8) and
-    scales_scales (f32).
+    scales_scales (f32).  The scale of scales belongs to the whole tensor:
+    `g`, when given, is the max over all of the tensor's block scales (for a
+    part of a tensor whose other blocks are elsewhere); by default it is the
+    max of `absmax` itself.
     """
     absmax = np.asarray(absmax, dtype=np.float32)
-    g = np.float32(absmax.max()) if absmax.size else np.float32(0.0)
+    if g is None:
+        g = np.float32(absmax.max()) if absmax.size else np.float32(0.0)
+    g = np.float32(g)
     if g == 0.0:
         return np.zeros(absmax.size, dtype=np.uint8), np.float32(0.0)
     s_g = np.float32(g / np.float32(255.0))

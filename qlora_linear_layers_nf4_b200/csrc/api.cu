@@ -81,7 +81,7 @@ double g_prof_ms[nf4::kNumKernelIds];
 
 const char* const kKernelNames[nf4::kNumKernelIds] = {
     "nf4_quantize", "nf4_double_quant", "nf4_dequantize", "adapter_gemm",
-    "fused_nf4_gemm_fwd", "fused_nf4_gemm_dx", "nf4_gemv", "nf4_merge", "gemm_f32"};
+    "fused_nf4_gemm_fwd", "fused_nf4_gemm_dx", "nf4_gemv", "nf4_merge", "gemm_f32", "nf4_absmax_max"};
 
 cudaEvent_t prof_event() {
   if (!g_prof_free.empty()) {
@@ -279,6 +279,31 @@ nf4_status nf4_quantize_typed(const void* w, int in_dtype, int64_t rows, int64_t
   if (in_dtype != NF4_F32 && in_dtype != NF4_BF16 && in_dtype != NF4_F16) return NF4_ERR_INVALID_ARG;
   return quantize_impl(w, in_dtype, rows, cols, block_size, double_quant, codes, absmax, absmax_q,
                        absmax_scale, workspace, ws_bytes, stream);
+}
+
+nf4_status nf4_absmax_max(const float* absmax, int64_t n_blocks, float* gmax, void* stream) {
+  if (n_blocks < 0) return NF4_ERR_SHAPE;
+  if (gmax == nullptr || (n_blocks > 0 && absmax == nullptr)) return NF4_ERR_INVALID_ARG;
+  if (!aligned4(gmax) || (absmax && !aligned4(absmax))) return NF4_ERR_ALIGNMENT;
+  int launches = 0;
+  cudaError_t e = nf4::launch_absmax_max(absmax, n_blocks, reinterpret_cast<uint32_t*>(gmax),
+                                         sm_count(), static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
+}
+
+nf4_status nf4_double_quant(const float* absmax, int64_t n_blocks, const float* gmax,
+                            uint8_t* absmax_q, float* absmax_scale, void* stream) {
+  if (n_blocks < 0) return NF4_ERR_SHAPE;
+  if (gmax == nullptr || absmax_scale == nullptr) return NF4_ERR_INVALID_ARG;
+  if (n_blocks > 0 && (absmax == nullptr || absmax_q == nullptr)) return NF4_ERR_INVALID_ARG;
+  if (!aligned4(gmax) || !aligned4(absmax_scale) || (absmax && !aligned16(absmax)) ||
+      (absmax_q && !aligned16(absmax_q)))
+    return NF4_ERR_ALIGNMENT;
+  int launches = 0;
+  cudaError_t e = nf4::launch_double_quant(absmax, n_blocks, reinterpret_cast<const uint32_t*>(gmax),
+                                           absmax_q, absmax_scale, sm_count(),
+                                           static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches);
 }
 
 nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out, void* stream) {

@@ -18,6 +18,9 @@ cudaError_t launch_quantize(const void* w, int in_dtype, int64_t numel, int bs, 
 cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uint32_t* gmax,
                                 uint8_t* absmax_q, float* absmax_scale, int sms,
                                 cudaStream_t stream, int* launches);
+// Max of n non-negative fp32 scales into *gmax (bits), zeroing it first.
+cudaError_t launch_absmax_max(const float* absmax, int64_t n, uint32_t* gmax, int sms,
+                              cudaStream_t stream, int* launches);
 
 cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int sms,
                               cudaStream_t stream, int* launches);
@@ -93,6 +96,7 @@ enum KernelId {
   kKGemv,
   kKMerge,
   kKGemmF32,
+  kKAbsmaxMax,
   kNumKernelIds
 };
 

@@ -305,6 +305,18 @@ __global__ void __launch_bounds__(256) double_quant_kernel(
   if (tail < n_blocks) absmax_q[tail] = uint8_t(dq_code(at, g, s_g, fast, y));
 }
 
+// Max of n non-negative fp32 block scales into *gmax (bits; zeroed by the
+// caller): the global max of the simplified double quant when the scales of
+// one tensor are spread over several ranks.
+__global__ void __launch_bounds__(256) absmax_max_kernel(const float* __restrict__ absmax,
+                                                         int64_t n, uint32_t* __restrict__ gmax) {
+  float m = 0.0f;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
+    m = fmaxf(m, __ldg(absmax + i));
+  cta_global_max(m, gmax);
+}
+
 // ------------------------------------------------------------------ dequant
 
 template <typename OutT>
@@ -509,6 +521,20 @@ cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uin
                                      absmax_scale);
   NF4_PROF_END(stream, kKDoubleQuant);
   if (e == cudaSuccess) e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+cudaError_t launch_absmax_max(const float* absmax, int64_t n, uint32_t* gmax, int sms,
+                              cudaStream_t stream, int* launches) {
+  cudaError_t e = cudaMemsetAsync(gmax, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return e;
+  if (n <= 0) return cudaSuccess;
+  const int grid = grid_for(n, 256, sms, 2);
+  NF4_PROF_BEGIN(stream, kKAbsmaxMax);
+  absmax_max_kernel<<<grid, 256, 0, stream>>>(absmax, n, gmax);
+  NF4_PROF_END(stream, kKAbsmaxMax);
+  e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;
 }

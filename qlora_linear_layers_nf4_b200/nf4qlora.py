@@ -28,7 +28,8 @@ EXPORTED = (
     "nf4_profile_begin", "nf4_profile_end", "nf4_profile_kernel_count", "nf4_kernel_name",
     "nf4_profile_get", "nf4_workspace_bytes", "nf4_read_status", "nf4_quantize",
     "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "nf4_quantize_noalloc",
-    "nf4_merge", "nf4_quantize_typed", "nf4_check_wait_timeout",
+    "nf4_merge", "nf4_quantize_typed", "nf4_check_wait_timeout", "nf4_absmax_max",
+    "nf4_double_quant",
 )
 
 
@@ -102,6 +103,10 @@ def lib() -> ctypes.CDLL:
     L.nf4_quantize_typed.restype = i32
     L.nf4_check_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, ctypes.POINTER(ctypes.c_uint32), vp]
     L.nf4_check_wait_timeout.restype = i32
+    L.nf4_absmax_max.argtypes = [vp, i64, vp, vp]
+    L.nf4_absmax_max.restype = i32
+    L.nf4_double_quant.argtypes = [vp, i64, vp, vp, vp, vp]
+    L.nf4_double_quant.restype = i32
     _lib = L
     return L
 
@@ -247,6 +252,26 @@ def quantize(w, block_size: int = 64, double_quant: bool = False, keep_absmax: b
     if check_status:
         _check(ws.read_status(stream), "nf4_quantize (device)")
     return QuantizedWeight(codes, absmax, absmax_q, absmax_scale, rows, cols, block_size, double_quant)
+
+
+def absmax_max(absmax, stream=None):
+    """Max of a CUDA fp32 tensor of block scales, as a 1-element CUDA tensor."""
+    import torch
+    g = torch.empty(1, dtype=torch.float32, device=absmax.device)
+    _check(lib().nf4_absmax_max(_ptr(absmax), absmax.numel(), _ptr(g), _stream(stream)), "nf4_absmax_max")
+    return g
+
+
+def double_quant(absmax, gmax, stream=None):
+    """The double-quant stage against a given global max (1-element CUDA
+    tensor): returns (absmax_q uint8 [n], absmax_scale fp32 [1])."""
+    import torch
+    n = absmax.numel()
+    aq = torch.empty(max(n, 1), dtype=torch.uint8, device=absmax.device)
+    asc = torch.empty(1, dtype=torch.float32, device=absmax.device)
+    _check(lib().nf4_double_quant(_ptr(absmax), n, _ptr(gmax), _ptr(aq), _ptr(asc), _stream(stream)),
+           "nf4_double_quant")
+    return aq, asc
 
 
 def dequantize(q: QuantizedWeight, out_dtype: str = "f32", stream=None):

@@ -172,3 +172,17 @@ def test_bucket_encoding_conditions():
     assert np.min(np.abs(th[:, None] - edges[None, :])) > 2.0 ** -20
     counts = [np.sum((th >= edges[j]) & (th < edges[j] + 1 / 32)) for j in range(64)]
     assert max(counts) <= 1
+
+
+def test_sharded_double_quant_host_validation():
+    L = Q.lib()
+    assert L.nf4_absmax_max(FAKE, -1, FAKE, None) == 2
+    assert L.nf4_absmax_max(FAKE, 4, None, None) == 1
+    assert L.nf4_absmax_max(None, 4, FAKE, None) == 1
+    assert L.nf4_absmax_max(FAKE + 2, 4, FAKE, None) == 3
+    assert L.nf4_double_quant(FAKE, -1, FAKE, FAKE, FAKE, None) == 2
+    assert L.nf4_double_quant(FAKE, 4, None, FAKE, FAKE, None) == 1
+    assert L.nf4_double_quant(FAKE, 4, FAKE, None, FAKE, None) == 1
+    assert L.nf4_double_quant(FAKE, 4, FAKE, FAKE, None, None) == 1
+    assert L.nf4_double_quant(FAKE + 4, 4, FAKE, FAKE, FAKE, None) == 3   # absmax 16-byte aligned
+    assert L.nf4_double_quant(FAKE, 4, FAKE, FAKE + 4, FAKE, None) == 3

@@ -460,3 +460,31 @@ def test_tail_block_double_quant_counts_every_block():
     q = O.quantize(w, 64, double=True)
     assert q["absmax_q"].size == 16                   # 15 full blocks + the tail
     assert q["absmax_q"].max() == 255
+
+
+# --------------------------------------------------------------------------- a part of a tensor (R6)
+
+def test_double_quant_of_a_part_uses_the_whole_max():
+    # One scale of scales per tensor: the blocks of a part, encoded against the
+    # tensor's max, are exactly those blocks of the whole tensor's encoding.
+    w = WL.draw_weight((48, 256), seed=21)
+    w[40:] *= np.float32(6.0)                              # the max lies in the last part
+    whole = O.quantize(w, 64, double=True)
+    g = np.float32(whole["absmax"].max())
+    parts = [w[:16], w[16:40], w[40:]]
+    qs, ss = [], []
+    for part in parts:
+        qp = O.quantize(part, 64, double=False)
+        q, s = O.double_quant(qp["absmax"], g=g)
+        qs.append(q)
+        ss.append(s)
+    assert np.array_equal(np.concatenate(qs), whole["absmax_q"])
+    assert all(s == np.float32(whole["absmax_scale"]) for s in ss)
+    # a part encoded against its own max differs: the exchange is needed
+    own, _ = O.double_quant(O.quantize(parts[0], 64)["absmax"])
+    assert not np.array_equal(own, qs[0])
+    # the default max is the part's own
+    a = O.quantize(parts[1], 64)["absmax"]
+    q_default, s_default = O.double_quant(a)
+    q_given, s_given = O.double_quant(a, g=a.max())
+    assert np.array_equal(q_default, q_given) and s_default == s_given
