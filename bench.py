@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -78,7 +79,10 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # the raw samples (the JSON line carries their summary); BENCH_OUT_DIR
+        # keeps them with a run's other outputs
+        out_dir = os.environ.get("BENCH_OUT_DIR", tempfile.gettempdir())
+        self.path = os.path.join(out_dir, f"nf4_bench_clocks_gpu{gpu_index}.csv")
 
     def start(self):
         try:

@@ -24,7 +24,7 @@ follows):
        (alpha/r scaling), "NF4: quantizing the frozen base" (levels at normal
        quantiles, equally likely), "The merge math" (equation 6.3.6).
 
-Readings of points the pages leave open (each is also listed in the design doc):
+Readings of points the pages leave open:
   R1  NF4 construction: the pages print the levels to three decimals and say
       they sit at normal quantiles; the formula itself (equations 6.3.4-6.3.5)
       did not survive.  Reading: 8 positive quantiles
@@ -55,6 +55,9 @@ Readings of points the pages leave open (each is also listed in the design doc):
   R19 A tensor whose size is not a multiple of the block: the last block holds
       the remaining elements and its absmax is theirs alone; for an odd
       element count the last byte's low nibble is 7 (the exact-zero level).
+  R20 F32 compute (listed as honoured, called the debugging mode): the base
+      is the fp32 dequant w' itself, not rounded further; the forward and
+      backward below are evaluated in fp64 from it and the fp32 inputs.
 """
 from __future__ import annotations
 
