@@ -14,7 +14,8 @@ the seven-target decoder block).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Under torchrun each rank runs the same layer on its own 4096 tokens (weak
-scaling) and the adapter gradients are all-reduced over NCCL each step.
+scaling) and the adapter gradients are all-reduced over NCCL each step; the
+secondary rows and the CPU baseline are taken at N = 1 only.
 --impl reference times the CPU oracle instead (rank 0 only).
 """
 from __future__ import annotations
@@ -373,8 +374,10 @@ def run_ours(args):
                          "while the previous step computes; dA, dB copied back every step; "
                          "L2 flushed before each step's compute"}
 
+    # The secondary rows are single-GPU kernel figures: taken at N = 1 only, so
+    # a multi-GPU run holds its GPUs for the data-parallel step alone.
     rows = {}
-    if not args.no_rows:
+    if not args.no_rows and world == 1:
         rows = measure_rows(args, dev, flush, pk, pk_kind, barrier)
 
     cpu = None
