@@ -8,6 +8,7 @@
 
 #include "nf4_common.cuh"
 #include "kernels.h"
+#include "nvtx_range.h"
 
 namespace {
 
@@ -268,6 +269,7 @@ extern "C" {
 nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int block_size,
                         int double_quant, uint8_t* codes, float* absmax, uint8_t* absmax_q,
                         float* absmax_scale, void* workspace, size_t ws_bytes, void* stream) {
+  NF4_API_RANGE("nf4_quantize");
   return quantize_impl(w, NF4_F32, rows, cols, block_size, double_quant, codes, absmax, absmax_q,
                        absmax_scale, workspace, ws_bytes, stream);
 }
@@ -276,12 +278,14 @@ nf4_status nf4_quantize_typed(const void* w, int in_dtype, int64_t rows, int64_t
                               int block_size, int double_quant, uint8_t* codes, float* absmax,
                               uint8_t* absmax_q, float* absmax_scale, void* workspace,
                               size_t ws_bytes, void* stream) {
+  NF4_API_RANGE("nf4_quantize_typed");
   if (in_dtype != NF4_F32 && in_dtype != NF4_BF16 && in_dtype != NF4_F16) return NF4_ERR_INVALID_ARG;
   return quantize_impl(w, in_dtype, rows, cols, block_size, double_quant, codes, absmax, absmax_q,
                        absmax_scale, workspace, ws_bytes, stream);
 }
 
 nf4_status nf4_absmax_max(const float* absmax, int64_t n_blocks, float* gmax, void* stream) {
+  NF4_API_RANGE("nf4_absmax_max");
   if (n_blocks < 0) return NF4_ERR_SHAPE;
   if (gmax == nullptr || (n_blocks > 0 && absmax == nullptr)) return NF4_ERR_INVALID_ARG;
   if (!aligned4(gmax) || (absmax && !aligned4(absmax))) return NF4_ERR_ALIGNMENT;
@@ -293,6 +297,7 @@ nf4_status nf4_absmax_max(const float* absmax, int64_t n_blocks, float* gmax, vo
 
 nf4_status nf4_double_quant(const float* absmax, int64_t n_blocks, const float* gmax,
                             uint8_t* absmax_q, float* absmax_scale, void* stream) {
+  NF4_API_RANGE("nf4_double_quant");
   if (n_blocks < 0) return NF4_ERR_SHAPE;
   if (gmax == nullptr || absmax_scale == nullptr) return NF4_ERR_INVALID_ARG;
   if (n_blocks > 0 && (absmax == nullptr || absmax_q == nullptr)) return NF4_ERR_INVALID_ARG;
@@ -307,6 +312,7 @@ nf4_status nf4_double_quant(const float* absmax, int64_t n_blocks, const float* 
 }
 
 nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out, void* stream) {
+  NF4_API_RANGE("nf4_dequantize");
   if (w == nullptr || out == nullptr || w->codes == nullptr) return NF4_ERR_INVALID_ARG;
   if (out_dtype != NF4_F32 && out_dtype != NF4_BF16 && out_dtype != NF4_F16)
     return NF4_ERR_INVALID_ARG;
@@ -333,6 +339,7 @@ nf4_status qlora_linear_fwd(const nf4_weight* w, const void* x, int64_t M, const
                             const void* B, int r, float alpha, int compute_dtype,
                             const void* bias, void* y, void* t_out, void* workspace,
                             size_t ws_bytes, void* stream) {
+  NF4_API_RANGE("qlora_linear_fwd");
   nf4_status s = check_linear(w, x, M, A, B, r, alpha, compute_dtype);
   if (s != NF4_OK) return s;
   if (y == nullptr) return NF4_ERR_INVALID_ARG;
@@ -372,6 +379,7 @@ nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const
                             const void* B, int r, float alpha, int compute_dtype,
                             const void* dy, const void* t, float* dA, float* dB, void* dx,
                             void* workspace, size_t ws_bytes, void* stream) {
+  NF4_API_RANGE("qlora_linear_bwd");
   nf4_status s = check_linear(w, x, M, A, B, r, alpha, compute_dtype);
   if (s != NF4_OK) return s;
   if (dy == nullptr || dA == nullptr || dB == nullptr) return NF4_ERR_INVALID_ARG;
@@ -412,6 +420,7 @@ nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const
 
 nf4_status nf4_check_wait_timeout(void* workspace, size_t ws_bytes, uint32_t limit_us,
                                   uint32_t* released, void* stream) {
+  NF4_API_RANGE("nf4_check_wait_timeout");
   if (workspace == nullptr || !aligned16(workspace) || ws_bytes < nf4::kWsHeader) return NF4_ERR_WORKSPACE;
   if (released == nullptr || limit_us < 1 || limit_us > 1000000) return NF4_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -435,6 +444,7 @@ nf4_status nf4_check_wait_timeout(void* workspace, size_t ws_bytes, uint32_t lim
 
 nf4_status nf4_merge(const nf4_weight* w, const void* A, const void* B, int r, float alpha,
                      int out_dtype, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  NF4_API_RANGE("nf4_merge");
   // the linear checks with a stand-in x (the merge has no activations)
   nf4_status s = check_linear(w, A, 1, A, B, r, alpha, NF4_BF16);
   if (s != NF4_OK) return s;

@@ -21,6 +21,7 @@
 
 #include "kernels.h"
 #include "nf4_common.cuh"
+#include "nvtx_range.h"
 
 namespace nf4 {
 namespace {
@@ -64,6 +65,7 @@ extern "C" nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t
                                            int block_size, int double_quant, uint8_t* codes,
                                            float* absmax, uint8_t* absmax_q, float* absmax_scale,
                                            void* stream) {
+  NF4_API_RANGE("nf4_quantize_noalloc");
   using namespace nf4;
   if (rows < 0 || cols < 0) return NF4_ERR_SHAPE;
   if (block_size <= 0 || (block_size % 2) != 0) return NF4_ERR_SHAPE;
