@@ -289,7 +289,13 @@ def merge(q: QuantizedWeight, A, B, alpha: float, out_dtype: str = "bf16", out=N
     """Dense merged weight dequant(W) + (alpha/r) B A, [rows, cols] in bf16 or f32."""
     import torch
     dt = {"f32": (NF4_F32, torch.float32), "bf16": (NF4_BF16, torch.bfloat16)}[out_dtype]
+    if A.dim() != 2:
+        raise ValueError("A must be 2-D ([r, K])")
     r = A.shape[0]
+    dev = q.device
+    _expect("A", A, (r, q.cols), torch.bfloat16, dev)
+    _expect("B", B, (q.rows, r), torch.bfloat16, dev)
+    _expect("out", out, (q.rows, q.cols), dt[1], dev)
     if out is None:
         out = torch.empty((q.rows, q.cols), dtype=dt[1], device=q.device)
     ws = workspace if workspace is not None else Workspace(q.device)
@@ -314,6 +320,27 @@ def _compute_dtype(x):
     raise TypeError(f"compute dtype must be bfloat16, float16 or float32, got {x.dtype}")
 
 
+def _expect(name: str, t, shape, dtype, device):
+    """The C ABI sees only a pointer: a tensor of the wrong shape, dtype,
+    layout or device would be read as garbage, so the binding refuses it."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the weight on {device}")
+
+
+def _linear_shapes(q: QuantizedWeight, x, A):
+    if x.dim() != 2 or A.dim() != 2:
+        raise ValueError("x and A must be 2-D ([M, K] and [r, K])")
+    return int(x.shape[0]), int(A.shape[0]), q.rows, q.cols
+
+
 def linear_fwd(q: QuantizedWeight, x, A, B, alpha: float, bias=None, want_t: bool = True,
                out=None, t_out=None, workspace: Workspace | None = None, stream=None):
     """y = x W'^T + (alpha/r) (x A^T) B^T (+ bias); returns (y, T or None).
@@ -322,8 +349,14 @@ def linear_fwd(q: QuantizedWeight, x, A, B, alpha: float, bias=None, want_t: boo
     (the fp32 reference mode); y and T come back in it."""
     import torch
     dt = _compute_dtype(x)
-    M = x.shape[0]
-    r = A.shape[0]
+    M, r, N, K = _linear_shapes(q, x, A)
+    dev = q.device
+    _expect("x", x, (M, K), x.dtype, dev)
+    _expect("A", A, (r, K), x.dtype, dev)
+    _expect("B", B, (N, r), x.dtype, dev)
+    _expect("bias", bias, (N,), x.dtype, dev)
+    _expect("out", out, (M, N), x.dtype, dev)
+    _expect("t_out", t_out, (M, r), x.dtype, dev)
     y = out if out is not None else torch.empty((M, q.rows), dtype=x.dtype, device=x.device)
     if want_t and t_out is None:
         t_out = torch.empty((M, r), dtype=x.dtype, device=x.device)
@@ -342,8 +375,16 @@ def linear_bwd(q: QuantizedWeight, x, A, B, alpha: float, dy, t=None, want_dx: b
     """Adapter backward; returns (dA fp32 [r,K], dB fp32 [N,r], dx [M,K] in x's dtype or None)."""
     import torch
     dt = _compute_dtype(x)
-    M = x.shape[0]
-    r = A.shape[0]
+    M, r, N, K = _linear_shapes(q, x, A)
+    dev = q.device
+    _expect("x", x, (M, K), x.dtype, dev)
+    _expect("A", A, (r, K), x.dtype, dev)
+    _expect("B", B, (N, r), x.dtype, dev)
+    _expect("dy", dy, (M, N), x.dtype, dev)
+    _expect("t", t, (M, r), x.dtype, dev)
+    _expect("dA", dA, (r, K), torch.float32, dev)
+    _expect("dB", dB, (N, r), torch.float32, dev)
+    _expect("dx", dx, (M, K), x.dtype, dev)
     dA = dA if dA is not None else torch.empty((r, q.cols), dtype=torch.float32, device=x.device)
     dB = dB if dB is not None else torch.empty((q.rows, r), dtype=torch.float32, device=x.device)
     if want_dx and dx is None:

@@ -186,3 +186,45 @@ def test_sharded_double_quant_host_validation():
     assert L.nf4_double_quant(FAKE, 4, FAKE, FAKE, None, None) == 1
     assert L.nf4_double_quant(FAKE + 4, 4, FAKE, FAKE, FAKE, None) == 3   # absmax 16-byte aligned
     assert L.nf4_double_quant(FAKE, 4, FAKE, FAKE + 4, FAKE, None) == 3
+
+
+def _cpu_weight(rows=64, cols=128):
+    import torch
+    return Q.QuantizedWeight(codes=torch.zeros(rows * cols // 2, dtype=torch.uint8),
+                             absmax=torch.zeros(rows * cols // 64, dtype=torch.float32),
+                             absmax_q=None, absmax_scale=None, rows=rows, cols=cols,
+                             block_size=64, double_quant=False)
+
+
+def test_binding_refuses_mismatched_tensors():
+    # Checked in the binding before anything reaches the C ABI (which sees
+    # only pointers), so these run without a GPU.
+    import torch
+    q = _cpu_weight()
+    bf, f16 = torch.bfloat16, torch.float16
+    x = torch.zeros(8, 128, dtype=bf)
+    A = torch.zeros(16, 128, dtype=bf)
+    B = torch.zeros(64, 16, dtype=bf)
+    with pytest.raises(TypeError):
+        Q.linear_fwd(q, x, A.to(f16), B, 32.0)                  # A in another dtype than x
+    with pytest.raises(ValueError):
+        Q.linear_fwd(q, x, torch.zeros(16, 64, dtype=bf), B, 32.0)   # A's K is not the weight's
+    with pytest.raises(ValueError):
+        Q.linear_fwd(q, x, A, torch.zeros(32, 16, dtype=bf), 32.0)   # B's N is not the weight's
+    with pytest.raises(ValueError):
+        Q.linear_fwd(q, x, A, B.t().contiguous().t(), 32.0)          # not row-major
+    with pytest.raises(ValueError):
+        Q.linear_fwd(q, x, A, B, 32.0, bias=torch.zeros(63, dtype=bf))
+    with pytest.raises(TypeError):
+        Q.linear_fwd(q, x.to(torch.int32), A, B, 32.0)               # no such compute dtype
+    dy = torch.zeros(8, 64, dtype=bf)
+    with pytest.raises(ValueError):
+        Q.linear_bwd(q, x, A, B, 32.0, torch.zeros(8, 63, dtype=bf))
+    with pytest.raises(TypeError):
+        Q.linear_bwd(q, x, A, B, 32.0, dy, dA=torch.zeros(16, 128, dtype=bf))   # dA is fp32
+    with pytest.raises(ValueError):
+        Q.linear_bwd(q, x, A, B, 32.0, dy, t=torch.zeros(8, 8, dtype=bf))
+    with pytest.raises(TypeError):
+        Q.merge(q, A.to(f16), B, 32.0)                               # merge adapters are bf16
+    with pytest.raises(ValueError):
+        Q.merge(q, A, B, 32.0, "bf16", out=torch.zeros(64, 64, dtype=bf))
