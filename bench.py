@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the hash of the kernel source it was taken on (see profiles/); reported as
 # null once the source changes.
 NCU_TRAFFIC = {
-    # profiles/fused_nf4_gemm_pair_11008x4096_M4096.md: forward 126.3 MB, dx 183.3 MB per launch
-    "fa61b052feb383c2": {"fwd": 126_256_640, "dx": 183_307_008},
+    # profiles/fused_nf4_gemm_pair_11008x4096_M4096.md: forward 124.3 MB, dx 178.8 MB per launch
+    "f29217272332d356": {"fwd": 124_325_632, "dx": 178_798_080},
 }
 
 

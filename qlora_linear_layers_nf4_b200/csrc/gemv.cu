@@ -501,15 +501,16 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
     if (f16) return n8 == 1 ? nf4_gemv<1, true> : (n8 == 2 ? nf4_gemv<2, true> : nf4_gemv<4, true>);
     return n8 == 1 ? nf4_gemv<1, false> : (n8 == 2 ? nf4_gemv<2, false> : nf4_gemv<4, false>);
   };
-  static bool attr_done[6] = {false, false, false, false, false, false};
+  static PerDeviceOnce attr_done[6];
   const int slot = (nt8 == 1 ? 0 : (nt8 == 2 ? 1 : 2)) + (a.f16 ? 3 : 0);
   auto* kernel = kernel_for(nt8, a.f16 != 0);
   cudaError_t e = cudaSuccess;
-  if (!attr_done[slot]) {
+  const int dev = PerDeviceOnce::current();
+  if (!attr_done[slot].done(dev)) {
     const int max_smem = 190 * 1024;   // + the 32 KB static lookup table
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     if (e != cudaSuccess) return e;
-    attr_done[slot] = true;
+    attr_done[slot].mark(dev);
   }
   NF4_PROF_BEGIN(st, kKGemv);
   e = cudaLaunchKernelEx(&cfg, kernel, tc, tx, ta, tb, p);

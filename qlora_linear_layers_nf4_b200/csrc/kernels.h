@@ -2,6 +2,7 @@
 // and increments *launches once per kernel it launched successfully.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -9,6 +10,24 @@
 #include "../../include/nf4qlora.h"
 
 namespace nf4 {
+
+// One-time setup per device (a kernel's shared-memory opt-in applies to the
+// current device only): one bit per device index, set atomically, so that
+// several host threads or several devices in one process are safe.  Two
+// threads may both run the setup once; it is idempotent.
+struct PerDeviceOnce {
+  std::atomic<uint64_t> bits{0};
+  static int current() {
+    int dev = -1;
+    return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+  }
+  bool done(int dev) const {
+    return dev >= 0 && dev < 64 && ((bits.load(std::memory_order_acquire) >> dev) & 1u) != 0;
+  }
+  void mark(int dev) {
+    if (dev >= 0 && dev < 64) bits.fetch_or(uint64_t(1) << dev, std::memory_order_acq_rel);
+  }
+};
 
 // w holds numel elements of in_dtype (NF4_F32, NF4_BF16 or NF4_F16).
 cudaError_t launch_quantize(const void* w, int in_dtype, int64_t numel, int bs, uint8_t* codes,

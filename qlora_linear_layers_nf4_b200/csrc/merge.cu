@@ -251,12 +251,13 @@ size_t merge_smem_bytes(int chunks) {
 
 cudaError_t launch_merge(const nf4_weight& w, const void* A, const void* B, int r, float alpha,
                          int out_f32, void* out, uint32_t* status, cudaStream_t st, int* launches) {
-  static bool attr_done = false;
-  if (!attr_done) {
+  static PerDeviceOnce attr_done;
+  const int dev = PerDeviceOnce::current();
+  if (!attr_done.done(dev)) {
     const cudaError_t e = cudaFuncSetAttribute(nf4_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                int(merge_smem_bytes(kMgMaxChunks)));
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    attr_done.mark(dev);
   }
   if (r < 1 || r > 64 * kMgMaxChunks) return cudaErrorInvalidValue;
   const size_t smem = merge_smem_bytes((r + 63) / 64);

@@ -1074,10 +1074,11 @@ int round_np(int r) { return int(cdiv(r, 64) * 64); }
 
 
 
-bool g_attr_done = false;
+PerDeviceOnce g_attr_done;
 
 cudaError_t set_attrs() {
-  if (g_attr_done) return cudaSuccess;
+  const int dev = PerDeviceOnce::current();
+  if (g_attr_done.done(dev)) return cudaSuccess;
   const void* single[4] = {(const void*)fused_nf4_gemm<kFwd, false>, (const void*)fused_nf4_gemm<kDx, false>,
                            (const void*)fused_nf4_gemm<kFwd, true>, (const void*)fused_nf4_gemm<kDx, true>};
   const void* pair[4] = {(const void*)fused_nf4_gemm_pair<kFwd, false>, (const void*)fused_nf4_gemm_pair<kDx, false>,
@@ -1090,7 +1091,7 @@ cudaError_t set_attrs() {
   const size_t ad_smem = kAdStages * (kAdABytes + 256 * 128) + 1024 + 256;
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(adapter_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, int(ad_smem));
-  if (e == cudaSuccess) g_attr_done = true;
+  if (e == cudaSuccess) g_attr_done.mark(dev);
   return e;
 }
 
