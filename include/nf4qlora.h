@@ -27,7 +27,8 @@
  *              nf4_read_status.
  *   Layouts    Row-major, densely packed.  W is [rows = N out, cols = K in].
  *              x is [M, K], A is [r, K], B is [N, r], y and dy are [M, N].
- *   Alignment  Device pointers must be 16-byte aligned (NF4_ERR_ALIGNMENT).
+ *   Alignment  Device pointers must be 16-byte aligned unless the entry
+ *              point states otherwise (NF4_ERR_ALIGNMENT).
  *   Errors     Arguments are validated on the host before anything is
  *              launched; a call that returns an error has enqueued nothing.
  *              Conditions only the GPU can see (non-finite input to quantize,

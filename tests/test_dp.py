@@ -129,3 +129,12 @@ def test_two_rank_sharded_double_quant():
     assert np.array_equal(codes, whole["codes"])
     assert np.array_equal(aq, whole["absmax_q"])
     assert all(np.float32(r[3]) == np.float32(whole["absmax_scale"]) for r in res)
+
+
+def test_sharded_quantize_refuses_a_shard_that_splits_a_block():
+    import torch
+    from qlora_linear_layers_nf4_b200.dp import quantize_sharded
+    with pytest.raises(ValueError):
+        quantize_sharded(torch.zeros(3, 40), 64, True, ops=_OracleOps)      # 120 elements: not whole blocks
+    q = quantize_sharded(torch.zeros(2, 64), 64, True, ops=_OracleOps)    # one rank, no process group
+    assert q.double_quant and float(q.absmax_scale.item()) == 0.0 and int(q.absmax_q.max()) == 0
