@@ -32,8 +32,13 @@ __device__ __forceinline__ bool finite8(const float4& a, const float4& b) {
 // per block (CUDA's correctly rounded reciprocal), q = RN(w y), then one
 // FMA-based correction q' = q + (w - a q) y.  That is Markstein's correction
 // step; with a correctly rounded reciprocal it yields the correctly rounded
-// quotient when nothing overflows or underflows, which the callers ensure by
-// keeping 2^-120 < a < 2^120 (other blocks take the division).
+// quotient when the remainder w - a q is representable.  Its lowest bit is
+// ulp(a) ulp(q) = 2^(ea + eq - 46), so it must satisfy ea + eq >= -103 not to
+// fall below the smallest subnormal.  Only quotients of magnitude >= 2^-5
+// can decide an NF4 code (every decision threshold is >= 0.0398 from zero)
+// and >= 2^-2 a double-quant code, so the step is taken for 2^-98 <= a <
+// 2^120 and other blocks take the division.  A host test runs the three
+// steps in C over that range against the IEEE quotient.
 //
 // The nearest level then comes from a 65-entry bucket table over [-1, 1]:
 // bucket i = floor(32 (v + 1)) holds base_i = #{thresholds below the bucket's
@@ -78,7 +83,7 @@ __device__ __forceinline__ float div_corrected(float w, float a, float y) {
 }
 
 __device__ __forceinline__ bool fast_scale(float a) {
-  return a > 0x1p-120f && a < 0x1p120f;
+  return a >= 0x1p-98f && a < 0x1p120f;
 }
 
 // Codes of two elements packed as one byte, even element in the high nibble.

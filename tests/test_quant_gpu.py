@@ -110,6 +110,28 @@ def test_edge_values(cuda_device):
         _check_dequant(q, ref, cuda_device)
 
 
+def test_small_block_scales_near_thresholds(cuda_device):
+    # Block scales a with arbitrary significands in the lowest binades, both
+    # sides of the 2^-98 edge where the kernel's division-free quotient stops
+    # being exact, and elements RN(t a) for every decision threshold t and its
+    # neighbours: quotients that sit on or next to a threshold, where one ulp
+    # decides the code.
+    rng = np.random.default_rng(31)
+    _, th = _q().codebook()
+    th = np.array(th, dtype=np.float32)
+    ts = np.concatenate([th, np.nextafter(th, np.float32(2)), np.nextafter(th, np.float32(-2))])
+    blocks = []
+    for e in list(range(-125, -90)) + [-60, -20, 0, 40, 100, 118, 119]:
+        for _ in range(40):
+            a = np.float32((1.0 + rng.random()) * 2.0 ** e)
+            vals = (np.resize(rng.permutation(ts), 63).astype(np.float64) * float(a)).astype(np.float32)
+            blocks.append(np.concatenate([vals, [a]]).astype(np.float32))
+    w = np.stack(blocks)
+    for dq in (False, True):
+        q, ref = _check_quant(w, 64, dq, cuda_device)
+        _check_dequant(q, ref, cuda_device)
+
+
 def test_absmax_element_exact(cuda_device):
     # values a for which multiplying by a reciprocal would not give exactly 1
     rng = np.random.default_rng(5)
