@@ -61,6 +61,9 @@ def _run(case, dev, zero_w=False, bias=False, rows=None):
 @pytest.mark.parametrize("m,n,k,rank,dq,bias", [
     (16, 256, 256, 8, False, False),       # decode path (mma.sync, f16 lookup table)
     (1, 512, 1024, 16, True, True),        # decode path, one token
+    (17, 4096, 4096, 16, True, False),     # decode path, widest instantiation (17..32 tokens)
+    (32, 1024, 2048, 16, False, True),     # decode path, 32 tokens, fp32 block scales
+    (24, 512, 512, 64, True, True),        # decode path, largest decode adapter
     (200, 512, 512, 32, True, True),       # single-CTA fused kernel
     (300, 264, 320, 16, True, True),       # pair kernel, ragged M and N
     (512, 512, 512, 64, True, False),      # pair kernel, full tiles

@@ -129,6 +129,23 @@ def test_decode_shapes(cuda_device, case):
     r.check_backward()
     r0 = Run(case, cuda_device, zero_w=True)
     r0.check_forward()
+    r0.check_backward()
+
+
+# Decode with 17..32 tokens takes the widest decode instantiation (four 8-token
+# MMA column groups); r = 8 and r = 64 are the smallest and largest adapter the
+# decode kernel takes in one K step of its adapter warps.
+@pytest.mark.parametrize("m,rank,dq", [
+    (17, 16, True), (24, 16, True), (32, 16, True), (32, 16, False),
+    (5, 8, True), (32, 8, True), (9, 64, True), (32, 64, False),
+])
+def test_decode_wide_and_rank_edges(cuda_device, m, rank, dq):
+    case = WL.LinearCase(f"decode 4096x4096 M={m} r={rank}", n=4096, k=4096, m=m, r=rank,
+                         alpha=2.0 * rank, seed=2, double_quant=dq)
+    for zero_w in (False, True):
+        r = Run(case, cuda_device, zero_w=zero_w, bias=not zero_w)
+        r.check_forward()
+        r.check_backward()
 
 
 def test_prefill_full_size_sampled(cuda_device):
@@ -150,7 +167,11 @@ def test_prefill_full_size_adapter_only(cuda_device):
 
 @pytest.mark.parametrize("case", WL.BLOCK, ids=lambda c: c.name.split()[1])
 def test_decoder_block_targets_sampled(cuda_device, case):
-    r = Run(case, cuda_device)
-    rows = np.random.default_rng(2).choice(r.xn.shape[0], 32, replace=False)
-    r.check_forward(rows)
-    r.check_backward(rows)
+    # With a zero base weight only the adapter path is left in y and dx, which
+    # the full-weight check alone cannot see (the adapter term is ~1.5 % of
+    # |y| and |dx|).
+    for zero_w in (False, True):
+        r = Run(case, cuda_device, zero_w=zero_w)
+        rows = np.random.default_rng(2).choice(r.xn.shape[0], 32, replace=False)
+        r.check_forward(rows)
+        r.check_backward(rows)

@@ -246,6 +246,44 @@ def test_bf16_round_matches_torch():
     assert np.array_equal(ours, theirs)
 
 
+def _weight_with_scales(scales):
+    # One block per scale, the 16 codes twice each: every level times every scale.
+    codes = np.tile(np.arange(16, dtype=np.uint8), 4)
+    q = {"codes": O.pack_codes(np.tile(codes, len(scales))),
+         "absmax": np.asarray(scales, dtype=np.float32), "shape": (len(scales), 64),
+         "block_size": 64}
+    return q
+
+
+def test_f16_dequant_matches_torch_half():
+    # The F16 dequant is the fp32 product rounded to binary16, nearest, ties to
+    # even.  Checked against torch's own fp32 -> f16 conversion on scales that
+    # put products on f16 halfway points (both tie directions), past the f16
+    # maximum (overflow to inf, and the 65520 tie that rounds to inf), into
+    # the subnormal range (including the tie at half the smallest subnormal,
+    # which rounds to zero) and on ordinary random scales.
+    import torch
+    lv = O.nf4_levels()
+    ties = [1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 2.0 ** -14 * (1 + 2.0 ** -11)]
+    big = [65504.0, 65519.0, 65520.0, 70000.0, 3.0e38]
+    tiny = [2.0 ** -25, 3 * 2.0 ** -25, 1e-6, 6.0e-8, 2.0 ** -24, 1e-30]
+    rand = list(np.random.default_rng(12).uniform(0.001, 2.0, 200))
+    # scales that make a level land exactly on an f16 tie: level * s = 1 + 2^-11 etc.
+    on_tie = [np.float32(t / float(lv[c])) for t in (1.0 + 2.0 ** -11, 2.0 ** -25) for c in (9, 12, 14)]
+    scales = np.array(ties + big + tiny + rand + on_tie, dtype=np.float32)
+    q = _weight_with_scales(scales)
+    w32 = O.dequantize(q, "f32")
+    with np.errstate(over="ignore"):       # overflow to inf is one of the cases
+        ours = O.dequantize(q, "f16")
+    theirs = torch.from_numpy(w32).half().numpy()
+    assert ours.dtype == np.float16
+    assert np.array_equal(ours.view(np.uint16), theirs.view(np.uint16))
+    # the classes really occur: infinities, subnormals, zeros from nonzero products, exact ties
+    assert np.any(np.isinf(ours)) and np.any((ours != 0) & (np.abs(ours) < np.float16(6.104e-5)))
+    assert np.any((ours == 0) & (w32 != 0))
+    assert ours[0, 15] == np.float16(1.0) and ours[1, 15] == np.float16(1.0 + 2.0 ** -9)
+
+
 def test_dequant_single_product_per_element():
     lv = O.nf4_levels()
     rng = np.random.default_rng(1)
@@ -273,6 +311,24 @@ def test_worked_linear_example():
     assert np.array_equal(d_b.ravel(), f("dB"))
     assert np.array_equal(d_a.ravel(), f("dA"))
     assert np.array_equal(d_x.ravel(), f("dx"))
+    # the same example with a bias on the output feature
+    yb, tb = O.qlora_forward(x, w, a, b, alpha, bias=f("bias"))
+    assert yb[0, 0] == float(g["y_bias"][0]) and tb[0, 0] == float(g["t"][0])
+
+
+def test_bias_adds_once_per_output_feature():
+    # Brute force with a bias: every row of y gains exactly the bias vector.
+    inp, w_hat, x, a, b, dy = _tiny()
+    bias = np.random.default_rng(5).standard_normal(w_hat.shape[0]) * 0.1
+    y0, _ = O.qlora_forward(x, w_hat, a, b, inp.case.alpha)
+    y1, _ = O.qlora_forward(x, w_hat, a, b, inp.case.alpha, bias=bias)
+    s = inp.case.alpha / inp.case.r
+    y_bf = (O.matmul_bruteforce(x, w_hat.T) + s * O.matmul_bruteforce(O.matmul_bruteforce(x, a.T), b.T)
+            + np.repeat(bias[None, :], x.shape[0], axis=0))
+    assert np.max(np.abs(y1 - y_bf)) <= 1e-12 * np.max(np.abs(y_bf))
+    # a bias of all zeros changes nothing, and adding one is a per-column shift
+    assert np.array_equal(O.qlora_forward(x, w_hat, a, b, inp.case.alpha, bias=np.zeros_like(bias))[0], y0)
+    assert np.allclose(y1 - y0, np.broadcast_to(bias, y0.shape), rtol=0, atol=1e-12)
 
 
 def _tiny():
