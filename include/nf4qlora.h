@@ -29,8 +29,12 @@
  *              x is [M, K], A is [r, K], B is [N, r], y and dy are [M, N].
  *   Alignment  Device pointers must be 16-byte aligned unless the entry
  *              point states otherwise (NF4_ERR_ALIGNMENT).
- *   Errors     Arguments are validated on the host before anything is
- *              launched; a call that returns an error has enqueued nothing.
+ *   Errors     Arguments are validated, and every launch of a call is
+ *              prepared (tensor maps encoded, grid sizes checked), on the
+ *              host before the first launch: a call that returns any error
+ *              other than NF4_ERR_CUDA has enqueued nothing.  NF4_ERR_CUDA
+ *              means the CUDA runtime refused a launch or copy; launches of
+ *              the same call that were enqueued before it may still run.
  *              Conditions only the GPU can see (non-finite input to quantize,
  *              an internal wait that exceeded its limit) are recorded in the
  *              status word at the head of `workspace` and returned by
@@ -206,11 +210,13 @@ NF4_API nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int 
  * and absmax == NULL the block scales are kept there, so rows*cols/block_size
  * may not exceed 1048576 (NF4_ERR_WORKSPACE otherwise); with a caller absmax
  * buffer there is no size limit.  Calls no allocator (no cudaMalloc or
- * cudaFree).  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) and should come before any stream capture.  All
- * calls share the array and it keeps the last call's contents (the global-max
- * word is cleared at the start of each call); calls whose GPU work overlaps
- * race.  Non-finite input is not reported (there is no status word to read).
+ * cudaFree).  Every call looks up the array's device address on the current
+ * device (cudaGetSymbolAddress); the first call on a device is the one that
+ * may load the library's device code there, so it should come before any
+ * stream capture.  All calls share the array and it keeps the last call's
+ * contents (the global-max word is cleared at the start of each call); calls
+ * whose GPU work overlaps race.  Launches are counted in nf4_launch_count.
+ * Non-finite input is not reported (there is no status word to read).
  */
 NF4_API nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t cols,
                                         int block_size, int double_quant, uint8_t* codes,
@@ -308,8 +314,10 @@ NF4_API nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out,
  *   bias           [N] compute_dtype, or NULL.
  *   y              [M, N] compute_dtype, written.
  *   t_out          [M, r] compute_dtype, or NULL: when given, receives
- *                  T = s (x A^T) rounded to compute_dtype, which
- *                  qlora_linear_bwd accepts as `t`.
+ *                  T = s (x A^T) -- the adapter activation already scaled
+ *                  by s and rounded to compute_dtype (2-byte elements for
+ *                  BF16 / F16, not an fp32 x A^T) -- which qlora_linear_bwd
+ *                  accepts as `t`.
  *   workspace      >= nf4_workspace_bytes(NF4_OP_LINEAR_FWD, M, N, K, r, 64, dq)
  *                  (the same size serves every compute dtype).
  * BF16 / F16: M <= 32 uses the weight-streaming decode path, larger M the

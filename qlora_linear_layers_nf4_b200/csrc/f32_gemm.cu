@@ -17,6 +17,8 @@
 // 256 threads with an 8 x 8 register tile each, the reduction in slices of 8
 // staged through double-buffered shared memory with the next slice's global
 // loads in flight while the current one is multiplied.
+#include <algorithm>
+
 #include <cuda_runtime.h>
 
 #include "kernels.h"
@@ -284,9 +286,19 @@ cudaError_t gemm_T(const LinearArgs& a, float* T, cudaStream_t st, int* launches
   return run_gemm(p, st, launches);
 }
 
+// Every product of the layer fits one launch's grid (checked before the first
+// launch, so a refused call enqueues nothing): the largest is M x max(N, K).
+bool grids_fit(const LinearArgs& a) {
+  const int64_t big = std::max(std::max(a.N, a.K), int64_t(a.r));
+  return ((a.M + kFT - 1) / kFT) * ((big + kFT - 1) / kFT) <= int64_t(0x7fffffff) &&
+         ((a.N + kFT - 1) / kFT) * ((a.r + kFT - 1) / kFT) <= int64_t(0x7fffffff) &&
+         ((a.K + kFT - 1) / kFT) * ((a.r + kFT - 1) / kFT) <= int64_t(0x7fffffff);
+}
+
 }  // namespace
 
 cudaError_t launch_linear_fwd_f32(const LinearArgs& a, cudaStream_t st, int* launches) {
+  if (!grids_fit(a)) return cudaErrorInvalidValue;
   float* T = a.t_out ? static_cast<float*>(a.t_out) : reinterpret_cast<float*>(a.ws + kWsHeader);
   cudaError_t e = gemm_T(a, T, st, launches);
   if (e != cudaSuccess) return e;
@@ -309,6 +321,7 @@ cudaError_t launch_linear_fwd_f32(const LinearArgs& a, cudaStream_t st, int* lau
 }
 
 cudaError_t launch_linear_bwd_f32(const LinearArgs& a, cudaStream_t st, int* launches) {
+  if (!grids_fit(a)) return cudaErrorInvalidValue;
   uint8_t* ws = a.ws + kWsHeader;
   const float* T = static_cast<const float*>(a.t_in);
   cudaError_t e = cudaSuccess;

@@ -29,6 +29,10 @@ struct PerDeviceOnce {
   }
 };
 
+// Adds to the library's launch counter (nf4_launch_count), for entry points
+// outside api.cu.
+void add_launches(int n);
+
 // w holds numel elements of in_dtype (NF4_F32, NF4_BF16 or NF4_F16).
 cudaError_t launch_quantize(const void* w, int in_dtype, int64_t numel, int bs, uint8_t* codes,
                             float* absmax_out, uint32_t* status, uint32_t* gmax, int sms,

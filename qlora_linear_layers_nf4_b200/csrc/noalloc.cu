@@ -12,13 +12,12 @@
 // The scratch array is a file-scope __device__ variable: every GPU that loads
 // the library holds it (kNoAllocScratchBytes) until the process exits.  Its
 // host-side name is only a stand-in for the symbol, never a device address;
-// the address is fetched once per device with cudaGetSymbolAddress and handed
-// to the kernels.  All calls on a device share the array and it keeps the
-// last call's contents, so the global-max word is cleared at the start of
-// every call; calls whose GPU work overlaps (different streams, no ordering)
-// race on it.
-#include <mutex>
-
+// every call looks the address up with cudaGetSymbolAddress on the current
+// device (cheap once the module is loaded, and never stale after the context
+// was reset) and hands it to the kernels.  All calls on a device share the
+// array and it keeps the last call's contents, so the global-max word is
+// cleared at the start of every call; calls whose GPU work overlaps
+// (different streams, no ordering) race on it.
 #include "kernels.h"
 #include "nf4_common.cuh"
 #include "nvtx_range.h"
@@ -33,25 +32,14 @@ constexpr size_t kNoAllocScratchBytes = kWsHeader + size_t(kNoAllocMaxBlocks) * 
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-uint8_t* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (set up on the
-// first call per device).
+// Device address of the scratch array on the current device.  Looked up on
+// every call: a cached pointer would dangle once the context it came from is
+// destroyed (cudaDeviceReset) and the module is loaded again.
 cudaError_t scratch_address(uint8_t** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev] = static_cast<uint8_t*>(p);
-  }
-  *out = g_noalloc_ptr[dev];
+  *out = static_cast<uint8_t*>(p);
   return cudaSuccess;
 }
 
@@ -113,5 +101,6 @@ extern "C" nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t
                         double_quant ? gmax : nullptr, sms, st, &launches);
   if (e == cudaSuccess && double_quant)
     e = launch_double_quant(amax, n_blocks, gmax, absmax_q, absmax_scale, sms, st, &launches);
+  add_launches(launches);
   return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
 }

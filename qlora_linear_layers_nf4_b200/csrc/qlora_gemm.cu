@@ -1109,17 +1109,24 @@ struct AdapterJob {
   float* out_f32;
 };
 
-cudaError_t run_adapter(const AdapterJob& j, uint32_t* status, int sms, cudaStream_t st,
-                        int* launches) {
-  const int NP = round_np(j.r);
+// A launch fully prepared on the host (tensor maps encoded, parameters set),
+// so that a call can build every launch before it enqueues the first one.
+struct AdapterLaunch {
   CUtensorMap ma, mb;
-  bool ok = j.a_mn ? make_map(&ma, j.a, true, j.a_inner, j.a_outer, 64, 64, true)
-                   : make_map(&ma, j.a, true, j.a_inner, j.a_outer, 64, 128, true);
-  ok = ok && (j.b_mn ? make_map(&mb, j.b, true, j.b_inner, j.b_outer, 64, 64, true)
-                     : make_map(&mb, j.b, true, j.b_inner, j.b_outer, 64, uint32_t(NP), true));
-  if (!ok) return cudaErrorInvalidValue;
-  const SplitPlan sp = plan_split(j.Mo, j.red);
   AdapterParams p;
+  dim3 grid;
+  size_t smem;
+};
+
+bool prepare_adapter(const AdapterJob& j, uint32_t* status, AdapterLaunch* L) {
+  const int NP = round_np(j.r);
+  bool ok = j.a_mn ? make_map(&L->ma, j.a, true, j.a_inner, j.a_outer, 64, 64, true)
+                   : make_map(&L->ma, j.a, true, j.a_inner, j.a_outer, 64, 128, true);
+  ok = ok && (j.b_mn ? make_map(&L->mb, j.b, true, j.b_inner, j.b_outer, 64, 64, true)
+                     : make_map(&L->mb, j.b, true, j.b_inner, j.b_outer, 64, uint32_t(NP), true));
+  if (!ok) return false;
+  const SplitPlan sp = plan_split(j.Mo, j.red);
+  AdapterParams& p = L->p;
   p.Mo = int(j.Mo);
   p.NP = NP;
   p.r = j.r;
@@ -1134,22 +1141,26 @@ cudaError_t run_adapter(const AdapterJob& j, uint32_t* status, int sms, cudaStre
   p.out_bf16 = j.out_bf16;
   p.out_f32 = j.out_f32;
   p.status = status;
-  (void)sms;
-  const size_t smem = kAdStages * (kAdABytes + size_t(NP) * 128) + 1024 + 256;
+  L->grid = dim3(unsigned(sp.tiles), unsigned(sp.slices), 1);
+  L->smem = kAdStages * (kAdABytes + size_t(NP) * 128) + 1024 + 256;
+  return true;
+}
+
+cudaError_t launch_adapter(const AdapterLaunch& L, cudaStream_t st, int* launches) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(sp.tiles), unsigned(sp.slices), 1);
+  cfg.gridDim = L.grid;
   cfg.blockDim = dim3(kAdThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = L.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = unsigned(sp.slices);
+  attr[0].val.clusterDim.y = L.grid.y;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   NF4_PROF_BEGIN(st, kKAdapterGemm);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, adapter_gemm, ma, mb, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, adapter_gemm, L.ma, L.mb, L.p);
   NF4_PROF_END(st, kKAdapterGemm);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
@@ -1187,13 +1198,86 @@ FusedParams fused_params(const LinearArgs& a, int mode) {
 // same workspace serves every compute dtype (the F32 path keeps them in fp32).
 size_t mr_bytes(int64_t M, int r) { return align256(size_t(M) * size_t(r) * 4); }
 
-cudaError_t forward_adapter_T(const LinearArgs& a, __nv_bfloat16* T, int sms, cudaStream_t st,
-                              int* launches) {
+AdapterJob job_T(const LinearArgs& a, __nv_bfloat16* T) {
   AdapterJob j{};
   j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = false;
   j.b = a.A; j.b_inner = a.K; j.b_outer = a.r; j.b_mn = false;
   j.Mo = a.M; j.red = a.K; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = T; j.f16 = a.f16;
-  return run_adapter(j, a.status, sms, st, launches);
+  return j;
+}
+
+// One fused dequant + tensor-core GEMM launch, prepared on the host.
+struct FusedLaunch {
+  CUtensorMap ta, ta2, tb2, tc, to;
+  FusedParams p;
+  bool pair;
+  int mode;
+  bool f16;
+  dim3 grid;
+};
+
+// Forward: A = x, A2 = T, B2 = B_lora, out = y.  dx: A = dy, A2 = U, B2 = A_lora, out = dx.
+bool prepare_fused(const LinearArgs& a, int mode, const __nv_bfloat16* a2, FusedLaunch* L) {
+  L->pair = use_pair(a.M);
+  L->mode = mode;
+  L->f16 = a.f16 != 0;
+  const bool pair = L->pair;
+  const uint32_t arows = pair ? uint32_t(kP2ARows) : 256u;   // A rows per TMA box
+  const int64_t m_tiles = cdiv(a.M, pair ? kP2TileM : kTileM);
+  if (m_tiles > 65535) return false;                         // grid.y
+  bool ok;
+  if (mode == kFwd) {
+    const uint32_t brows = pair ? 128 : 256;     // W' rows per CTA
+    ok = make_map(&L->ta, a.x, true, a.K, a.M, 64, arows, true);
+    ok = ok && make_map(&L->ta2, a2, true, a.r, a.M, 64, arows, true);
+    ok = ok && make_map(&L->tb2, a.B, true, a.r, a.N, 64, brows, true);
+    ok = ok && (pair ? make_map(&L->tc, a.w->codes, false, a.K / 2, a.N, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)
+                     : make_map(&L->tc, a.w->codes, false, a.K / 2, a.N, 32, brows, false));
+    // y [M, N]: 32 x 32 boxes in the epilogues' staging layout
+    ok = ok && make_map_2d_bf16(&L->to, a.y, uint64_t(a.N), uint64_t(a.M), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    L->grid = pair ? dim3(unsigned(2 * cdiv(a.N, kTileN)), unsigned(m_tiles))
+                   : dim3(unsigned(cdiv(a.N, kTileN)), unsigned(m_tiles));
+  } else {
+    ok = make_map(&L->ta, a.dy, true, a.N, a.M, 64, arows, true);
+    ok = ok && make_map(&L->ta2, a2, true, a.r, a.M, 64, arows, true);
+    ok = ok && make_map(&L->tb2, a.A, true, a.K, a.r, 64, 64, true);
+    ok = ok && (pair ? make_map(&L->tc, a.w->codes, false, a.K / 2, a.N, 64, 256, CU_TENSOR_MAP_SWIZZLE_64B)
+                     : make_map(&L->tc, a.w->codes, false, a.K / 2, a.N, 32, 64, false));
+    // dx [M, K]: 32 x 32 boxes in the epilogues' staging layout
+    ok = ok && make_map_2d_bf16(&L->to, a.dx, uint64_t(a.K), uint64_t(a.M), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    L->grid = pair ? dim3(unsigned(2 * cdiv(a.K, kTileN)), unsigned(m_tiles))
+                   : dim3(unsigned(cdiv(a.K, kTileN)), unsigned(m_tiles));
+  }
+  if (!ok) return false;
+  L->p = fused_params(a, mode);
+  return true;
+}
+
+cudaError_t launch_fused(const FusedLaunch& L, cudaStream_t st, int* launches) {
+  const dim3 grid = L.grid;
+  const int id = L.mode == kFwd ? kKFusedFwd : kKFusedDx;
+  NF4_PROF_BEGIN(st, id);
+  if (L.pair) {
+    if (L.mode == kFwd) {
+      if (L.f16) fused_nf4_gemm_pair<kFwd, true><<<grid, kP2Threads, kP2Smem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
+      else fused_nf4_gemm_pair<kFwd, false><<<grid, kP2Threads, kP2Smem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
+    } else {
+      if (L.f16) fused_nf4_gemm_pair<kDx, true><<<grid, kP2Threads, kP2Smem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
+      else fused_nf4_gemm_pair<kDx, false><<<grid, kP2Threads, kP2Smem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
+    }
+  } else {
+    if (L.mode == kFwd) {
+      if (L.f16) fused_nf4_gemm<kFwd, true><<<grid, kFusedThreads, kFusedSmem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
+      else fused_nf4_gemm<kFwd, false><<<grid, kFusedThreads, kFusedSmem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
+    } else {
+      if (L.f16) fused_nf4_gemm<kDx, true><<<grid, kFusedThreads, kFusedSmem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
+      else fused_nf4_gemm<kDx, false><<<grid, kFusedThreads, kFusedSmem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
+    }
+  }
+  NF4_PROF_END(st, id);
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 }  // namespace
@@ -1227,7 +1311,10 @@ size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, in
   return (backward ? 2 : 1) * mr_bytes(M, r);
 }
 
+// Every launch of a call is prepared (its tensor maps encoded) before the
+// first is enqueued, so a call that fails on the host enqueues nothing.
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches) {
+  (void)sms;
   if (decode_supported(a.M, a.N, a.K, a.r)) {
     const cudaError_t d = launch_decode_fwd(a, sms, st, launches);
     if (d != cudaErrorNotSupported) return d;
@@ -1236,106 +1323,61 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   if (e != cudaSuccess) return e;
   uint8_t* ws = a.ws + kWsHeader;
   __nv_bfloat16* T = a.t_out ? static_cast<__nv_bfloat16*>(a.t_out) : reinterpret_cast<__nv_bfloat16*>(ws);
-
-  e = forward_adapter_T(a, T, sms, st, launches);
+  AdapterLaunch lt;
+  FusedLaunch lf;
+  if (!prepare_adapter(job_T(a, T), a.status, &lt) || !prepare_fused(a, kFwd, T, &lf))
+    return cudaErrorInvalidValue;
+  e = launch_adapter(lt, st, launches);
   if (e != cudaSuccess) return e;
-
-  const bool pair = use_pair(a.M);
-  const uint32_t brows = pair ? 128 : 256;     // W' rows per CTA
-  CUtensorMap ta, ta2, tb2, tc;
-  const uint32_t arows = pair ? uint32_t(kP2ARows) : 256u;   // A rows per TMA box
-  bool ok = make_map(&ta, a.x, true, a.K, a.M, 64, arows, true);
-  ok = ok && make_map(&ta2, T, true, a.r, a.M, 64, arows, true);
-  ok = ok && make_map(&tb2, a.B, true, a.r, a.N, 64, brows, true);
-  ok = ok && (pair ? make_map(&tc, a.w->codes, false, a.K / 2, a.N, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)
-                   : make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, brows, false));
-  CUtensorMap to;   // y [M, N]: 32 x 32 boxes in the epilogues' staging layout
-  ok = ok && make_map_2d_bf16(&to, a.y, uint64_t(a.N), uint64_t(a.M), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (!ok) return cudaErrorInvalidValue;
-  const FusedParams p = fused_params(a, kFwd);
-  NF4_PROF_BEGIN(st, kKFusedFwd);
-  if (pair) {
-    dim3 grid(unsigned(2 * cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kP2TileM)));
-    if (a.f16) fused_nf4_gemm_pair<kFwd, true><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, to, p);
-    else fused_nf4_gemm_pair<kFwd, false><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, to, p);
-  } else {
-    dim3 grid(unsigned(cdiv(a.N, kTileN)), unsigned(cdiv(a.M, kTileM)));
-    if (a.f16) fused_nf4_gemm<kFwd, true><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, to, p);
-    else fused_nf4_gemm<kFwd, false><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, to, p);
-  }
-  NF4_PROF_END(st, kKFusedFwd);
-  e = cudaGetLastError();
-  if (e == cudaSuccess) ++*launches;
-  return e;
+  return launch_fused(lf, st, launches);
 }
 
 cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches) {
+  (void)sms;
   cudaError_t e = set_attrs();
   if (e != cudaSuccess) return e;
   uint8_t* ws = a.ws + kWsHeader;
   __nv_bfloat16* T_ws = reinterpret_cast<__nv_bfloat16*>(ws);
   __nv_bfloat16* U = reinterpret_cast<__nv_bfloat16*>(ws + mr_bytes(a.M, a.r));
+  const bool recompute_t = a.t_in == nullptr;
+  const __nv_bfloat16* T = recompute_t ? T_ws : static_cast<const __nv_bfloat16*>(a.t_in);
 
-  const __nv_bfloat16* T = static_cast<const __nv_bfloat16*>(a.t_in);
-  if (T == nullptr) {
-    e = forward_adapter_T(a, T_ws, sms, st, launches);
-    if (e != cudaSuccess) return e;
-    T = T_ws;
-  }
-  // U = s dy B   (A: dy K-major over n; B: B_lora [N, r] MN-major over n)
-  {
+  AdapterLaunch lt, lu, ldb, lda;
+  FusedLaunch ldx;
+  bool ok = !recompute_t || prepare_adapter(job_T(a, T_ws), a.status, &lt);
+  {  // U = s dy B   (A: dy K-major over n; B: B_lora [N, r] MN-major over n)
     AdapterJob j{};
     j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = false;
     j.b = a.B; j.b_inner = a.r; j.b_outer = a.N; j.b_mn = true;
     j.Mo = a.M; j.red = a.N; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = U; j.f16 = a.f16;
-    e = run_adapter(j, a.status, sms, st, launches);
-    if (e != cudaSuccess) return e;
+    ok = ok && prepare_adapter(j, a.status, &lu);
   }
-  // dB = dy^T T   (A: dy^T MN-major over m; B: T [M, r] MN-major over m)
-  {
+  {  // dB = dy^T T   (A: dy^T MN-major over m; B: T [M, r] MN-major over m)
     AdapterJob j{};
     j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = true;
     j.b = T; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
     j.Mo = a.N; j.red = a.M; j.r = a.r; j.kind = 1; j.scale = 1.0f; j.out_f32 = a.dB; j.f16 = a.f16;
-    e = run_adapter(j, a.status, sms, st, launches);
-    if (e != cudaSuccess) return e;
+    ok = ok && prepare_adapter(j, a.status, &ldb);
   }
-  // dA^T = x^T U  (A: x^T MN-major over m; B: U [M, r] MN-major over m), stored as dA [r, K]
-  {
+  {  // dA^T = x^T U  (A: x^T MN-major over m; B: U [M, r] MN-major over m), stored as dA [r, K]
     AdapterJob j{};
     j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = true;
     j.b = U; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
     j.Mo = a.K; j.red = a.M; j.r = a.r; j.kind = 2; j.scale = 1.0f; j.out_f32 = a.dA; j.f16 = a.f16;
-    e = run_adapter(j, a.status, sms, st, launches);
+    ok = ok && prepare_adapter(j, a.status, &lda);
+  }
+  // dx = dy W' + U A
+  ok = ok && (a.dx == nullptr || prepare_fused(a, kDx, U, &ldx));
+  if (!ok) return cudaErrorInvalidValue;
+
+  if (recompute_t) {
+    e = launch_adapter(lt, st, launches);
     if (e != cudaSuccess) return e;
   }
-  if (a.dx == nullptr) return cudaSuccess;
-  // dx = dy W' + U A
-  CUtensorMap ta, ta2, tb2, tc;
-  const bool pair = use_pair(a.M);
-  const uint32_t arows = pair ? uint32_t(kP2ARows) : 256u;   // A rows per TMA box
-  bool ok = make_map(&ta, a.dy, true, a.N, a.M, 64, arows, true);
-  ok = ok && make_map(&ta2, U, true, a.r, a.M, 64, arows, true);
-  ok = ok && make_map(&tb2, a.A, true, a.K, a.r, 64, 64, true);
-  ok = ok && (pair ? make_map(&tc, a.w->codes, false, a.K / 2, a.N, 64, 256, CU_TENSOR_MAP_SWIZZLE_64B)
-                   : make_map(&tc, a.w->codes, false, a.K / 2, a.N, 32, 64, false));
-  CUtensorMap to;   // dx [M, K]: 32 x 32 boxes in the epilogues' staging layout
-  ok = ok && make_map_2d_bf16(&to, a.dx, uint64_t(a.K), uint64_t(a.M), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (!ok) return cudaErrorInvalidValue;
-  const FusedParams p = fused_params(a, kDx);
-  NF4_PROF_BEGIN(st, kKFusedDx);
-  if (pair) {
-    dim3 grid(unsigned(2 * cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kP2TileM)));
-    if (a.f16) fused_nf4_gemm_pair<kDx, true><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, to, p);
-    else fused_nf4_gemm_pair<kDx, false><<<grid, kP2Threads, kP2Smem, st>>>(ta, ta2, tb2, tc, to, p);
-  } else {
-    dim3 grid(unsigned(cdiv(a.K, kTileN)), unsigned(cdiv(a.M, kTileM)));
-    if (a.f16) fused_nf4_gemm<kDx, true><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, to, p);
-    else fused_nf4_gemm<kDx, false><<<grid, kFusedThreads, kFusedSmem, st>>>(ta, ta2, tb2, tc, to, p);
-  }
-  NF4_PROF_END(st, kKFusedDx);
-  e = cudaGetLastError();
-  if (e == cudaSuccess) ++*launches;
+  e = launch_adapter(lu, st, launches);
+  if (e == cudaSuccess) e = launch_adapter(ldb, st, launches);
+  if (e == cudaSuccess) e = launch_adapter(lda, st, launches);
+  if (e == cudaSuccess && a.dx != nullptr) e = launch_fused(ldx, st, launches);
   return e;
 }
 

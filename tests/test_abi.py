@@ -151,6 +151,23 @@ def test_merge_host_validation():
     assert m(_cw(), wsb=0) == 5
 
 
+def test_noalloc_host_validation():
+    # nf4_quantize_noalloc checks its sizes against its fixed scratch array on
+    # the host, before it looks the array up or launches anything.
+    L = Q.lib()
+    rows, cols = 16384, 4160          # 1,064,960 blocks of 64 > 1,048,576
+    assert L.nf4_quantize_noalloc(FAKE, rows, cols, 64, 1, FAKE, None, FAKE, FAKE, None) == 5
+    # with a caller absmax buffer the array holds no block scales: no size limit,
+    # so the same size reaches the alignment check of `codes`
+    assert L.nf4_quantize_noalloc(FAKE, rows, cols, 64, 1, FAKE + 8, FAKE, FAKE, FAKE, None) == 3
+    assert L.nf4_quantize_noalloc(FAKE, 4, 64, 63, 0, FAKE, FAKE, None, None, None) == 2
+    assert L.nf4_quantize_noalloc(FAKE, 4, 64, 64, 2, FAKE, FAKE, None, None, None) == 1
+    assert L.nf4_quantize_noalloc(None, 4, 64, 64, 0, FAKE, FAKE, None, None, None) == 1
+    assert L.nf4_quantize_noalloc(FAKE, 4, 64, 64, 0, FAKE, None, None, None, None) == 1
+    assert L.nf4_quantize_noalloc(FAKE, 4, 64, 64, 1, FAKE, None, None, FAKE, None) == 1
+    assert L.nf4_quantize_noalloc(FAKE + 4, 4, 64, 64, 0, FAKE, FAKE, None, None, None) == 3
+
+
 def test_wait_check_host_validation():
     L = Q.lib()
     rel = ctypes.c_uint32(0)
