@@ -56,6 +56,72 @@ def test_two_rank_gradient_allreduce():
     assert all(m == 10.0 * world for _, _, m in res)
 
 
+def _grad_worker(rank, world, port, q, split):
+    """Each rank takes its token shard of the tiny layer, computes the adapter
+    gradients of its shard (the CPU oracle stands in for the GPU call), and
+    sums them with the other ranks through AdapterGradBuffer."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from oracle import nf4_oracle as O
+    from qlora_linear_layers_nf4_b200 import workloads as WL
+    from qlora_linear_layers_nf4_b200.dp import AdapterGradBuffer
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        case = WL.TINY
+        inp = WL.draw_linear(case)
+        w_hat = O.bf16_to_f32(O.dequantize(O.quantize(inp.w, 64), "bf16"))
+        f = WL.bf16_bits_to_f32
+        x, a, b, dy = (f(v).astype(np.float64) for v in (inp.x, inp.a, inp.b, inp.dy))
+        lo, hi = split[rank], split[rank + 1]
+        d_a, d_b, _ = O.qlora_backward(x[lo:hi], w_hat, a, b, case.alpha, dy[lo:hi])
+        g = AdapterGradBuffer(case.r, case.k, case.n, "cpu", dtype=torch.float64)
+        g.dA.copy_(torch.from_numpy(d_a))
+        g.dB.copy_(torch.from_numpy(d_b))
+        g.all_reduce()
+        q.put((rank, g.dA.numpy().copy(), g.dB.numpy().copy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("split", [(0, 8, 16), (0, 3, 16)])
+def test_token_sharded_gradients_sum_to_the_full_batch(split):
+    # Data parallelism over tokens is exact: dA = s sum_m u_m^T x_m and
+    # dB = s sum_m dy_m^T t_m are sums over tokens, so the per-rank sums,
+    # added by the all-reduce, equal the full-batch gradients (up to fp64
+    # rounding of the summation order).  An uneven split gives the same.
+    import numpy as np
+    import torch.multiprocessing as mp
+    from oracle import nf4_oracle as O
+    from qlora_linear_layers_nf4_b200 import workloads as WL
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 2
+    procs = [ctx.Process(target=_grad_worker, args=(i, world, port, q, split)) for i in range(world)]
+    for p in procs:
+        p.start()
+    # read the results before joining: a child cannot exit while its queued
+    # arrays are still waiting in the pipe
+    res = sorted((q.get(timeout=120) for _ in range(world)), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    case = WL.TINY
+    inp = WL.draw_linear(case)
+    w_hat = O.bf16_to_f32(O.dequantize(O.quantize(inp.w, 64), "bf16"))
+    f = WL.bf16_bits_to_f32
+    x, a, b, dy = (f(v).astype(np.float64) for v in (inp.x, inp.a, inp.b, inp.dy))
+    d_a, d_b, _ = O.qlora_backward(x, w_hat, a, b, case.alpha, dy)
+    for _, got_a, got_b in res:
+        assert np.max(np.abs(got_a - d_a)) <= 1e-12 * np.max(np.abs(d_a))
+        assert np.max(np.abs(got_b - d_b)) <= 1e-12 * np.max(np.abs(d_b))
+    # both ranks hold the same sum
+    assert np.array_equal(res[0][1], res[1][1]) and np.array_equal(res[0][2], res[1][2])
+
+
 class _OracleOps:
     """The three steps of a sharded quantization, by the CPU oracle (test
     stand-ins for the CUDA calls; the exchange between them is real)."""
