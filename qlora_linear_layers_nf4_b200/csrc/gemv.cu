@@ -5,20 +5,29 @@
 //
 // (qlora-rs README, QuantizedLinear::forward; "LoRA and QLoRA,
 // mathematically", equation 6.3.6 read as a layer.)  With a handful of tokens
-// the weight bytes are the whole cost, so the design is about getting every
-// byte in flight at once and spending few instructions per element:
-//   - a CTA owns 128 W rows and one K slice; all of its code tiles are
-//     requested by TMA before anything else happens;
+// the weight bytes are the whole cost, so the design is about keeping every
+// byte in flight and the SM busy while they land:
+//   - a CTA owns 128 W rows and one K slice.  Its block scales are requested
+//     first (plain loads, so they are not queued behind the weight bytes),
+//     then every code tile, x tile and A tile of the slice by TMA, one
+//     mbarrier per 64-wide K block, so compute starts on the first block to
+//     land;
 //   - a 4-bit pair becomes two bf16 levels with one shared-memory lookup in a
 //     256-entry table replicated per lane (conflict-free); the block scale is
 //     applied to each 64-wide block's fp32 partial, not to every element;
 //   - the dequantized values never leave registers: they are the A fragments
 //     of mma.sync m16n8k16 with x as B (the K order inside each block is
 //     permuted identically for both so a thread's fragments are contiguous
-//     bytes); x A^T rides along as extra rows from the same x fragments;
-//   - the S K-slices of a row tile are one thread-block cluster; partials are
-//     summed through distributed shared memory in slice order, and the adapter
-//     term, bias and bf16 rounding are applied in that reduction.
+//     bytes).  A warp takes one K block at a time for two 16-row groups, so
+//     each x fragment it loads serves both;
+//   - x A^T (the slice's share of the adapter activation) is computed by four
+//     more warps from the same x tiles; its product with the tile's B rows is
+//     one more short MMA chain on the W-row accumulators;
+//   - the S K-slices of a row tile are one thread-block cluster.  CTA q owns
+//     rows [q 128/S, (q+1) 128/S) of the tile: every CTA pushes its partial
+//     for those rows into CTA q's shared memory and arrives on CTA q's
+//     mbarrier; CTA q sums the S partials in slice order (deterministic), adds
+//     the bias and rounds once.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -32,19 +41,25 @@ namespace {
 
 using namespace tc;
 
-constexpr int kGvWWarps = 16;                       // 2 per 16-row group (alternate K blocks)
+constexpr int kGvWWarps = 16;                       // W-row warps
 constexpr int kGvAWarps = 4;                        // up to 64 adapter rows of x A^T
-constexpr int kGvThreads = (kGvWWarps + kGvAWarps) * 32;
+constexpr int kGvWarps = kGvWWarps + kGvAWarps;
+constexpr int kGvThreads = kGvWarps * 32;
 constexpr int kGvRows = 128;                        // W rows per CTA
 constexpr int kGvMaxBlocks = 16;                    // 64-wide K blocks per CTA
-static_assert(kGvWWarps + kGvAWarps > kGvMaxBlocks, "one issuing warp per K block plus one for B");
+constexpr int kGvGroup = 4;                         // K blocks per TMA box: 128 code bytes a row
+constexpr int kGvMaxGroups = kGvMaxBlocks / kGvGroup;
+static_assert(3 * kGvMaxGroups + 1 <= kGvWarps, "one issuing warp per box");
 constexpr int kGvMaxR = 16 * kGvAWarps;
-constexpr int kGvLutBytes = 0;                      // the table is a static array
+constexpr int kGvMaxSlices = 8;
+// 227 KB per CTA at most, less the 32 KB static lookup table (and a little).
+constexpr size_t kGvMaxDynSmem = 194u * 1024u;
 
 struct GemvParams {
   int M, N, K, r;
   int kb_per_row;       // K / 64
   int blocks_per_slice;
+  int vec_scales;       // 16-byte aligned scale rows: vector loads
   int slices;
   int r_pad;            // r rounded up to 16 (rows of the A tiles)
   float s;              // alpha / r
@@ -52,38 +67,51 @@ struct GemvParams {
   const uint8_t* absmax_q;
   const float* absmax;
   const float* absmax_scale;
-  const __nv_bfloat16* B;
   const __nv_bfloat16* bias;
   __nv_bfloat16* y;
   __nv_bfloat16* t_out;
   uint32_t* status;
 };
 
-// Shared memory (after 1024-byte alignment), every region 1024-byte aligned:
-//   lut    256 entries x 32 lanes x 4 B                  32 KB
-//   codes  [block][128 W rows][32 B]                      4 KB per block
-//   xs     [block][NP token rows][128 B], 128-byte swizzle
-//   as     [block][r_pad adapter rows][128 B], 128-byte swizzle
+// Shared memory (after 1024-byte alignment), every region 1024-byte aligned;
+// G = ceil(blocks per slice / 4) TMA groups of four K blocks:
+//   codes  [G][128 W rows][128 B], 128-byte swizzle (the codes of 4 blocks)
+//   xs     [4 G blocks][NP token rows][128 B], 128-byte swizzle
+//   as     [4 G blocks][r_pad adapter rows][128 B], 128-byte swizzle
 //   bs     [128 W rows][r] bf16 (this tile's rows of B)
 //   scales [128 rows][kGvMaxBlocks] fp32                 8 KB
-//   part   [128][NP] fp32, tpart [64][NP] fp32, barriers
+//   recv   [slice][128 / S rows][NP] fp32: partials pushed by the cluster
+//   tpart  [r_pad][NP] fp32: this slice's x A^T
+//   red    [block phase - 1][128][NP] fp32: in-CTA partials (over codes and
+//          xs once they are consumed, when they are large enough)
+//   bars   [G] TMA groups, B tile, recv
 struct GemvLayout {
-  size_t codes, xs, as, bs, scales, part, tpart, bar, total;
+  size_t codes, xs, as, bs, scales, recv, tpart, red, bar, total;
 };
 
 __host__ __device__ constexpr size_t align1k(size_t v) { return (v + 1023) & ~size_t(1023); }
 
-__host__ __device__ inline GemvLayout gemv_layout(int bps, int np, int r_pad, int r) {
+__host__ __device__ inline GemvLayout gemv_layout(int bps, int np, int r_pad, int r, int phases) {
+  const int groups = (bps + kGvGroup - 1) / kGvGroup;
+  const int blocks = groups * kGvGroup;
   GemvLayout L{};
-  L.codes = kGvLutBytes;
-  L.xs = align1k(L.codes + size_t(bps) * 4096);
-  L.as = align1k(L.xs + size_t(bps) * np * 128);
-  L.bs = align1k(L.as + size_t(bps) * r_pad * 128);
+  L.codes = 0;
+  L.xs = align1k(L.codes + size_t(groups) * kGvRows * 128);
+  L.as = align1k(L.xs + size_t(blocks) * np * 128);
+  L.bs = align1k(L.as + size_t(blocks) * r_pad * 128);
   L.scales = align1k(L.bs + size_t(kGvRows) * r * 2);
-  L.part = L.scales + size_t(kGvRows) * kGvMaxBlocks * 4;
-  L.tpart = L.part + size_t(kGvRows) * np * 4;
-  L.bar = L.tpart + size_t(kGvMaxR) * np * 4;
-  L.total = 1024 + L.bar + 8 * (kGvMaxBlocks + 1);
+  L.recv = align1k(L.scales + size_t(kGvRows) * kGvMaxBlocks * 4);
+  L.tpart = L.recv + size_t(kGvRows) * np * 4;
+  size_t end = align1k(L.tpart + size_t(r_pad) * np * 4);
+  const size_t red_bytes = size_t(phases - 1) * kGvRows * np * 4;
+  if (red_bytes <= L.as - L.codes) {
+    L.red = L.codes;
+  } else {
+    L.red = end;
+    end = align1k(end + red_bytes);
+  }
+  L.bar = end;
+  L.total = 1024 + L.bar + 8 * (kGvMaxGroups + 2);
   return L;
 }
 
@@ -119,11 +147,14 @@ __device__ __forceinline__ __nv_bfloat16 from_f32(float v) {
   }
   return __float2bfloat16_rn(v);
 }
-
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
-  return v;
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2_rn(float lo, float hi) {
+  if (F16) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Byte offset of lane `lane`'s copy of table entry `byte j of word`, for a
@@ -141,6 +172,13 @@ __device__ __forceinline__ void load_row16(const uint8_t* tile, int row, int q, 
   hi = *reinterpret_cast<const uint4*>(tile + sw128_offset(uint32_t(row), uint32_t(2 * q + 1)));
 }
 
+// The 8 code bytes of K block j (0..3 of its group) that lane quarter q owns,
+// in row `row` of a group's [128 rows][128 B] 128-byte-swizzled code box.
+__device__ __forceinline__ uint2 load_codes8(const uint8_t* box, uint32_t row, uint32_t j, uint32_t q) {
+  const uint32_t chunk = 2u * j + (q >> 1);
+  return *reinterpret_cast<const uint2*>(box + row * 128u + ((chunk ^ (row & 7u)) << 4) + ((q & 1u) << 3));
+}
+
 // Fragments of MMA i (0..3) from 16 consecutive values: elements (4i, 4i+1)
 // and (4i+2, 4i+3).
 __device__ __forceinline__ void frag_pair(const uint4& lo, const uint4& hi, int i, uint32_t& f0,
@@ -155,24 +193,36 @@ __device__ __forceinline__ void frag_pair(const uint4& lo, const uint4& hi, int 
   }
 }
 
-template <int NT8, bool F16>
+// NT8: token columns in groups of 8 (M <= 8 NT8).  RG: 16-row groups per W
+// warp (each x fragment a warp loads serves RG groups).
+//
+// Row mapping: MMA row g (0..7) of a 16-row group is W row 2g of the group and
+// MMA row g + 8 is W row 2g + 1.  In a half-warp the four rows a code load
+// touches then differ in bits 1..2 of the row, which the 128-byte swizzle
+// turns into four different 32-byte bank groups: the loads are conflict-free.
+template <int NT8, int RG, bool F16>
 __global__ void __launch_bounds__(kGvThreads, 1)
     nf4_gemv(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
              const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
              const GemvParams p) {
   constexpr int NP = 8 * NT8;                  // token rows (M padded)
+  constexpr int kSets = 8 / RG;                // row-group sets = W warps per block phase
+  constexpr int kPhases = kGvWWarps / kSets;   // W warps that share one row-group set
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(1024) uint32_t lut[256 * 32];      // [entry][lane] copies
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const GemvLayout L = gemv_layout(p.blocks_per_slice, NP, p.r_pad, p.r);
+  const GemvLayout L = gemv_layout(p.blocks_per_slice, NP, p.r_pad, p.r, kPhases);
   uint8_t* codes = smem + L.codes;
   uint8_t* xs = smem + L.xs;
   uint8_t* as = smem + L.as;
   const __nv_bfloat16* bs = reinterpret_cast<const __nv_bfloat16*>(smem + L.bs);
   float* scales = reinterpret_cast<float*>(smem + L.scales);
-  float* part = reinterpret_cast<float*>(smem + L.part);
+  float* recv = reinterpret_cast<float*>(smem + L.recv);
   float* tpart = reinterpret_cast<float*>(smem + L.tpart);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);   // [block], then B rows
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);   // [group], B rows, recv
+  uint64_t* bar_b = &bar[kGvMaxGroups];
+  uint64_t* bar_recv = &bar[kGvMaxGroups + 1];
   __shared__ uint32_t abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -181,126 +231,192 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   const int q = lane & 3;
   const int n0 = blockIdx.x * kGvRows;
   const int slice = blockIdx.y;                // = rank in the (1, S, 1) cluster
+  const int S = p.slices;
   const int kb0 = slice * p.blocks_per_slice;
   const int nblk = max(0, min(p.blocks_per_slice, p.kb_per_row - kb0));
+  const int groups = (nblk + kGvGroup - 1) / kGvGroup;
   const uint32_t xbytes = uint32_t(NP) * 128u;
   const uint32_t abytes = uint32_t(p.r_pad) * 128u;
+  const int band = kGvRows / S;                // rows of the tile this CTA finishes
+  const bool pull_t = p.t_out != nullptr && blockIdx.x == 0;   // uniform over the cluster
 
-  // Every byte this CTA reads is requested before anything else, one barrier
-  // per 64-wide K block so compute starts on the first block to land.  Warp b
-  // issues block b's copies (and warp kGvMaxBlocks the B tile): one warp keeps
-  // only a few TMA copies going per microsecond, so the issue is spread.
-  if (threadIdx.x == 0) abort_flag = 0;
-  if (lane == 0 && warp <= kGvMaxBlocks) {
-    mbar_init(&bar[warp], 1);
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int c = 0; c < kGvMaxGroups; ++c) mbar_init(&bar[c], 3);   // codes, x and A issuers
+    mbar_init(bar_b, 1);
+    mbar_init(bar_recv, 1);
     fence_barrier_init();
+    // every slice pushes its partial of this CTA's band: S x band x NP fp32
+    mbar_arrive_expect_tx(bar_recv, uint32_t(kGvRows) * NP * 4u);
     fence_proxy_async_smem();
-    if (warp == kGvMaxBlocks) {
-      mbar_arrive_expect_tx(&bar[kGvMaxBlocks], uint32_t(kGvRows) * uint32_t(p.r) * 2u);
-      tma_load_2d(smem + L.bs, &tm_b, &bar[kGvMaxBlocks], 0, n0);
-    } else if (warp < nblk) {
-      const int b = warp, kb = kb0 + b;
-      mbar_arrive_expect_tx(&bar[b], 4096u + xbytes + abytes);
-      tma_load_2d(codes + b * 4096, &tm_codes, &bar[b], kb * 32, n0);
-      tma_load_2d(xs + b * xbytes, &tm_x, &bar[b], kb * 64, 0);
-      tma_load_2d(as + b * abytes, &tm_a, &bar[b], kb * 64, 0);
+  } else if (threadIdx.x == 32) {
+    tma_prefetch(&tm_codes);
+    tma_prefetch(&tm_x);
+    tma_prefetch(&tm_a);
+    tma_prefetch(&tm_b);
+  }
+  // Lookup table: byte (even element in the high nibble) -> the two unscaled
+  // levels in the compute type, one copy per lane so 32 lanes never share a
+  // bank.  A warp writes the 32 copies of one entry at a time; lane c holds
+  // level c (mod 16) and the entry's two levels come by shuffle.  It reads no
+  // input, so it runs before the wait on the previous kernel.
+  {
+    uint32_t my = 0;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) my = (lane & 15) == c ? level_bits(c) : my;
+    const float lv = __uint_as_float(my);
+    for (int e = warp; e < 256; e += kGvWarps) {
+      const float hi = __shfl_sync(0xffffffffu, lv, e >> 4);
+      const float lo = __shfl_sync(0xffffffffu, lv, e & 15);
+      lut[e * 32 + lane] = pack2_rn<F16>(hi, lo);
     }
   }
-  // Block scales: independent loads issued up front (row = t & 127).
+  __syncthreads();
+  // This CTA's barriers are initialized: the cluster may push to it once every
+  // CTA has arrived here (the matching wait comes before the first push).
+  cluster_arrive();
+  // Programmatic dependent launch: the next kernel on the stream may start its
+  // own set-up now; this one reads no input and writes no output before the
+  // previous kernel has completed and its writes are visible.
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // Block scales: raw loads, converted after the TMA copies are out.  A row's
+  // 16 u8 scales (or 16 fp32) are one or four 16-byte loads when aligned.
   const bool dq = p.double_quant != 0;
+  const float s_g = dq ? __ldg(p.absmax_scale) : 0.0f;
+  const int srow = threadIdx.x & (kGvRows - 1);
+  const int64_t swr = int64_t(n0) + srow;
+  const int64_t sidx0 = swr * p.kb_per_row + kb0;
+  const bool svec = nblk == kGvMaxBlocks && swr < p.N && p.vec_scales;
+  uint4 sv = make_uint4(0u, 0u, 0u, 0u);
+  if (svec && dq) {
+    if (threadIdx.x < kGvRows) sv = __ldg(reinterpret_cast<const uint4*>(p.absmax_q + sidx0));
+  } else if (svec) {
+    if (threadIdx.x < 4 * kGvRows)
+      sv = __ldg(reinterpret_cast<const uint4*>(p.absmax + sidx0) + (threadIdx.x >> 7));
+  }
   constexpr int kScaleSteps = kGvThreads / kGvRows;          // threads per row
-  float sc_reg[(kGvMaxBlocks + kScaleSteps - 1) / kScaleSteps];
-  {
-    const float s_g = dq ? __ldg(p.absmax_scale) : 0.0f;
-    const int row = threadIdx.x & (kGvRows - 1);
-    const int64_t wr = int64_t(n0) + row;
+  constexpr int kScaleRegs = (kGvMaxBlocks + kScaleSteps - 1) / kScaleSteps;
+  uint32_t sc_raw[kScaleRegs];
+  if (!svec) {
 #pragma unroll
-    for (int j = 0; j < (kGvMaxBlocks + kScaleSteps - 1) / kScaleSteps; ++j) {
+    for (int j = 0; j < kScaleRegs; ++j) {
       const int b = (threadIdx.x >> 7) + kScaleSteps * j;
-      float v = 0.0f;
-      if (b < nblk && wr < p.N) {
-        const int64_t idx = wr * p.kb_per_row + kb0 + b;
-        v = dq ? __fmul_rn(float(__ldg(p.absmax_q + idx)), s_g) : __ldg(p.absmax + idx);
+      uint32_t v = 0;
+      if (b < nblk && swr < p.N)
+        v = dq ? uint32_t(__ldg(p.absmax_q + sidx0 + b)) : __float_as_uint(__ldg(p.absmax + sidx0 + b));
+      sc_raw[j] = v;
+    }
+  }
+
+  // Every byte this CTA reads is requested now: per group of four K blocks one
+  // code box (128 rows x 128 B), one x box and one A box, each issued by its
+  // own warp (one warp keeps only a few TMA copies going per microsecond), all
+  // three completing on the group's barrier; the last warp loads the B rows.
+  if (lane == 0) {
+    if (warp < 3 * groups) {
+      const int grp = warp / 3, part = warp % 3, b = grp * kGvGroup, kb = kb0 + b;
+      if (part == 0) {
+        mbar_arrive_expect_tx(&bar[grp], uint32_t(kGvRows) * 128u);
+        tma_load_2d(codes + grp * (kGvRows * 128), &tm_codes, &bar[grp], kb * 32, n0);
+      } else if (part == 1) {
+        mbar_arrive_expect_tx(&bar[grp], xbytes * kGvGroup);
+        tma_load_3d(xs + b * xbytes, &tm_x, &bar[grp], 0, 0, kb);
+      } else {
+        mbar_arrive_expect_tx(&bar[grp], abytes * kGvGroup);
+        tma_load_3d(as + b * abytes, &tm_a, &bar[grp], 0, 0, kb);
       }
-      sc_reg[j] = v;
+    } else if (warp == kGvWarps - 1) {
+      mbar_arrive_expect_tx(bar_b, uint32_t(kGvRows) * uint32_t(p.r) * 2u);
+      tma_load_2d(smem + L.bs, &tm_b, bar_b, 0, n0);
     }
   }
-  // Lookup table: byte (even element in the high nibble) -> bf16x2 of the two
-  // unscaled levels, one copy per lane so 32 lanes never share a bank.
-  for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-    const int e = i >> 5;
-    if (F16) {
-      const __half2 h = __floats2half2_rn(level(e >> 4), level(e & 15));
-      lut[i] = *reinterpret_cast<const uint32_t*>(&h);
-    } else {
-      const __nv_bfloat162 h = __floats2bfloat162_rn(level(e >> 4), level(e & 15));
-      lut[i] = *reinterpret_cast<const uint32_t*>(&h);
-    }
-  }
+
   {
-    const int row = threadIdx.x & (kGvRows - 1);
+    float* srow_dst = scales + srow * kGvMaxBlocks;
+    if (svec && dq) {
+      if (threadIdx.x < kGvRows) {
+        const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
-    for (int j = 0; j < (kGvMaxBlocks + kScaleSteps - 1) / kScaleSteps; ++j) {
-      const int b = (threadIdx.x >> 7) + kScaleSteps * j;
-      if (b < kGvMaxBlocks) scales[row * kGvMaxBlocks + b] = sc_reg[j];
+        for (int b = 0; b < 16; ++b) srow_dst[b] = __fmul_rn(float((w[b >> 2] >> (8 * (b & 3))) & 0xffu), s_g);
+      }
+    } else if (svec) {
+      if (threadIdx.x < 4 * kGvRows)
+        *reinterpret_cast<uint4*>(srow_dst + 4 * (threadIdx.x >> 7)) = sv;
+    } else {
+#pragma unroll
+      for (int j = 0; j < kScaleRegs; ++j) {
+        const int b = (threadIdx.x >> 7) + kScaleSteps * j;
+        const float v = dq ? __fmul_rn(float(sc_raw[j]), s_g) : __uint_as_float(sc_raw[j]);
+        if (b < kGvMaxBlocks) srow_dst[b] = v;
+      }
     }
   }
   __syncthreads();
 
-  float acc[NT8][4];
+  float acc[RG][NT8][4];
 #pragma unroll
-  for (int t = 0; t < NT8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+  for (int i = 0; i < RG; ++i)
+#pragma unroll
+    for (int t = 0; t < NT8; ++t) acc[i][t][0] = acc[i][t][1] = acc[i][t][2] = acc[i][t][3] = 0.0f;
   bool ok = true;
+  const int set = warp % kSets;                // W warps: row groups set*RG .. +RG-1
+  const int phase = warp / kSets;              //          K blocks phase, phase + kPhases, ...
 
   if (warp < kGvWWarps) {
-    // ---- W rows r0 and r0 + 8 of a 16-row group; the two warps of a group
-    // take alternate K blocks.
-    const int r0 = (warp & 7) * 16 + g;
-    const int half = warp >> 3;
     const uint32_t lane_off = uint32_t(lane) << 2;
     const uint8_t* lut_bytes = reinterpret_cast<const uint8_t*>(lut);
-    for (int b = half; b < nblk; b += 2) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar[b], 0, &abort_flag, p.status));
+    for (int b = phase; b < nblk; b += kPhases) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar[b / kGvGroup], 0, &abort_flag, p.status));
       if (!ok) break;
-      const uint8_t* cb = codes + b * 4096;
-      const uint2 w0 = *reinterpret_cast<const uint2*>(cb + r0 * 32 + 8 * q);
-      const uint2 w1 = *reinterpret_cast<const uint2*>(cb + (r0 + 8) * 32 + 8 * q);
-      uint32_t afr[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t wa = i < 2 ? w0.x : w0.y, wb = i < 2 ? w1.x : w1.y;
-        const int j = (2 * i) & 3;
-        afr[i][0] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wa, j, lane_off));
-        afr[i][1] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wb, j, lane_off));
-        afr[i][2] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wa, j + 1, lane_off));
-        afr[i][3] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wb, j + 1, lane_off));
-      }
-      const float s0 = scales[r0 * kGvMaxBlocks + b];
-      const float s8 = scales[(r0 + 8) * kGvMaxBlocks + b];
+      const uint8_t* cb = codes + (b / kGvGroup) * (kGvRows * 128);
       const uint8_t* xt = xs + b * xbytes;
+      uint4 xl[NT8], xh[NT8];
 #pragma unroll
-      for (int t = 0; t < NT8; ++t) {
-        uint4 xl, xh;
-        load_row16(xt, 8 * t + g, q, xl, xh);
-        float blk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int t = 0; t < NT8; ++t) load_row16(xt, 8 * t + g, q, xl[t], xh[t]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t b0, b1;
-          frag_pair(xl, xh, i, b0, b1);
-          mma_16816<F16>(blk, afr[i], b0, b1);
+      for (int i = 0; i < RG; ++i) {
+        const int wr0 = (set * RG + i) * 16 + 2 * g;      // W rows wr0 (MMA row g), wr0 + 1 (g + 8)
+        const uint2 w0 = load_codes8(cb, uint32_t(wr0), uint32_t(b % kGvGroup), uint32_t(q));
+        const uint2 w1 = load_codes8(cb, uint32_t(wr0 + 1), uint32_t(b % kGvGroup), uint32_t(q));
+        uint32_t afr[4][4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t wa = k < 2 ? w0.x : w0.y, wb = k < 2 ? w1.x : w1.y;
+          const int j = (2 * k) & 3;
+          afr[k][0] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wa, j, lane_off));
+          afr[k][1] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wb, j, lane_off));
+          afr[k][2] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wa, j + 1, lane_off));
+          afr[k][3] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wb, j + 1, lane_off));
         }
-        acc[t][0] = fmaf(s0, blk[0], acc[t][0]);
-        acc[t][1] = fmaf(s0, blk[1], acc[t][1]);
-        acc[t][2] = fmaf(s8, blk[2], acc[t][2]);
-        acc[t][3] = fmaf(s8, blk[3], acc[t][3]);
+        const float s0 = scales[wr0 * kGvMaxBlocks + b];
+        const float s1 = scales[(wr0 + 1) * kGvMaxBlocks + b];
+#pragma unroll
+        for (int t = 0; t < NT8; ++t) {
+          float blk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint32_t b0, b1;
+            frag_pair(xl[t], xh[t], k, b0, b1);
+            mma_16816<F16>(blk, afr[k], b0, b1);
+          }
+          acc[i][t][0] = fmaf(s0, blk[0], acc[i][t][0]);
+          acc[i][t][1] = fmaf(s0, blk[1], acc[i][t][1]);
+          acc[i][t][2] = fmaf(s1, blk[2], acc[i][t][2]);
+          acc[i][t][3] = fmaf(s1, blk[3], acc[i][t][3]);
+        }
       }
     }
   } else {
     // ---- adapter rows j0 + g and j0 + g + 8 of x A^T over this K slice
     const int j0 = (warp - kGvWWarps) * 16;
     if (j0 < p.r) {
+      float ta[NT8][4];
+#pragma unroll
+      for (int t = 0; t < NT8; ++t) ta[t][0] = ta[t][1] = ta[t][2] = ta[t][3] = 0.0f;
       for (int b = 0; b < nblk; ++b) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar[b], 0, &abort_flag, p.status));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[b / kGvGroup], 0, &abort_flag, p.status));
         if (!ok) break;
         const uint8_t* at = as + b * abytes;
         const uint8_t* xt = xs + b * xbytes;
@@ -309,125 +425,149 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         load_row16(at, j0 + g + 8, q, bl, bh);
         uint32_t afr[4][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          frag_pair(al, ah, i, afr[i][0], afr[i][2]);
-          frag_pair(bl, bh, i, afr[i][1], afr[i][3]);
+        for (int k = 0; k < 4; ++k) {
+          frag_pair(al, ah, k, afr[k][0], afr[k][2]);
+          frag_pair(bl, bh, k, afr[k][1], afr[k][3]);
         }
 #pragma unroll
         for (int t = 0; t < NT8; ++t) {
           uint4 xl, xh;
           load_row16(xt, 8 * t + g, q, xl, xh);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int k = 0; k < 4; ++k) {
             uint32_t b0, b1;
-            frag_pair(xl, xh, i, b0, b1);
-            mma_16816<F16>(acc[t], afr[i], b0, b1);
+            frag_pair(xl, xh, k, b0, b1);
+            mma_16816<F16>(ta[t], afr[k], b0, b1);
           }
         }
       }
 #pragma unroll
       for (int t = 0; t < NT8; ++t) {
-        tpart[(j0 + g) * NP + 8 * t + 2 * q] = acc[t][0];
-        tpart[(j0 + g) * NP + 8 * t + 2 * q + 1] = acc[t][1];
-        tpart[(j0 + g + 8) * NP + 8 * t + 2 * q] = acc[t][2];
-        tpart[(j0 + g + 8) * NP + 8 * t + 2 * q + 1] = acc[t][3];
+        tpart[(j0 + g) * NP + 8 * t + 2 * q] = ta[t][0];
+        tpart[(j0 + g) * NP + 8 * t + 2 * q + 1] = ta[t][1];
+        tpart[(j0 + g + 8) * NP + 8 * t + 2 * q] = ta[t][2];
+        tpart[(j0 + g + 8) * NP + 8 * t + 2 * q + 1] = ta[t][3];
+      }
+    }
+  }
+  __syncthreads();    // every K block consumed; tpart complete
+
+  // The block phases of each row-group set meet in phase 0.
+  if (warp < kGvWWarps && phase > 0) {
+    float* dst = red + size_t(phase - 1) * kGvRows * NP;
+#pragma unroll
+    for (int i = 0; i < RG; ++i) {
+      const int wr0 = (set * RG + i) * 16 + 2 * g;
+#pragma unroll
+      for (int t = 0; t < NT8; ++t) {
+        *reinterpret_cast<float2*>(dst + wr0 * NP + 8 * t + 2 * q) = make_float2(acc[i][t][0], acc[i][t][1]);
+        *reinterpret_cast<float2*>(dst + (wr0 + 1) * NP + 8 * t + 2 * q) = make_float2(acc[i][t][2], acc[i][t][3]);
       }
     }
   }
   __syncthreads();
+  cluster_wait();     // every CTA of the cluster has initialized its barriers
 
-  // The odd-block half of each row group hands its sums to the even half.
-  if (warp >= 8 && warp < kGvWWarps) {
-    const int r0 = (warp & 7) * 16 + g;
+  if (warp < kGvWWarps && phase == 0) {
 #pragma unroll
-    for (int t = 0; t < NT8; ++t) {
-      part[r0 * NP + 8 * t + 2 * q] = acc[t][0];
-      part[r0 * NP + 8 * t + 2 * q + 1] = acc[t][1];
-      part[(r0 + 8) * NP + 8 * t + 2 * q] = acc[t][2];
-      part[(r0 + 8) * NP + 8 * t + 2 * q + 1] = acc[t][3];
-    }
-  }
-  __syncthreads();
-  if (warp < 8) {
-    // This slice's share of the adapter term, s (x A^T)_slice B^T, on the
-    // W-row accumulators; then the partial tile goes to shared memory.
-    const int r0 = warp * 16 + g;
+    for (int ph = 1; ph < kPhases; ++ph) {
+      const float* src = red + size_t(ph - 1) * kGvRows * NP;
 #pragma unroll
-    for (int t = 0; t < NT8; ++t) {
-      acc[t][0] += part[r0 * NP + 8 * t + 2 * q];
-      acc[t][1] += part[r0 * NP + 8 * t + 2 * q + 1];
-      acc[t][2] += part[(r0 + 8) * NP + 8 * t + 2 * q];
-      acc[t][3] += part[(r0 + 8) * NP + 8 * t + 2 * q + 1];
-    }
-    ok = __all_sync(0xffffffffu, mbar_wait(&bar[kGvMaxBlocks], 0, &abort_flag, p.status));
-    if (ok) {
-      const __nv_bfloat16* b0row = bs + r0 * p.r;
-      const __nv_bfloat16* b8row = bs + (r0 + 8) * p.r;
-      for (int j = 0; j < p.r; ++j) {
-        const float bv0 = p.s * to_f32<F16>(b0row[j]);
-        const float bv8 = p.s * to_f32<F16>(b8row[j]);
+      for (int i = 0; i < RG; ++i) {
+        const int wr0 = (set * RG + i) * 16 + 2 * g;
 #pragma unroll
         for (int t = 0; t < NT8; ++t) {
-          const float t0 = tpart[j * NP + 8 * t + 2 * q];
-          const float t1 = tpart[j * NP + 8 * t + 2 * q + 1];
-          acc[t][0] = fmaf(bv0, t0, acc[t][0]);
-          acc[t][1] = fmaf(bv0, t1, acc[t][1]);
-          acc[t][2] = fmaf(bv8, t0, acc[t][2]);
-          acc[t][3] = fmaf(bv8, t1, acc[t][3]);
+          const float2 u = *reinterpret_cast<const float2*>(src + wr0 * NP + 8 * t + 2 * q);
+          const float2 v = *reinterpret_cast<const float2*>(src + (wr0 + 1) * NP + 8 * t + 2 * q);
+          acc[i][t][0] += u.x;
+          acc[i][t][1] += u.y;
+          acc[i][t][2] += v.x;
+          acc[i][t][3] += v.y;
         }
       }
     }
+    // This slice's share of the adapter term, (s T_slice) B^T, as MMAs with
+    // the tile's B rows (bf16 in shared memory) as A and s T_slice rounded to
+    // the compute type as B.
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar_b, 0, &abort_flag, p.status));
+    if (ok) {
+      for (int j0 = 0; j0 < p.r_pad; j0 += 16) {
+        uint32_t tfr[NT8][2];
 #pragma unroll
-    for (int t = 0; t < NT8; ++t) {
-      part[r0 * NP + 8 * t + 2 * q] = acc[t][0];
-      part[r0 * NP + 8 * t + 2 * q + 1] = acc[t][1];
-      part[(r0 + 8) * NP + 8 * t + 2 * q] = acc[t][2];
-      part[(r0 + 8) * NP + 8 * t + 2 * q + 1] = acc[t][3];
+        for (int t = 0; t < NT8; ++t) {
+          const int m = 8 * t + g;
+          const int ja = j0 + 2 * q, jb = j0 + 2 * q + 8;
+          tfr[t][0] = pack2_rn<F16>(p.s * tpart[ja * NP + m], p.s * tpart[(ja + 1) * NP + m]);
+          tfr[t][1] = pack2_rn<F16>(p.s * tpart[jb * NP + m], p.s * tpart[(jb + 1) * NP + m]);
+        }
+        // B columns j >= r hold no adapter: masked to 0 (tpart rows r .. r_pad-1
+        // are 0 too, from the zero-filled A rows)
+        const bool lo_ok = j0 + 2 * q < p.r, hi_ok = j0 + 2 * q + 8 < p.r;
+#pragma unroll
+        for (int i = 0; i < RG; ++i) {
+          const int wr0 = (set * RG + i) * 16 + 2 * g;
+          const uint32_t* b0row = reinterpret_cast<const uint32_t*>(bs + wr0 * p.r);
+          const uint32_t* b1row = reinterpret_cast<const uint32_t*>(bs + (wr0 + 1) * p.r);
+          uint32_t afr[4];
+          afr[0] = lo_ok ? b0row[(j0 >> 1) + q] : 0u;
+          afr[1] = lo_ok ? b1row[(j0 >> 1) + q] : 0u;
+          afr[2] = hi_ok ? b0row[(j0 >> 1) + q + 4] : 0u;
+          afr[3] = hi_ok ? b1row[(j0 >> 1) + q + 4] : 0u;
+#pragma unroll
+          for (int t = 0; t < NT8; ++t) mma_16816<F16>(acc[i][t], afr, tfr[t][0], tfr[t][1]);
+        }
+      }
+    }
+    // Push each row's partial to the CTA that owns its band of the tile; the
+    // bytes complete on that CTA's receive barrier.
+#pragma unroll
+    for (int i = 0; i < RG; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = (set * RG + i) * 16 + 2 * g + h;
+        const int owner = row / band;
+        const uint32_t dst = mapa_shared(
+            smem_u32(recv + (size_t(slice) * band + (row - owner * band)) * NP), uint32_t(owner));
+        const uint32_t obar = mapa_shared(smem_u32(bar_recv), uint32_t(owner));
+#pragma unroll
+        for (int t = 0; t < NT8; ++t)
+          st_async_f2(dst + uint32_t(8 * t + 2 * q) * 4u, acc[i][t][2 * h], acc[i][t][2 * h + 1], obar);
+      }
     }
   }
 
-  cluster_sync();
-
-  if (p.t_out != nullptr && blockIdx.x == 0 && slice == 0) {
-    // T = s x A^T for the caller: the slices' adapter partials summed.
-    const uint32_t tbase = smem_u32(tpart);
-    for (int i = threadIdx.x; i < p.M * p.r; i += blockDim.x) {
-      const int m = i / p.r, j = i % p.r;
-      const uint32_t off = uint32_t((j * NP + m) * 4);
+  // This CTA's band: the slices' partials summed in slice order, plus bias,
+  // rounded once.  Thread = (row, token); consecutive threads on consecutive
+  // rows so the y stores coalesce.
+  const bool got = mbar_wait_cluster(bar_recv, 0, &abort_flag, p.status);
+  if (got) {
+    for (int i = threadIdx.x; i < band * p.M; i += blockDim.x) {
+      const int rr = i % band, m = i / band;
+      const int n = n0 + slice * band + rr;
+      if (n >= p.N) continue;
       float v = 0.0f;
-      for (int sl = 0; sl < p.slices; ++sl) v += ld_shared_cluster_f32(mapa_shared(tbase + off, uint32_t(sl)));
-      p.t_out[i] = from_f32<F16>(p.s * v);
+      for (int sl = 0; sl < S; ++sl) v += recv[(size_t(sl) * band + rr) * NP + m];
+      if (p.bias != nullptr) v += to_f32<F16>(p.bias[n]);
+      p.y[int64_t(m) * p.N + n] = from_f32<F16>(v);
     }
   }
-
-  // This CTA's band of the 128 rows: the slices' partials summed in slice
-  // order, plus bias, rounded to bf16.  Thread = (row, 4 tokens); consecutive
-  // threads on consecutive rows so the y stores coalesce.
-  const int rows_per = kGvRows / p.slices;
-  const uint32_t pbase = smem_u32(part);
-  for (int i = threadIdx.x; i < rows_per * (NP / 4); i += blockDim.x) {
-    const int rr = i % rows_per, mq = i / rows_per;
-    const int trow = slice * rows_per + rr;
-    const int n = n0 + trow;
-    if (n >= p.N || 4 * mq >= p.M) continue;
-    const uint32_t off = uint32_t((trow * NP + 4 * mq) * 4);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sl = 0; sl < p.slices; ++sl) {
-      const float4 w = ld_shared_cluster_f4(mapa_shared(pbase + off, uint32_t(sl)));
-      v.x += w.x;
-      v.y += w.y;
-      v.z += w.z;
-      v.w += w.w;
+  if (pull_t) {
+    // T = s x A^T for the caller: the slices' adapter partials summed in slice
+    // order by slice 0, between two cluster barriers (the first publishes every
+    // CTA's tpart, the second keeps it alive until it has been read).
+    cluster_sync();
+    if (slice == 0) {
+      const uint32_t tbase = smem_u32(tpart);
+      for (int i = threadIdx.x; i < p.M * p.r; i += blockDim.x) {
+        const int m = i / p.r, j = i % p.r;
+        const uint32_t off = uint32_t((j * NP + m) * 4);
+        float v = 0.0f;
+        for (int sl = 0; sl < S; ++sl) v += ld_shared_cluster_f32(mapa_shared(tbase + off, uint32_t(sl)));
+        p.t_out[i] = from_f32<F16>(p.s * v);
+      }
     }
-    const float bias = p.bias != nullptr ? to_f32<F16>(p.bias[n]) : 0.0f;
-    const float vals[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int m = 4 * mq + e;
-      if (m < p.M) p.y[int64_t(m) * p.N + n] = from_f32<F16>(vals[e] + bias);
-    }
+    cluster_sync();
   }
-  cluster_sync();
 }
 
 }  // namespace
@@ -443,23 +583,29 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   const int kb = int(a.K / 64);
   const int tiles = int((a.N + kGvRows - 1) / kGvRows);
   const int nt8 = a.M <= 8 ? 1 : (a.M <= 16 ? 2 : 4);
+  const int rg = nt8 == 4 ? 1 : 2;             // 16-row groups per W warp
+  const int phases = kGvWWarps / (8 / rg);
   const int np = 8 * nt8;
   const int r_pad = (a.r + 15) / 16 * 16;
   // K slices: one wave of one CTA per SM where possible, and everything a CTA
   // reads fits in its shared memory at once.
   int slices = 1;
-  while (slices < 8 && tiles * slices * 2 <= 148 && slices * 2 <= kb) slices *= 2;
+  while (slices < kGvMaxSlices && tiles * slices * 2 <= 148 && slices * 2 <= kb) slices *= 2;
   int bps = (kb + slices - 1) / slices;
-  while ((bps > kGvMaxBlocks || gemv_layout(bps, np, r_pad, a.r).total > 190u * 1024u) && slices < 8) {
+  auto fits = [&](int b) { return b <= kGvMaxBlocks && gemv_layout(b, np, r_pad, a.r, phases).total <= kGvMaxDynSmem; };
+  while (!fits(bps) && slices < kGvMaxSlices) {
     slices *= 2;
     bps = (kb + slices - 1) / slices;
   }
-  if (bps > kGvMaxBlocks || gemv_layout(bps, np, r_pad, a.r).total > 190u * 1024u)
-    return cudaErrorNotSupported;
+  if (!fits(bps)) return cudaErrorNotSupported;
   CUtensorMap tc, tx, ta, tb;
-  bool ok = make_map_2d(&tc, a.w->codes, false, uint64_t(a.K / 2), uint64_t(a.N), 32, kGvRows, false);
-  ok = ok && make_map_2d(&tx, a.x, true, uint64_t(a.K), uint64_t(a.M), 64, uint32_t(np), true);
-  ok = ok && make_map_2d(&ta, a.A, true, uint64_t(a.K), uint64_t(a.r), 64, uint32_t(r_pad), true);
+  // codes: 128 W rows x 128 code bytes (four K blocks) per box, 128-byte swizzle;
+  // x and A: [64 elements][rows][K blocks] boxes of four K blocks
+  bool ok = make_map_2d(&tc, a.w->codes, false, uint64_t(a.K / 2), uint64_t(a.N), 128, kGvRows, true);
+  ok = ok && make_map_3d(&tx, a.x, true, 64, uint64_t(a.M), uint64_t(kb), uint64_t(a.K) * 2, 128, 64,
+                         uint32_t(np), kGvGroup, true);
+  ok = ok && make_map_3d(&ta, a.A, true, 64, uint64_t(a.r), uint64_t(kb), uint64_t(a.K) * 2, 128, 64,
+                         uint32_t(r_pad), kGvGroup, true);
   ok = ok && make_map_2d(&tb, a.B, true, uint64_t(a.r), uint64_t(a.N), uint32_t(a.r), kGvRows, false);
   if (!ok) return cudaErrorInvalidValue;
   GemvParams p;
@@ -469,6 +615,11 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   p.r = a.r;
   p.kb_per_row = kb;
   p.blocks_per_slice = bps;
+  // a row's 16 scales of a slice start on a 16-byte boundary (u8) or a
+  // 16-byte boundary of fp32 (four vectors) for every row and slice
+  p.vec_scales = bps == kGvMaxBlocks &&
+                 (a.w->double_quant ? (kb % 16 == 0 && (reinterpret_cast<uintptr_t>(a.w->absmax_q) & 15u) == 0)
+                                    : (kb % 4 == 0 && (reinterpret_cast<uintptr_t>(a.w->absmax) & 15u) == 0));
   p.slices = slices;
   p.r_pad = r_pad;
   p.s = a.s;
@@ -476,30 +627,33 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   p.absmax_q = a.w->absmax_q;
   p.absmax = a.w->absmax;
   p.absmax_scale = a.w->absmax_scale;
-  p.B = static_cast<const __nv_bfloat16*>(a.B);
   p.bias = static_cast<const __nv_bfloat16*>(a.bias);
   p.y = static_cast<__nv_bfloat16*>(a.y);
   p.t_out = static_cast<__nv_bfloat16*>(a.t_out);
   p.status = a.status;
 
-  const size_t smem = gemv_layout(bps, np, r_pad, a.r).total;
+  const size_t smem = gemv_layout(bps, np, r_pad, a.r, phases).total;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(tiles), unsigned(slices), 1);
   cfg.blockDim = dim3(kGvThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = unsigned(slices);
   attr[0].val.clusterDim.z = 1;
+  // The kernel reads its inputs only after griddepcontrol.wait, so it may be
+  // launched while the previous kernel on the stream is still running.
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   // The shared-memory opt-in is set once per instantiation (the maximum the
   // decode path can ask for), not on every call.
   auto kernel_for = [](int n8, bool f16) {
-    if (f16) return n8 == 1 ? nf4_gemv<1, true> : (n8 == 2 ? nf4_gemv<2, true> : nf4_gemv<4, true>);
-    return n8 == 1 ? nf4_gemv<1, false> : (n8 == 2 ? nf4_gemv<2, false> : nf4_gemv<4, false>);
+    if (f16) return n8 == 1 ? nf4_gemv<1, 2, true> : (n8 == 2 ? nf4_gemv<2, 2, true> : nf4_gemv<4, 1, true>);
+    return n8 == 1 ? nf4_gemv<1, 2, false> : (n8 == 2 ? nf4_gemv<2, 2, false> : nf4_gemv<4, 1, false>);
   };
   static PerDeviceOnce attr_done[6];
   const int slot = (nt8 == 1 ? 0 : (nt8 == 2 ? 1 : 2)) + (a.f16 ? 3 : 0);
@@ -507,8 +661,7 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   cudaError_t e = cudaSuccess;
   const int dev = PerDeviceOnce::current();
   if (!attr_done[slot].done(dev)) {
-    const int max_smem = 190 * 1024;   // + the 32 KB static lookup table
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGvMaxDynSmem));
     if (e != cudaSuccess) return e;
     attr_done[slot].mark(dev);
   }

@@ -85,6 +85,12 @@ bool make_map_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_
 bool make_map_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                       uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
+// 3-D map (bf16 or u8 elements): dims innermost first, strides of dims 1 and
+// 2 in bytes, box per dim, optional 128-byte swizzle.
+bool make_map_3d(CUtensorMap* map, const void* base, bool bf16, uint64_t d0, uint64_t d1,
+                 uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0,
+                 uint32_t box1, uint32_t box2, bool swizzle128);
+
 // Decode-shape forward (gemv.cu): one kernel for M <= 32 tokens.
 bool decode_supported(int64_t M, int64_t N, int64_t K, int r);
 cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
