@@ -7,6 +7,7 @@
 // one u32 of packed codes out); the absmax of a block of bs elements is a
 // shuffle-xor reduction over the bs/8 lanes that hold it.
 #include <algorithm>
+#include <mutex>
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -40,41 +41,42 @@ __device__ __forceinline__ bool finite8(const float4& a, const float4& b) {
 // 2^120 and other blocks take the division.  A host test runs the three
 // steps in C over that range against the IEEE quotient.
 //
-// The nearest level then comes from a 65-entry bucket table over [-1, 1]:
-// bucket i = floor(32 (v + 1)) holds base_i = #{thresholds below the bucket's
-// lower edge} and the one threshold inside it (or +inf); code = base_i +
-// (v > threshold_i).  No threshold lies within 0.0016 of a bucket edge, far
-// beyond the 2^-24 rounding of the bucket index, so an index that lands one
-// bucket off for v next to an edge still gives the same code.
-struct Bucket {
-  float thr;
-  uint32_t base;
+// The nearest level then comes from two small tables.  One FFMA rounds
+// 32 v + 32 to an integer i in 0..64 (v is in [-1, 1]): bucket i covers
+// [(i - 32.5) / 32, (i - 31.5) / 32).  base[i] is the number of decision
+// thresholds below the bucket's lower edge, so the only threshold that can lie
+// inside it is thr[base[i]] and code = base[i] + (v > thr[base[i]]).  No
+// threshold lies within 2e-4 of a bucket edge, far beyond the index rounding,
+// so a v next to an edge gets the same code from either bucket.  base has 128
+// entries (every value of the low 7 bits, so a NaN, which the absmax pass
+// flags, still indexes inside the table) and thr ends with +inf.  A 128-byte
+// u8 table and a 64-byte fp32 table each occupy distinct banks, so no lookup
+// conflicts whatever the 32 lanes ask for.
+struct EncodeTables {
+  uint8_t base[128];
+  float thr[16];
 };
 
-__device__ __forceinline__ void init_buckets(Bucket* b) {
-  for (int i = threadIdx.x; i < 65; i += blockDim.x) {
-    const float lo = float(i) / 32.0f - 1.0f;           // exact
-    const float hi = lo + 1.0f / 32.0f;
+__device__ __forceinline__ void init_tables(EncodeTables& t) {
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+    const float lo = (float(i) - 32.5f) * (1.0f / 32.0f);   // exact
     uint32_t base = 0;
-    float thr = __int_as_float(0x7f800000);               // +inf
 #pragma unroll
-    for (int j = 0; j < 15; ++j) {
-      const float t = __uint_as_float(threshold_bits(j));
-      base += (t < lo) ? 1u : 0u;
-      if (t >= lo && t < hi) thr = t;
-    }
-    b[i].thr = thr;
-    b[i].base = base;
+    for (int j = 0; j < 15; ++j) base += (__uint_as_float(threshold_bits(j)) < lo) ? 1u : 0u;
+    t.base[i] = uint8_t(i <= 64 ? base : 15u);
   }
+#pragma unroll
+  for (int j = 0; j < 15; ++j)
+    if (threadIdx.x == j) t.thr[j] = __uint_as_float(threshold_bits(j));
+  if (threadIdx.x == 15) t.thr[15] = __int_as_float(0x7f800000);   // +inf
 }
 
-__device__ __forceinline__ uint32_t encode_bucket(float v, const Bucket* b) {
-  const float y = fmaf(v, 32.0f, 31.5f);
-  // Round to an integer in 0..64 for |v| <= 1; the min keeps a NaN (outside
-  // the contract, flagged by the absmax pass) inside the 65-entry table.
-  const uint32_t idx = min(__float_as_uint(__fadd_rn(y, 12582912.0f)) & 0x7fu, 64u);
-  const Bucket e = b[idx];
-  return e.base + (v > e.thr ? 1u : 0u);
+__device__ __forceinline__ uint32_t encode_fast(float v, const EncodeTables& t) {
+  // 12582944 = 1.5 * 2^23 + 32: the sum's ulp is 1, so the FFMA rounds 32 v to
+  // an integer, and the low 7 bits hold 32 + round(32 v)
+  const uint32_t i = __float_as_uint(fmaf(v, 32.0f, 12582944.0f)) & 0x7fu;
+  const uint32_t b = t.base[i];
+  return b + (v > t.thr[b] ? 1u : 0u);
 }
 
 __device__ __forceinline__ float div_corrected(float w, float a, float y) {
@@ -88,8 +90,8 @@ __device__ __forceinline__ bool fast_scale(float a) {
 
 // Codes of two elements packed as one byte, even element in the high nibble.
 __device__ __forceinline__ uint32_t pair_byte_fast(float w0, float w1, float a, float y,
-                                                   const Bucket* b) {
-  return (encode_bucket(div_corrected(w0, a, y), b) << 4) | encode_bucket(div_corrected(w1, a, y), b);
+                                                   const EncodeTables& t) {
+  return (encode_fast(div_corrected(w0, a, y), t) << 4) | encode_fast(div_corrected(w1, a, y), t);
 }
 
 // Codes of two elements packed as one byte, even element in the high nibble.
@@ -149,16 +151,16 @@ __device__ __forceinline__ float load1(const void* w, int64_t e) {
 }
 
 // G = block_size / 8 lanes per block (1, 2, 4, 8, 16 or 32); IN the input type.
+// Launched as exactly one resident wave; each thread walks the words a grid
+// stride apart, two words per step, and issues the next step's two loads
+// before encoding the current two, so 64 bytes per thread are always in
+// flight.
 template <int G, int IN>
 __global__ void __launch_bounds__(256) quantize_vec_kernel(
-    const void* __restrict__ w, int64_t n_words, int64_t blocks_per_row_unused,
-    uint32_t* __restrict__ codes, float* __restrict__ absmax, uint32_t* __restrict__ status,
-    uint32_t* __restrict__ gmax) {
-  (void)blocks_per_row_unused;
-  // let a programmatic dependent (the double-quant kernel) start launching
-  asm volatile("griddepcontrol.launch_dependents;");
-  __shared__ Bucket buckets[65];
-  init_buckets(buckets);
+    const void* __restrict__ w, int64_t n_words, uint32_t* __restrict__ codes,
+    float* __restrict__ absmax, uint32_t* __restrict__ status, uint32_t* __restrict__ gmax) {
+  __shared__ EncodeTables tab;
+  init_tables(tab);
   __syncthreads();
   float cta_max = 0.0f;
   bool bad = false;
@@ -169,9 +171,8 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
     uint32_t word;
     if (fast_scale(m)) {
       const float y = __frcp_rn(m);
-      word = pair_byte_fast(a.x, a.y, m, y, buckets) | (pair_byte_fast(a.z, a.w, m, y, buckets) << 8) |
-             (pair_byte_fast(b.x, b.y, m, y, buckets) << 16) |
-             (pair_byte_fast(b.z, b.w, m, y, buckets) << 24);
+      word = pair_byte_fast(a.x, a.y, m, y, tab) | (pair_byte_fast(a.z, a.w, m, y, tab) << 8) |
+             (pair_byte_fast(b.x, b.y, m, y, tab) << 16) | (pair_byte_fast(b.z, b.w, m, y, tab) << 24);
     } else {
       word = pair_byte(a.x, a.y, m) | (pair_byte(a.z, a.w, m) << 8) |
              (pair_byte(b.x, b.y, m) << 16) | (pair_byte(b.z, b.w, m) << 24);
@@ -179,16 +180,22 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
     __stcs(codes + i, word);
     if ((threadIdx.x & (G - 1)) == 0 && absmax != nullptr) absmax[i / G] = m;
   };
-  // Two words per thread per iteration, a grid-stride apart, both loaded before
-  // either is encoded (64 bytes in flight per thread).  The loop runs in whole
-  // warps so every lane takes part in the shuffles.
-  for (int64_t base = int64_t(blockIdx.x) * blockDim.x; base < n_words; base += 2 * stride) {
-    const int64_t i0 = base + threadIdx.x;
-    const int64_t i1 = i0 + stride;
+  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  int64_t base = int64_t(blockIdx.x) * blockDim.x;
+  float4 a0 = z4, b0 = z4, a1 = z4, b1 = z4;
+  {
+    const int64_t i0 = base + threadIdx.x, i1 = i0 + stride;
+    if (i0 < n_words) load8<IN>(w, i0, a0, b0);
+    if (i1 < n_words) load8<IN>(w, i1, a1, b1);
+  }
+  // The loop runs in whole warps so every lane takes part in the shuffles.
+  for (; base < n_words; base += 2 * stride) {
+    const int64_t i0 = base + threadIdx.x, i1 = i0 + stride;
+    const int64_t n0 = i0 + 2 * stride, n1 = n0 + stride;
+    float4 c0 = z4, d0 = z4, c1 = z4, d1 = z4;
+    if (n0 < n_words) load8<IN>(w, n0, c0, d0);
+    if (n1 < n_words) load8<IN>(w, n1, c1, d1);
     const bool v0 = i0 < n_words, v1 = i1 < n_words;
-    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), b0 = a0, a1 = a0, b1 = a0;
-    if (v0) load8<IN>(w, i0, a0, b0);
-    if (v1) load8<IN>(w, i1, a1, b1);
     bad |= (v0 && !finite8(a0, b0)) || (v1 && !finite8(a1, b1));
     float m0 = max_abs8(a0, b0), m1 = max_abs8(a1, b1);
 #pragma unroll
@@ -199,9 +206,16 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
     encode_word(i0, v0, a0, b0, m0);
     encode_word(i1, v1, a1, b1, m1);
     cta_max = fmaxf(cta_max, fmaxf(m0, m1));
+    a0 = c0;
+    b0 = d0;
+    a1 = c1;
+    b1 = d1;
   }
   if (bad) report(status, NF4_ERR_NONFINITE);
   if (gmax != nullptr) cta_global_max(cta_max, gmax);
+  // let a programmatic dependent (the double-quant kernel) launch: only now,
+  // so that its waiting CTAs never hold SM slots this grid still needs
+  asm volatile("griddepcontrol.launch_dependents;");
 }
 
 // Any even block size: one thread per block, two passes over its elements.
@@ -209,7 +223,6 @@ template <int IN>
 __global__ void __launch_bounds__(256) quantize_generic_kernel(
     const void* __restrict__ w, int64_t n_blocks, int bs, uint8_t* __restrict__ codes,
     float* __restrict__ absmax, uint32_t* __restrict__ status, uint32_t* __restrict__ gmax) {
-  asm volatile("griddepcontrol.launch_dependents;");
   float cta_max = 0.0f;
   bool bad = false;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
@@ -232,6 +245,7 @@ __global__ void __launch_bounds__(256) quantize_generic_kernel(
   }
   if (bad) report(status, NF4_ERR_NONFINITE);
   if (gmax != nullptr) cta_global_max(cta_max, gmax);
+  asm volatile("griddepcontrol.launch_dependents;");
 }
 
 // The short last block of a tensor whose size is not a multiple of the block
@@ -324,18 +338,6 @@ __global__ void __launch_bounds__(256) absmax_max_kernel(const float* __restrict
 
 // ------------------------------------------------------------------ dequant
 
-template <typename OutT>
-struct Store8;
-
-template <>
-struct Store8<float> {
-  __device__ __forceinline__ static void run(float* out, int64_t word, const float (&v)[8]) {
-    float4* o = reinterpret_cast<float4*>(out) + 2 * word;
-    __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
-    __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
-  }
-};
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -345,61 +347,89 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+
+
+// EPL elements per lane per step, so that every lane stores one 16-byte vector
+// and a warp's store covers 512 contiguous bytes: 4 for fp32 output (two code
+// bytes in), 8 for bf16 / f16 (four code bytes in).
+template <typename OutT>
+struct DqUnit;
 template <>
-struct Store8<__nv_bfloat16> {
-  __device__ __forceinline__ static void run(__nv_bfloat16* out, int64_t word, const float (&v)[8]) {
-    uint4 u = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                         pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-    __stcs(reinterpret_cast<uint4*>(out) + word, u);
-  }
+struct DqUnit<float> {
+  static constexpr int kElems = 4;
+  using Code = uint16_t;
+};
+template <>
+struct DqUnit<__nv_bfloat16> {
+  static constexpr int kElems = 8;
+  using Code = uint32_t;
+};
+template <>
+struct DqUnit<__half> {
+  static constexpr int kElems = 8;
+  using Code = uint32_t;
 };
 
+template <typename OutT>
+__device__ __forceinline__ void store_unit(OutT* out, int64_t unit, const float (&v)[8]);
 template <>
-struct Store8<__half> {
-  __device__ __forceinline__ static void run(__half* out, int64_t word, const float (&v)[8]) {
-    uint4 u = make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
-                         pack_f16x2(v[6], v[7]));
-    __stcs(reinterpret_cast<uint4*>(out) + word, u);
-  }
-};
+__device__ __forceinline__ void store_unit<float>(float* out, int64_t unit, const float (&v)[8]) {
+  __stcs(reinterpret_cast<float4*>(out) + unit, make_float4(v[0], v[1], v[2], v[3]));
+}
+template <>
+__device__ __forceinline__ void store_unit<__nv_bfloat16>(__nv_bfloat16* out, int64_t unit, const float (&v)[8]) {
+  __stcs(reinterpret_cast<uint4*>(out) + unit,
+         make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                    pack_bf16x2(v[6], v[7])));
+}
+template <>
+__device__ __forceinline__ void store_unit<__half>(__half* out, int64_t unit, const float (&v)[8]) {
+  __stcs(reinterpret_cast<uint4*>(out) + unit,
+         make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
+                    pack_f16x2(v[6], v[7])));
+}
 
-// Four code words per thread per iteration, a grid-stride apart, so every
-// warp-wide load and store stays contiguous while four loads are in flight.
+// Whole units of whole blocks (bs a multiple of 8).  Launched as one resident
+// wave; each thread handles kDqSteps units a grid stride apart per iteration,
+// all of their code and scale loads issued before the first is decoded.
+constexpr int kDqSteps = 4;
 template <typename OutT, bool kDouble>
-__global__ void __launch_bounds__(256) dequant_x4_kernel(
-    const uint32_t* __restrict__ codes, int64_t n_words, int bs_words_shift, int bs_words,
+__global__ void __launch_bounds__(256) dequant_vec_kernel(
+    const uint8_t* __restrict__ codes, int64_t n_units, int unit_shift, int units_per_block,
     const float* __restrict__ absmax, const uint8_t* __restrict__ absmax_q,
     const float* __restrict__ absmax_scale, OutT* __restrict__ out) {
-  __shared__ float lut[16];
+  using Code = typename DqUnit<OutT>::Code;
+  constexpr int E = DqUnit<OutT>::kElems;
+  __shared__ float lut[16];   // 16 words in 16 banks: conflict-free for any codes
   if (threadIdx.x < 16) lut[threadIdx.x] = level(threadIdx.x);
   __syncthreads();
   const float s_g = kDouble ? *absmax_scale : 0.0f;
+  const Code* c = reinterpret_cast<const Code*>(codes);
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t base = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; base < n_words;
-       base += 4 * stride) {
-    uint32_t words[4];
-    float scales[4];
+  for (int64_t base = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; base < n_units;
+       base += kDqSteps * stride) {
+    uint32_t word[kDqSteps];
+    float scale[kDqSteps];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kDqSteps; ++u) {
       const int64_t i = base + u * stride;
-      words[u] = i < n_words ? __ldcs(codes + i) : 0u;
-      const int64_t blk = bs_words_shift >= 0 ? (i >> bs_words_shift) : (i / bs_words);
-      scales[u] = i < n_words ? (kDouble ? __fmul_rn(float(__ldg(absmax_q + blk)), s_g)
-                                         : __ldg(absmax + blk))
-                              : 0.0f;
+      const bool ok = i < n_units;
+      word[u] = ok ? uint32_t(__ldcs(c + i)) : 0u;
+      const int64_t blk = unit_shift >= 0 ? (i >> unit_shift) : (i / units_per_block);
+      scale[u] = ok ? (kDouble ? __fmul_rn(float(__ldg(absmax_q + blk)), s_g) : __ldg(absmax + blk)) : 0.0f;
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kDqSteps; ++u) {
       const int64_t i = base + u * stride;
-      if (i >= n_words) break;
+      if (i >= n_units) break;
       float v[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t byte = (words[u] >> (8 * j)) & 0xffu;
-        v[2 * j] = __fmul_rn(lut[byte >> 4], scales[u]);
-        v[2 * j + 1] = __fmul_rn(lut[byte & 15u], scales[u]);
+      for (int j = 0; j < E / 2; ++j) {
+        const uint32_t byte = (word[u] >> (8 * j)) & 0xffu;
+        v[2 * j] = __fmul_rn(lut[byte >> 4], scale[u]);
+        v[2 * j + 1] = __fmul_rn(lut[byte & 15u], scale[u]);
       }
-      Store8<OutT>::run(out, i, v);
+      store_unit<OutT>(out, i, v);
     }
   }
 }
@@ -435,6 +465,27 @@ __global__ void __launch_bounds__(256) dequant_bytes_kernel(
   }
 }
 
+// CTAs of `kernel` (threads per CTA, no dynamic shared memory) resident on one
+// SM, from the occupancy calculator, cached per kernel and device.
+int resident_ctas(const void* kernel, int threads) {
+  struct Entry {
+    const void* fn;
+    int dev, n;
+  };
+  static std::mutex mu;
+  static Entry cache[64];
+  static int used = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].fn == kernel && cache[i].dev == dev) return cache[i].n;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1) n = 1;
+  if (used < 64) cache[used++] = Entry{kernel, dev, n};
+  return n;
+}
+
 int grid_for(int64_t work_items, int threads, int sms, int per_sm) {
   int64_t g = (work_items + threads - 1) / threads;
   const int64_t cap = int64_t(sms) * per_sm;
@@ -462,15 +513,19 @@ void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes,
   const bool vec = (bs % 8 == 0) && bs <= 256 && log2_exact(bs) >= 0;
   if (n_full > 0 && vec) {
     const int64_t n_words = n_full * bs / 8;
-    const int grid = grid_for(n_words, threads, sms, 8);
     uint32_t* c32 = reinterpret_cast<uint32_t*>(codes);
+    auto run = [&](auto kernel) {
+      // one resident wave: every CTA stays for the whole pass
+      const int grid = grid_for(n_words, threads, sms, resident_ctas(reinterpret_cast<const void*>(kernel), threads));
+      kernel<<<grid, threads, 0, stream>>>(w, n_words, c32, absmax_out, status, gmax);
+    };
     switch (bs / 8) {
-      case 1: quantize_vec_kernel<1, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
-      case 2: quantize_vec_kernel<2, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
-      case 4: quantize_vec_kernel<4, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
-      case 8: quantize_vec_kernel<8, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
-      case 16: quantize_vec_kernel<16, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
-      default: quantize_vec_kernel<32, IN><<<grid, threads, 0, stream>>>(w, n_words, 0, c32, absmax_out, status, gmax); break;
+      case 1: run(quantize_vec_kernel<1, IN>); break;
+      case 2: run(quantize_vec_kernel<2, IN>); break;
+      case 4: run(quantize_vec_kernel<4, IN>); break;
+      case 8: run(quantize_vec_kernel<8, IN>); break;
+      case 16: run(quantize_vec_kernel<16, IN>); break;
+      default: run(quantize_vec_kernel<32, IN>); break;
     }
     ++*launches;
   } else if (n_full > 0) {
@@ -558,22 +613,27 @@ cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int
   int n = 0;
   NF4_PROF_BEGIN(stream, kKDequantize);
   if (n_words > 0) {
-    const int bs_words = bs / 8;
-    const int shift = log2_exact(bs_words);
-    const int grid = grid_for((n_words + 3) / 4, threads, sms, 8);
-    const uint32_t* c = reinterpret_cast<const uint32_t*>(w.codes);
-#define NF4_DQ4_LAUNCH(T, D)                                                                    \
-  dequant_x4_kernel<T, D><<<grid, threads, 0, stream>>>(c, n_words, shift, bs_words, w.absmax, \
-                                                        w.absmax_q, w.absmax_scale,            \
-                                                        reinterpret_cast<T*>(out))
+    // units of E elements: 4 for fp32 output, 8 for bf16 / f16
+    const int E = out_dtype == NF4_F32 ? 4 : 8;
+    const int64_t n_units = n_words * 8 / E;
+    const int units_per_block = bs / E;
+    const int shift = log2_exact(units_per_block);
+    auto run = [&](auto kernel, auto* o) {
+      const int grid = grid_for((n_units + kDqSteps - 1) / kDqSteps, threads, sms,
+                                resident_ctas(reinterpret_cast<const void*>(kernel), threads));
+      kernel<<<grid, threads, 0, stream>>>(w.codes, n_units, shift, units_per_block, w.absmax,
+                                           w.absmax_q, w.absmax_scale, o);
+    };
     if (out_dtype == NF4_F32) {
-      if (dq) NF4_DQ4_LAUNCH(float, true); else NF4_DQ4_LAUNCH(float, false);
+      float* o = reinterpret_cast<float*>(out);
+      if (dq) run(dequant_vec_kernel<float, true>, o); else run(dequant_vec_kernel<float, false>, o);
     } else if (out_dtype == NF4_BF16) {
-      if (dq) NF4_DQ4_LAUNCH(__nv_bfloat16, true); else NF4_DQ4_LAUNCH(__nv_bfloat16, false);
+      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+      if (dq) run(dequant_vec_kernel<__nv_bfloat16, true>, o); else run(dequant_vec_kernel<__nv_bfloat16, false>, o);
     } else {
-      if (dq) NF4_DQ4_LAUNCH(__half, true); else NF4_DQ4_LAUNCH(__half, false);
+      __half* o = reinterpret_cast<__half*>(out);
+      if (dq) run(dequant_vec_kernel<__half, true>, o); else run(dequant_vec_kernel<__half, false>, o);
     }
-#undef NF4_DQ4_LAUNCH
     ++n;
   }
   if (byte1 > byte0) {
