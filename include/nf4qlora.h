@@ -205,8 +205,8 @@ NF4_API nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int 
  * entry point; it exists for those callers.
  * Arguments and results are those of nf4_quantize (same kernels, bit-identical
  * output); the scratch that nf4_quantize keeps in `workspace` lives instead in
- * a fixed device array inside the library, 4 MiB + 256 B, which every GPU
- * that loads the library holds until the process exits.  With double_quant
+ * a fixed device array inside the library, 4 MiB + 8 KiB + 256 B, which every
+ * GPU that loads the library holds until the process exits.  With double_quant
  * and absmax == NULL the block scales are kept there, so rows*cols/block_size
  * may not exceed 1048576 (NF4_ERR_WORKSPACE otherwise); with a caller absmax
  * buffer there is no size limit.  Calls no allocator (no cudaMalloc or
@@ -214,8 +214,8 @@ NF4_API nf4_status nf4_quantize(const float* w, int64_t rows, int64_t cols, int 
  * device (cudaGetSymbolAddress); the first call on a device is the one that
  * may load the library's device code there, so it should come before any
  * stream capture.  All calls share the array and it keeps the last call's
- * contents (the global-max word is cleared at the start of each call); calls
- * whose GPU work overlaps race.  Launches are counted in nf4_launch_count.
+ * contents (each call writes every value it reads from it, so nothing needs
+ * clearing); calls whose GPU work overlaps race.  Launches are counted in nf4_launch_count.
  * Non-finite input is not reported (there is no status word to read).
  */
 NF4_API nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t cols,

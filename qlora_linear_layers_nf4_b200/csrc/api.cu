@@ -33,9 +33,12 @@ nf4_status finish(cudaError_t e, int launches) {
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Quantize workspace: the header; with double quant also the per-CTA maxima of
+// the quantize grid and room for the fp32 block scales.
 size_t quantize_ws(int64_t numel, int bs, int dq) {
   size_t bytes = nf4::kWsHeader;
-  if (dq && bs > 0 && numel > 0) bytes += round_up(size_t((numel + bs - 1) / bs) * sizeof(float), 256);
+  if (dq && bs > 0 && numel > 0)
+    bytes += nf4::kWsMaxSlotsBytes + round_up(size_t((numel + bs - 1) / bs) * sizeof(float), 256);
   return bytes;
 }
 
@@ -81,8 +84,9 @@ int64_t g_prof_count[nf4::kNumKernelIds];
 double g_prof_ms[nf4::kNumKernelIds];
 
 const char* const kKernelNames[nf4::kNumKernelIds] = {
-    "nf4_quantize", "nf4_double_quant", "nf4_dequantize", "adapter_gemm",
-    "fused_nf4_gemm_fwd", "fused_nf4_gemm_dx", "nf4_gemv", "nf4_merge", "gemm_f32", "nf4_absmax_max"};
+    "nf4_quantize", "nf4_double_quant", "nf4_dequantize", "adapter_gemm_T",
+    "fused_nf4_gemm_fwd", "fused_nf4_gemm_dx", "nf4_gemv", "nf4_merge", "gemm_f32", "nf4_absmax_max",
+    "adapter_gemm_U", "adapter_gemm_dB", "adapter_gemm_dA"};
 
 cudaEvent_t prof_event() {
   if (!g_prof_free.empty()) {
@@ -246,21 +250,18 @@ nf4_status quantize_impl(const void* w, int in_dtype, int64_t rows, int64_t cols
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + nf4::kWsStatus);
-  uint32_t* gmax = reinterpret_cast<uint32_t*>(ws + nf4::kWsGlobalMax);
+  float* max_slots = reinterpret_cast<float*>(ws + nf4::kWsHeader);
   const int sms = sm_count();
   int launches = 0;
-  cudaError_t e = cudaSuccess;
   float* amax = absmax;
-  if (double_quant) {
-    if (amax == nullptr) amax = reinterpret_cast<float*>(ws + nf4::kWsHeader);
-    e = cudaMemsetAsync(gmax, 0, sizeof(uint32_t), st);
-  }
-  if (e == cudaSuccess)
-    e = nf4::launch_quantize(w, in_dtype, numel, block_size, codes, amax, status,
-                             double_quant ? gmax : nullptr, sms, st, &launches);
+  if (double_quant && amax == nullptr)
+    amax = reinterpret_cast<float*>(ws + nf4::kWsHeader + nf4::kWsMaxSlotsBytes);
+  int n_slots = 0;
+  cudaError_t e = nf4::launch_quantize(w, in_dtype, numel, block_size, codes, amax, status,
+                                       double_quant ? max_slots : nullptr, &n_slots, sms, st, &launches);
   if (e == cudaSuccess && double_quant)
-    e = nf4::launch_double_quant(amax, (numel + block_size - 1) / block_size, gmax, absmax_q, absmax_scale, sms, st,
-                                 &launches);
+    e = nf4::launch_double_quant(amax, (numel + block_size - 1) / block_size, max_slots, n_slots,
+                                 absmax_q, absmax_scale, sms, st, &launches);
   return finish(e, launches);
 }
 
@@ -307,8 +308,7 @@ nf4_status nf4_double_quant(const float* absmax, int64_t n_blocks, const float* 
       (absmax_q && !aligned16(absmax_q)))
     return NF4_ERR_ALIGNMENT;
   int launches = 0;
-  cudaError_t e = nf4::launch_double_quant(absmax, n_blocks, reinterpret_cast<const uint32_t*>(gmax),
-                                           absmax_q, absmax_scale, sm_count(),
+  cudaError_t e = nf4::launch_double_quant(absmax, n_blocks, gmax, 1, absmax_q, absmax_scale, sm_count(),
                                            static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches);
 }

@@ -33,13 +33,16 @@ struct PerDeviceOnce {
 // outside api.cu.
 void add_launches(int n);
 
-// w holds numel elements of in_dtype (NF4_F32, NF4_BF16 or NF4_F16).
+// w holds numel elements of in_dtype (NF4_F32, NF4_BF16 or NF4_F16).  With
+// max_slots, every CTA writes the max |w| it saw to one slot; *n_slots
+// receives how many were written (at most kMaxSlots).
 cudaError_t launch_quantize(const void* w, int in_dtype, int64_t numel, int bs, uint8_t* codes,
-                            float* absmax_out, uint32_t* status, uint32_t* gmax, int sms,
-                            cudaStream_t stream, int* launches);
+                            float* absmax_out, uint32_t* status, float* max_slots, int* n_slots,
+                            int sms, cudaStream_t stream, int* launches);
 
-cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uint32_t* gmax,
-                                uint8_t* absmax_q, float* absmax_scale, int sms,
+// Double quant with G = max over max_slots[0 .. n_slots).
+cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const float* max_slots,
+                                int n_slots, uint8_t* absmax_q, float* absmax_scale, int sms,
                                 cudaStream_t stream, int* launches);
 // Max of n non-negative fp32 scales into *gmax (bits), zeroing it first.
 cudaError_t launch_absmax_max(const float* absmax, int64_t n, uint32_t* gmax, int sms,
@@ -119,13 +122,16 @@ enum KernelId {
   kKQuantize = 0,
   kKDoubleQuant,
   kKDequantize,
-  kKAdapterGemm,
+  kKAdapterT,        // adapter_gemm computing T = s x A^T
   kKFusedFwd,
   kKFusedDx,
   kKGemv,
   kKMerge,
   kKGemmF32,
   kKAbsmaxMax,
+  kKAdapterU,        // adapter_gemm computing U = s dy B
+  kKAdapterDB,       // adapter_gemm computing dB = dy^T T
+  kKAdapterDA,       // adapter_gemm computing dA^T = x^T U
   kNumKernelIds
 };
 

@@ -46,8 +46,11 @@ __host__ __device__ constexpr uint32_t threshold_bits(int i) {
 
 // Layout of the head of every workspace (bytes).
 constexpr size_t kWsStatus = 0;        // u32 sticky device status (first error wins)
-constexpr size_t kWsGlobalMax = 4;     // u32 bit pattern of max absmax (double quant)
 constexpr size_t kWsHeader = 256;      // op-specific scratch starts here
+// Quantize with double quant: per-CTA maxima of the quantize grid (its size
+// is capped below this), then the fp32 block scales when the caller keeps none.
+constexpr int kMaxSlots = 2048;
+constexpr size_t kWsMaxSlotsBytes = size_t(kMaxSlots) * 4;
 
 __device__ __forceinline__ float level(int c) {
   return __uint_as_float(kLevelBitsDev[c]);

@@ -15,8 +15,8 @@
 // every call looks the address up with cudaGetSymbolAddress on the current
 // device (cheap once the module is loaded, and never stale after the context
 // was reset) and hands it to the kernels.  All calls on a device share the
-// array and it keeps the last call's contents, so the global-max word is
-// cleared at the start of every call; calls whose GPU work overlaps
+// array and it keeps the last call's contents: every call writes the per-CTA
+// maxima it reads, so nothing needs clearing; calls whose GPU work overlaps
 // (different streams, no ordering) race on it.
 #include "kernels.h"
 #include "nf4_common.cuh"
@@ -25,10 +25,11 @@
 namespace nf4 {
 namespace {
 
-// Header (unused status word, global-max word) + fp32 block scales for up to
-// 2^20 blocks (64 Mi elements at block size 64).
+// Header (unused) + the quantize grid's per-CTA maxima + fp32 block scales
+// for up to 2^20 blocks (64 Mi elements at block size 64).
 constexpr int64_t kNoAllocMaxBlocks = int64_t(1) << 20;
-constexpr size_t kNoAllocScratchBytes = kWsHeader + size_t(kNoAllocMaxBlocks) * sizeof(float);
+constexpr size_t kNoAllocScratchBytes =
+    kWsHeader + kWsMaxSlotsBytes + size_t(kNoAllocMaxBlocks) * sizeof(float);
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -81,7 +82,7 @@ extern "C" nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t
 
   uint8_t* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return NF4_ERR_CUDA;
-  uint32_t* gmax = reinterpret_cast<uint32_t*>(scratch + kWsGlobalMax);
+  float* max_slots = reinterpret_cast<float*>(scratch + kWsHeader);
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) {
@@ -90,17 +91,15 @@ extern "C" nf4_status nf4_quantize_noalloc(const float* w, int64_t rows, int64_t
       sms = n;
   }
   int launches = 0;
-  cudaError_t e = cudaSuccess;
   float* amax = absmax;
-  if (double_quant) {
-    if (amax == nullptr) amax = reinterpret_cast<float*>(scratch + kWsHeader);
-    e = cudaMemsetAsync(gmax, 0, sizeof(uint32_t), st);   // the array keeps the last call's max
-  }
-  if (e == cudaSuccess)
-    e = launch_quantize(w, NF4_F32, numel, block_size, codes, amax, /*status=*/nullptr,
-                        double_quant ? gmax : nullptr, sms, st, &launches);
+  if (double_quant && amax == nullptr)
+    amax = reinterpret_cast<float*>(scratch + kWsHeader + kWsMaxSlotsBytes);
+  int n_slots = 0;
+  cudaError_t e = launch_quantize(w, NF4_F32, numel, block_size, codes, amax, /*status=*/nullptr,
+                                  double_quant ? max_slots : nullptr, &n_slots, sms, st, &launches);
   if (e == cudaSuccess && double_quant)
-    e = launch_double_quant(amax, n_blocks, gmax, absmax_q, absmax_scale, sms, st, &launches);
+    e = launch_double_quant(amax, n_blocks, max_slots, n_slots, absmax_q, absmax_scale, sms, st,
+                            &launches);
   add_launches(launches);
   return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
 }

@@ -1107,6 +1107,7 @@ struct AdapterJob {
   float scale;
   __nv_bfloat16* out_bf16;
   float* out_f32;
+  int prof_id;       // profiler kernel id of this product
 };
 
 // A launch fully prepared on the host (tensor maps encoded, parameters set),
@@ -1116,6 +1117,7 @@ struct AdapterLaunch {
   AdapterParams p;
   dim3 grid;
   size_t smem;
+  int prof_id;
 };
 
 bool prepare_adapter(const AdapterJob& j, uint32_t* status, AdapterLaunch* L) {
@@ -1143,6 +1145,7 @@ bool prepare_adapter(const AdapterJob& j, uint32_t* status, AdapterLaunch* L) {
   p.status = status;
   L->grid = dim3(unsigned(sp.tiles), unsigned(sp.slices), 1);
   L->smem = kAdStages * (kAdABytes + size_t(NP) * 128) + 1024 + 256;
+  L->prof_id = j.prof_id;
   return true;
 }
 
@@ -1159,9 +1162,9 @@ cudaError_t launch_adapter(const AdapterLaunch& L, cudaStream_t st, int* launche
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  NF4_PROF_BEGIN(st, kKAdapterGemm);
+  NF4_PROF_BEGIN(st, L.prof_id);
   cudaError_t e = cudaLaunchKernelEx(&cfg, adapter_gemm, L.ma, L.mb, L.p);
-  NF4_PROF_END(st, kKAdapterGemm);
+  NF4_PROF_END(st, L.prof_id);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;
@@ -1203,6 +1206,7 @@ AdapterJob job_T(const LinearArgs& a, __nv_bfloat16* T) {
   j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = false;
   j.b = a.A; j.b_inner = a.K; j.b_outer = a.r; j.b_mn = false;
   j.Mo = a.M; j.red = a.K; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = T; j.f16 = a.f16;
+  j.prof_id = kKAdapterT;
   return j;
 }
 
@@ -1365,6 +1369,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = false;
     j.b = a.B; j.b_inner = a.r; j.b_outer = a.N; j.b_mn = true;
     j.Mo = a.M; j.red = a.N; j.r = a.r; j.kind = 0; j.scale = a.s; j.out_bf16 = U; j.f16 = a.f16;
+    j.prof_id = kKAdapterU;
     ok = ok && prepare_adapter(j, a.status, &lu);
   }
   {  // dB = dy^T T   (A: dy^T MN-major over m; B: T [M, r] MN-major over m)
@@ -1372,6 +1377,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     j.a = a.dy; j.a_inner = a.N; j.a_outer = a.M; j.a_mn = true;
     j.b = T; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
     j.Mo = a.N; j.red = a.M; j.r = a.r; j.kind = 1; j.scale = 1.0f; j.out_f32 = a.dB; j.f16 = a.f16;
+    j.prof_id = kKAdapterDB;
     ok = ok && prepare_adapter(j, a.status, &ldb);
   }
   {  // dA^T = x^T U  (A: x^T MN-major over m; B: U [M, r] MN-major over m), stored as dA [r, K]
@@ -1379,6 +1385,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     j.a = a.x; j.a_inner = a.K; j.a_outer = a.M; j.a_mn = true;
     j.b = U; j.b_inner = a.r; j.b_outer = a.M; j.b_mn = true;
     j.Mo = a.K; j.red = a.M; j.r = a.r; j.kind = 2; j.scale = 1.0f; j.out_f32 = a.dA; j.f16 = a.f16;
+    j.prof_id = kKAdapterDA;
     ok = ok && prepare_adapter(j, a.status, &lda);
   }
   // dx = dy W' + U A

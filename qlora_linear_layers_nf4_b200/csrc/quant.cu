@@ -102,6 +102,22 @@ __device__ __forceinline__ uint32_t pair_byte(float w0, float w1, float amax) {
   return (c0 << 4) | c1;
 }
 
+// Block-wide max of a non-negative float into this CTA's slot: the double
+// quant reduces the slots itself, so no word has to be zeroed before a call
+// and none keeps a value from an earlier one.
+__device__ __forceinline__ void cta_max_to_slot(float v, float* slot) {
+  __shared__ float red[32];
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < int(blockDim.x >> 5) ? red[lane] : 0.0f;
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) *slot = v;
+  }
+}
+
 // Block-wide max of a non-negative float, then one atomicMax per CTA on its
 // bit pattern (non-negative floats order like their unsigned bits).
 __device__ __forceinline__ void cta_global_max(float v, uint32_t* gmax) {
@@ -158,7 +174,7 @@ __device__ __forceinline__ float load1(const void* w, int64_t e) {
 template <int G, int IN>
 __global__ void __launch_bounds__(256) quantize_vec_kernel(
     const void* __restrict__ w, int64_t n_words, uint32_t* __restrict__ codes,
-    float* __restrict__ absmax, uint32_t* __restrict__ status, uint32_t* __restrict__ gmax) {
+    float* __restrict__ absmax, uint32_t* __restrict__ status, float* __restrict__ max_slots) {
   __shared__ EncodeTables tab;
   init_tables(tab);
   __syncthreads();
@@ -212,7 +228,7 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
     b1 = d1;
   }
   if (bad) report(status, NF4_ERR_NONFINITE);
-  if (gmax != nullptr) cta_global_max(cta_max, gmax);
+  if (max_slots != nullptr) cta_max_to_slot(cta_max, max_slots + blockIdx.x);
   // let a programmatic dependent (the double-quant kernel) launch: only now,
   // so that its waiting CTAs never hold SM slots this grid still needs
   asm volatile("griddepcontrol.launch_dependents;");
@@ -222,7 +238,7 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
 template <int IN>
 __global__ void __launch_bounds__(256) quantize_generic_kernel(
     const void* __restrict__ w, int64_t n_blocks, int bs, uint8_t* __restrict__ codes,
-    float* __restrict__ absmax, uint32_t* __restrict__ status, uint32_t* __restrict__ gmax) {
+    float* __restrict__ absmax, uint32_t* __restrict__ status, float* __restrict__ max_slots) {
   float cta_max = 0.0f;
   bool bad = false;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
@@ -244,7 +260,7 @@ __global__ void __launch_bounds__(256) quantize_generic_kernel(
     cta_max = fmaxf(cta_max, m);
   }
   if (bad) report(status, NF4_ERR_NONFINITE);
-  if (gmax != nullptr) cta_global_max(cta_max, gmax);
+  if (max_slots != nullptr) cta_max_to_slot(cta_max, max_slots + blockIdx.x);
   asm volatile("griddepcontrol.launch_dependents;");
 }
 
@@ -257,7 +273,7 @@ template <int IN>
 __global__ void __launch_bounds__(256) quantize_tail_kernel(
     const void* __restrict__ w, int64_t e0, int t, uint8_t* __restrict__ codes,
     float* __restrict__ absmax, int64_t blk, uint32_t* __restrict__ status,
-    uint32_t* __restrict__ gmax) {
+    float* __restrict__ max_slot) {
   __shared__ float red[8];
   float m = 0.0f;
   bool bad = false;
@@ -283,7 +299,7 @@ __global__ void __launch_bounds__(256) quantize_tail_kernel(
   }
   if (threadIdx.x == 0) {
     if (absmax != nullptr) absmax[blk] = m;
-    if (gmax != nullptr && m > 0.0f) atomicMax(gmax, __float_as_uint(m));
+    if (max_slot != nullptr) *max_slot = m;
   }
 }
 
@@ -301,9 +317,11 @@ __device__ __forceinline__ uint32_t dq_code(float a, float g, float s_g, bool fa
   return uint32_t(min(max(__float2int_rn(ratio), 0), 255));
 }
 
+// G = the max over n_slots values (the quantize grid's per-CTA maxima, or one
+// global max from the caller), reduced by every CTA for itself.
 __global__ void __launch_bounds__(256) double_quant_kernel(
-    const float* __restrict__ absmax, int64_t n_blocks, const uint32_t* __restrict__ gmax,
-    uint8_t* __restrict__ absmax_q, float* __restrict__ absmax_scale) {
+    const float* __restrict__ absmax, int64_t n_blocks, const float* __restrict__ max_slots,
+    int n_slots, uint8_t* __restrict__ absmax_q, float* __restrict__ absmax_scale) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t n4 = n_blocks / 4;
   const int64_t i4 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -311,7 +329,14 @@ __global__ void __launch_bounds__(256) double_quant_kernel(
   if (i4 < n4) a4 = reinterpret_cast<const float4*>(absmax)[i4];
   const int64_t tail = n4 * 4 + i4;
   const float at = (tail < n_blocks) ? absmax[tail] : 0.0f;
-  const float g = __uint_as_float(*gmax);
+  __shared__ float red[8];
+  float gm = 0.0f;
+  for (int i = threadIdx.x; i < n_slots; i += blockDim.x) gm = fmaxf(gm, __ldg(max_slots + i));
+  for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = gm;
+  __syncthreads();
+  float g = red[0];
+  for (int k = 1; k < int(blockDim.x >> 5); ++k) g = fmaxf(g, red[k]);
   const float s_g = __fdiv_rn(g, 255.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *absmax_scale = s_g;
   const bool fast = fast_scale(s_g);
@@ -505,8 +530,9 @@ int log2_exact(int v) {
 
 template <int IN>
 void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes, float* absmax_out,
-                           uint32_t* status, uint32_t* gmax, int sms, cudaStream_t stream,
-                           int* launches) {
+                           uint32_t* status, float* max_slots, int* n_slots, int sms,
+                           cudaStream_t stream, int* launches) {
+  *n_slots = 0;
   const int threads = 256;
   const int64_t n_full = numel / bs;          // whole blocks
   const int tail = int(numel - n_full * bs);  // elements of the short last block
@@ -516,8 +542,10 @@ void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes,
     uint32_t* c32 = reinterpret_cast<uint32_t*>(codes);
     auto run = [&](auto kernel) {
       // one resident wave: every CTA stays for the whole pass
-      const int grid = grid_for(n_words, threads, sms, resident_ctas(reinterpret_cast<const void*>(kernel), threads));
-      kernel<<<grid, threads, 0, stream>>>(w, n_words, c32, absmax_out, status, gmax);
+      const int grid = std::min(kMaxSlots - 1, grid_for(n_words, threads, sms,
+                                                         resident_ctas(reinterpret_cast<const void*>(kernel), threads)));
+      kernel<<<grid, threads, 0, stream>>>(w, n_words, c32, absmax_out, status, max_slots);
+      *n_slots = grid;
     };
     switch (bs / 8) {
       case 1: run(quantize_vec_kernel<1, IN>); break;
@@ -529,38 +557,41 @@ void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes,
     }
     ++*launches;
   } else if (n_full > 0) {
-    const int grid = grid_for(n_full, threads, sms, 8);
+    const int grid = std::min(kMaxSlots - 1, grid_for(n_full, threads, sms, 8));
     quantize_generic_kernel<IN><<<grid, threads, 0, stream>>>(w, n_full, bs, codes, absmax_out,
-                                                              status, gmax);
+                                                              status, max_slots);
+    *n_slots = grid;
     ++*launches;
   }
   if (tail > 0) {
     // an ordinary launch: it starts once the full-block kernel has finished
     quantize_tail_kernel<IN><<<1, threads, 0, stream>>>(w, n_full * bs, tail, codes, absmax_out,
-                                                        n_full, status, gmax);
+                                                        n_full, status,
+                                                        max_slots ? max_slots + *n_slots : nullptr);
+    *n_slots += 1;
     ++*launches;
   }
 }
 
 cudaError_t launch_quantize(const void* w, int in_dtype, int64_t numel, int bs, uint8_t* codes,
-                            float* absmax_out, uint32_t* status, uint32_t* gmax, int sms,
-                            cudaStream_t stream, int* launches) {
+                            float* absmax_out, uint32_t* status, float* max_slots, int* n_slots,
+                            int sms, cudaStream_t stream, int* launches) {
   int n = 0;
   NF4_PROF_BEGIN(stream, kKQuantize);
   if (in_dtype == NF4_BF16)
-    launch_quantize_typed<kInBF16>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream, &n);
+    launch_quantize_typed<kInBF16>(w, numel, bs, codes, absmax_out, status, max_slots, n_slots, sms, stream, &n);
   else if (in_dtype == NF4_F16)
-    launch_quantize_typed<kInF16>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream, &n);
+    launch_quantize_typed<kInF16>(w, numel, bs, codes, absmax_out, status, max_slots, n_slots, sms, stream, &n);
   else
-    launch_quantize_typed<kInF32>(w, numel, bs, codes, absmax_out, status, gmax, sms, stream, &n);
+    launch_quantize_typed<kInF32>(w, numel, bs, codes, absmax_out, status, max_slots, n_slots, sms, stream, &n);
   NF4_PROF_END(stream, kKQuantize);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) *launches += n;
   return e;
 }
 
-cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uint32_t* gmax,
-                                uint8_t* absmax_q, float* absmax_scale, int sms,
+cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const float* max_slots,
+                                int n_slots, uint8_t* absmax_q, float* absmax_scale, int sms,
                                 cudaStream_t stream, int* launches) {
   const int threads = 256;
   (void)sms;
@@ -577,8 +608,8 @@ cudaError_t launch_double_quant(const float* absmax, int64_t n_blocks, const uin
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   NF4_PROF_BEGIN(stream, kKDoubleQuant);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, double_quant_kernel, absmax, n_blocks, gmax, absmax_q,
-                                     absmax_scale);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, double_quant_kernel, absmax, n_blocks, max_slots, n_slots,
+                                     absmax_q, absmax_scale);
   NF4_PROF_END(stream, kKDoubleQuant);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
