@@ -71,95 +71,104 @@ def source_hash():
 
 # --------------------------------------------------------------------- clocks
 
+_NVML_POLLER = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+uuid, period = sys.argv[1], float(sys.argv[2])
+try:
+    h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+except pynvml.NVMLError:
+    h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[3]))
+mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+        pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap)
+print("ready", flush=True)
+while True:
+    t = time.monotonic()
+    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+    act = "|".join(n for n, b in zip(names, bits) if rs & b)
+    print(f"{t:.6f},{sm},{mx},{pw:.1f},{act}", flush=True)
+    time.sleep(period)
+"""
+
+
 class ClockSampler:
     """SM clock, power and throttle reasons sampled while timing.
 
-    NVML is polled from a background thread every few milliseconds, so even a
-    timed region of a few tens of milliseconds carries its own samples; the
-    device is found by UUID (CUDA and NVML may number GPUs differently).
-    Without NVML, nvidia-smi is sampled at its shortest interval instead.
-    The raw samples go to BENCH_OUT_DIR (default: the temp dir)."""
+    A separate process polls NVML every few milliseconds (no GIL shared with
+    the launching thread), with CLOCK_MONOTONIC stamps; the summary keeps the
+    samples that fall inside [start(), stop()].  The device is found by UUID
+    (CUDA and NVML may number GPUs differently).  Without NVML, nvidia-smi is
+    sampled at its shortest interval instead.  Raw samples go to
+    BENCH_OUT_DIR (default: the temp dir)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
-               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
-               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
-               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device, period_s=0.002):
         self.device = device
         self.period = period_s
-        self.samples = []            # (sm_mhz, max_mhz, power_w, {reason names})
-        self.thread = None
         self.proc = None
+        self.kind = None
         out_dir = os.environ.get("BENCH_OUT_DIR", tempfile.gettempdir())
-        self.path = os.path.join(out_dir, f"nf4_bench_clocks_gpu{getattr(device, 'index', 0)}.csv")
+        self.path = os.path.join(out_dir, f"nf4_bench_clocks_gpu{getattr(device, 'index', 0) or 0}.csv")
 
-    def _nvml_handle(self):
-        import pynvml
+    def launch(self):
+        """Start the poller (before warm-up: it takes a moment to come up)."""
         import torch
-        pynvml.nvmlInit()
-        props = torch.cuda.get_device_properties(self.device)
-        uuid = str(getattr(props, "uuid", "") or "")
-        if uuid:
-            try:
-                return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid if not uuid.startswith("GPU-") else uuid)
-            except pynvml.NVMLError:
-                pass
-        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(getattr(self.device, "index", 0) or 0)
-
-    def start(self):
-        import threading
+        os.makedirs(os.path.dirname(self.path) or ".", exist_ok=True)
+        self.fh = open(self.path, "w")
+        idx = getattr(self.device, "index", 0) or 0
+        uuid = str(getattr(torch.cuda.get_device_properties(self.device), "uuid", "") or "")
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         try:
-            nv, h = self._nvml_handle()
-        except Exception:
-            nv = None
-        if nv is not None:
-            self.stop_flag = threading.Event()
-            bits = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
-            max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-
-            def poll():
-                while not self.stop_flag.is_set():
-                    try:
-                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                        self.samples.append((float(sm), float(max_mhz), pw,
-                                             {n for n, b in bits if rs & b}))
-                    except Exception:
-                        pass
-                    self.stop_flag.wait(self.period)
-
-            self.thread = threading.Thread(target=poll, daemon=True)
-            self.thread.start()
-            return
+            self.proc = subprocess.Popen([sys.executable, "-c", _NVML_POLLER, uuid, str(self.period), str(idx)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            if self.proc.stdout.readline().strip() == "ready":
+                self.kind = "nvml"
+                return self
+            self.proc.kill()
+        except OSError:
+            pass
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(getattr(self.device, "index", 0) or 0), "-lms", "10"],
-                stdout=self.fh, stderr=subprocess.DEVNULL)
+                 "-i", str(idx), "-lms", "10"], stdout=self.fh, stderr=subprocess.DEVNULL)
+            self.kind = "nvidia-smi"
         except OSError:
             self.proc = None
+        return self
+
+    def start(self):
+        if self.proc is None and self.kind is None:
+            self.launch()
+        self.t0 = time.monotonic()
 
     def stop(self):
-        if self.thread is not None:
-            self.stop_flag.set()
-            self.thread.join(timeout=5)
-            src = "nvml"
-            try:
-                os.makedirs(os.path.dirname(self.path), exist_ok=True)
-                with open(self.path, "w") as f:
-                    for sm, mx, pw, rs in self.samples:
-                        f.write(f"{sm},{mx},{pw},{'|'.join(sorted(rs))}\n")
-            except OSError:
-                pass
-        elif self.proc is not None:
-            src = "nvidia-smi"
-            self.proc.terminate()
+        t1 = time.monotonic()
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0,
+                    "reasons": ["no clock source (NVML and nvidia-smi unavailable)"]}
+        time.sleep(2 * self.period)
+        self.proc.terminate()
+        samples = []
+        if self.kind == "nvml":
+            out, _ = self.proc.communicate(timeout=10)
+            self.fh.write(out)
+            for line in out.splitlines():
+                parts = line.split(",")
+                if len(parts) != 5:
+                    continue
+                t = float(parts[0])
+                if self.t0 <= t <= t1:
+                    samples.append((float(parts[1]), float(parts[2]), float(parts[3]),
+                                    {r for r in parts[4].split("|") if r}))
+        else:
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
@@ -174,24 +183,23 @@ class ClockSampler:
                         vals = float(parts[1]), float(parts[2]), float(parts[3])
                     except ValueError:
                         continue
-                    rs = {n for (n, _), v in zip(self.REASONS, parts[5:9]) if v.lower().startswith("active")}
-                    self.samples.append((*vals, rs))
-        else:
-            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0,
-                    "reasons": ["no clock source (NVML and nvidia-smi unavailable)"]}
-        sm = [x[0] for x in self.samples]
-        reasons = set()
-        counts = {}
-        for x in self.samples:
+                    rs = {n for n, v in zip(self.NAMES, parts[5:9]) if v.lower().startswith("active")}
+                    samples.append((*vals, rs))
+        if not self.fh.closed:
+            self.fh.close()
+        self.proc = None
+        sm = [x[0] for x in samples]
+        reasons, counts = set(), {}
+        for x in samples:
             reasons |= x[3]
             for n in x[3]:
                 counts[n] = counts.get(n, 0) + 1
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(x[1] for x in self.samples) if self.samples else None,
+                "sm_max_mhz": max(x[1] for x in samples) if samples else None,
                 "sm_min_mhz": min(sm) if sm else None,
-                "power_w_max": max(x[2] for x in self.samples) if self.samples else None,
-                "samples": len(sm), "source": src, "reasons": sorted(reasons),
-                "reason_samples": counts}
+                "power_w_max": max(x[2] for x in samples) if samples else None,
+                "samples": len(sm), "window_ms": 1e3 * (t1 - self.t0), "source": self.kind,
+                "reasons": sorted(reasons), "reason_samples": counts}
 
 
 def choose_bf16_peak(pk, clk):
@@ -281,7 +289,7 @@ class Timer:
         return sum(a.elapsed_time(b) for a, b in zip(self.s, self.e))
 
 
-def time_steps(fn, steps, warmup, flush=None, barrier=None):
+def time_steps(fn, steps, warmup, flush=None, barrier=None, on_timed=None):
     """Run warmup + timed steps; each timed step bracketed by events, with an
     L2 flush before it (outside the brackets).  Returns total ms."""
     import torch
@@ -292,6 +300,8 @@ def time_steps(fn, steps, warmup, flush=None, barrier=None):
     torch.cuda.synchronize()
     if barrier:
         barrier()
+    if on_timed is not None:
+        on_timed()
     t = Timer(steps)
     for i in range(steps):
         if flush is not None:
@@ -307,9 +317,8 @@ def time_steps(fn, steps, warmup, flush=None, barrier=None):
 
 def time_steps_clocked(fn, steps, warmup, device, flush=None, barrier=None):
     """time_steps with the SM clocks sampled over the timed steps."""
-    clocks = ClockSampler(device)
-    clocks.start()
-    ms = time_steps(fn, steps, warmup, flush=flush, barrier=barrier)
+    clocks = ClockSampler(device).launch()
+    ms = time_steps(fn, steps, warmup, flush=flush, barrier=barrier, on_timed=clocks.start)
     return ms, clocks.stop()
 
 
@@ -352,7 +361,7 @@ def run_ours(args):
             grads.all_reduce()
 
     flops = linear_flops(M, N, K, r)
-    clocks = ClockSampler(dev)
+    clocks = ClockSampler(dev).launch()
     for _ in range(max(args.warmup, 0)):
         flush()
         step()
