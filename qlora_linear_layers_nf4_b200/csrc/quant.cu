@@ -24,6 +24,18 @@ __device__ __forceinline__ float max_abs8(const float4& a, const float4& b) {
   return fmaxf(m, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
 }
 
+// Max of |x| over 8 values as the integer max of their magnitude bits: for
+// non-negative floats integer order is float order, and an Inf (0x7f800000)
+// or NaN (above it) is the largest, so one compare of the block max finds
+// every non-finite input.
+__device__ __forceinline__ uint32_t max_abs_bits8(const float4& a, const float4& b) {
+  const uint32_t m = 0x7fffffffu;
+  uint32_t r = max(max(__float_as_uint(a.x) & m, __float_as_uint(a.y) & m),
+                   max(__float_as_uint(a.z) & m, __float_as_uint(a.w) & m));
+  return max(r, max(max(__float_as_uint(b.x) & m, __float_as_uint(b.y) & m),
+                    max(__float_as_uint(b.z) & m, __float_as_uint(b.w) & m)));
+}
+
 __device__ __forceinline__ bool finite8(const float4& a, const float4& b) {
   return isfinite(a.x) && isfinite(a.y) && isfinite(a.z) && isfinite(a.w) && isfinite(b.x) &&
          isfinite(b.y) && isfinite(b.z) && isfinite(b.w);
@@ -171,18 +183,18 @@ __device__ __forceinline__ float load1(const void* w, int64_t e) {
 // stride apart, two words per step, and issues the next step's two loads
 // before encoding the current two, so 64 bytes per thread are always in
 // flight.
-template <int G, int IN>
+template <int G, int IN, typename Idx>
 __global__ void __launch_bounds__(256) quantize_vec_kernel(
-    const void* __restrict__ w, int64_t n_words, uint32_t* __restrict__ codes,
+    const void* __restrict__ w, Idx n_words, uint32_t* __restrict__ codes,
     float* __restrict__ absmax, uint32_t* __restrict__ status, float* __restrict__ max_slots) {
   __shared__ EncodeTables tab;
   init_tables(tab);
   __syncthreads();
-  float cta_max = 0.0f;
-  bool bad = false;
-  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  // Encode one word (8 elements) whose block max over the G lanes is known.
-  auto encode_word = [&](int64_t i, bool valid, const float4& a, const float4& b, float m) {
+  uint32_t cta_max = 0;
+  const Idx stride = Idx(gridDim.x) * blockDim.x;
+  // Encode one word (8 elements) whose block max over the G lanes is known
+  // (finite: a non-finite block was flagged and is left to the fallback).
+  auto encode_word = [&](Idx i, bool valid, const float4& a, const float4& b, float m) {
     if (!valid) return;
     uint32_t word;
     if (fast_scale(m)) {
@@ -197,38 +209,38 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
     if ((threadIdx.x & (G - 1)) == 0 && absmax != nullptr) absmax[i / G] = m;
   };
   const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  int64_t base = int64_t(blockIdx.x) * blockDim.x;
+  Idx base = Idx(blockIdx.x) * blockDim.x;
   float4 a0 = z4, b0 = z4, a1 = z4, b1 = z4;
   {
-    const int64_t i0 = base + threadIdx.x, i1 = i0 + stride;
-    if (i0 < n_words) load8<IN>(w, i0, a0, b0);
-    if (i1 < n_words) load8<IN>(w, i1, a1, b1);
+    const Idx i0 = base + threadIdx.x, i1 = i0 + stride;
+    if (i0 < n_words) load8<IN>(w, int64_t(i0), a0, b0);
+    if (i1 < n_words) load8<IN>(w, int64_t(i1), a1, b1);
   }
   // The loop runs in whole warps so every lane takes part in the shuffles.
   for (; base < n_words; base += 2 * stride) {
-    const int64_t i0 = base + threadIdx.x, i1 = i0 + stride;
-    const int64_t n0 = i0 + 2 * stride, n1 = n0 + stride;
+    const Idx i0 = base + threadIdx.x, i1 = i0 + stride;
+    const Idx n0 = i0 + 2 * stride, n1 = n0 + stride;
     float4 c0 = z4, d0 = z4, c1 = z4, d1 = z4;
-    if (n0 < n_words) load8<IN>(w, n0, c0, d0);
-    if (n1 < n_words) load8<IN>(w, n1, c1, d1);
+    if (n0 < n_words) load8<IN>(w, int64_t(n0), c0, d0);
+    if (n1 < n_words) load8<IN>(w, int64_t(n1), c1, d1);
     const bool v0 = i0 < n_words, v1 = i1 < n_words;
-    bad |= (v0 && !finite8(a0, b0)) || (v1 && !finite8(a1, b1));
-    float m0 = max_abs8(a0, b0), m1 = max_abs8(a1, b1);
+    uint32_t m0 = max_abs_bits8(a0, b0), m1 = max_abs_bits8(a1, b1);
 #pragma unroll
     for (int o = G / 2; o > 0; o >>= 1) {
-      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
-      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      m0 = max(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+      m1 = max(m1, __shfl_xor_sync(0xffffffffu, m1, o));
     }
-    encode_word(i0, v0, a0, b0, m0);
-    encode_word(i1, v1, a1, b1, m1);
-    cta_max = fmaxf(cta_max, fmaxf(m0, m1));
+    encode_word(i0, v0, a0, b0, __uint_as_float(m0));
+    encode_word(i1, v1, a1, b1, __uint_as_float(m1));
+    cta_max = max(cta_max, max(v0 ? m0 : 0u, v1 ? m1 : 0u));
     a0 = c0;
     b0 = d0;
     a1 = c1;
     b1 = d1;
   }
-  if (bad) report(status, NF4_ERR_NONFINITE);
-  if (max_slots != nullptr) cta_max_to_slot(cta_max, max_slots + blockIdx.x);
+  // a NaN or Inf anywhere makes its block's max bits >= 0x7f800000
+  if (cta_max >= 0x7f800000u) report(status, NF4_ERR_NONFINITE);
+  if (max_slots != nullptr) cta_max_to_slot(__uint_as_float(cta_max), max_slots + blockIdx.x);
   // let a programmatic dependent (the double-quant kernel) launch: only now,
   // so that its waiting CTAs never hold SM slots this grid still needs
   asm volatile("griddepcontrol.launch_dependents;");
@@ -540,20 +552,24 @@ void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes,
   if (n_full > 0 && vec) {
     const int64_t n_words = n_full * bs / 8;
     uint32_t* c32 = reinterpret_cast<uint32_t*>(codes);
-    auto run = [&](auto kernel) {
+    auto run = [&](auto kernel, auto n) {
       // one resident wave: every CTA stays for the whole pass
       const int grid = std::min(kMaxSlots - 1, grid_for(n_words, threads, sms,
                                                          resident_ctas(reinterpret_cast<const void*>(kernel), threads)));
-      kernel<<<grid, threads, 0, stream>>>(w, n_words, c32, absmax_out, status, max_slots);
+      kernel<<<grid, threads, 0, stream>>>(w, n, c32, absmax_out, status, max_slots);
       *n_slots = grid;
     };
+    // 32-bit word indices while every index the loop forms (up to n_words plus
+    // four grid strides) fits
+    const bool small = n_words < (int64_t(1) << 30);
+    const uint32_t n32 = uint32_t(n_words);
     switch (bs / 8) {
-      case 1: run(quantize_vec_kernel<1, IN>); break;
-      case 2: run(quantize_vec_kernel<2, IN>); break;
-      case 4: run(quantize_vec_kernel<4, IN>); break;
-      case 8: run(quantize_vec_kernel<8, IN>); break;
-      case 16: run(quantize_vec_kernel<16, IN>); break;
-      default: run(quantize_vec_kernel<32, IN>); break;
+      case 1: if (small) run(quantize_vec_kernel<1, IN, uint32_t>, n32); else run(quantize_vec_kernel<1, IN, int64_t>, n_words); break;
+      case 2: if (small) run(quantize_vec_kernel<2, IN, uint32_t>, n32); else run(quantize_vec_kernel<2, IN, int64_t>, n_words); break;
+      case 4: if (small) run(quantize_vec_kernel<4, IN, uint32_t>, n32); else run(quantize_vec_kernel<4, IN, int64_t>, n_words); break;
+      case 8: if (small) run(quantize_vec_kernel<8, IN, uint32_t>, n32); else run(quantize_vec_kernel<8, IN, int64_t>, n_words); break;
+      case 16: if (small) run(quantize_vec_kernel<16, IN, uint32_t>, n32); else run(quantize_vec_kernel<16, IN, int64_t>, n_words); break;
+      default: if (small) run(quantize_vec_kernel<32, IN, uint32_t>, n32); else run(quantize_vec_kernel<32, IN, int64_t>, n_words); break;
     }
     ++*launches;
   } else if (n_full > 0) {
