@@ -264,7 +264,8 @@ def dequantize(q: dict, out_dtype: str = "f32") -> np.ndarray:
     if out_dtype == "bf16":
         return bf16_round(w).reshape(q["shape"])
     if out_dtype == "f16":
-        return w.astype(np.float16)
+        with np.errstate(over="ignore"):   # beyond the f16 range: +-inf, as IEEE rounding gives
+            return w.astype(np.float16)
     raise ValueError(out_dtype)
 
 

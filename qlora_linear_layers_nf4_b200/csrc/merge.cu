@@ -185,10 +185,13 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
       uint8_t* stage = smem + (warp - 2) * 2 * kMgStageBytes;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        const int k = kh + 32 * c;
+        // Stop at the first piece past the last column (warp-uniform), so that
+        // every staged piece is stored and the wait below frees the right buffer.
+        if (k >= p.K) break;
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + half * 128 + c * 32, v);
         tmem_ld_wait();
-        const int k = kh + 32 * c;
         const float sc = scale[c >> 1];
         const uint32_t words[4] = {cw[c].x, cw[c].y, cw[c].z, cw[c].w};
         float m[32];
@@ -222,7 +225,7 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && k < p.K) {
+        if (lane == 0) {
           tma_store_2d(&tm_out, buf, k, n0 + quad * 32);   // rows past N are clipped by the map
           bulk_commit_group();
         }

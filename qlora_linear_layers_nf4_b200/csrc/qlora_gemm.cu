@@ -21,6 +21,7 @@
 //                              CTAs sum their fp32 partials through
 //                              distributed shared memory
 #include <algorithm>
+#include <mutex>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -353,10 +354,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       constexpr bool f16 = F16;
 #pragma unroll 1
       for (int c = 0; c < kTileN / 32; ++c) {
+        const int col0 = tile_n0 + c * 32;
+        // Stop at the first piece that lies wholly past the output (warp-uniform):
+        // every piece staged below is then stored, so waiting for all but the
+        // last store group frees the buffer the piece two back used.
+        if (col0 >= p.out_cols || row0 >= p.M) break;
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + half * kTileN + c * 32, v);
         tmem_ld_wait();
-        const int col0 = tile_n0 + c * 32;
         uint32_t packed[16];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -386,7 +391,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
               make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && col0 < p.out_cols && row0 < p.M) {
+        if (lane == 0) {
           tma_store_2d(&tm_out, buf, col0, row0);   // rows past M, columns past the end: clipped
           bulk_commit_group();
         }
@@ -712,10 +717,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       constexpr bool f16 = F16;
 #pragma unroll 1
       for (int c = 0; c < kTileN / 32; ++c) {
+        const int col0 = tile_n0 + c * 32;
+        if (col0 >= p.out_cols || row0 >= p.M) break;   // see the single-CTA epilogue
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + h * kTileN + c * 32, v);
         tmem_ld_wait();
-        const int col0 = tile_n0 + c * 32;
         uint32_t packed[16];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -746,7 +752,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
               make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && col0 < p.out_cols && row0 < p.M) {
+        if (lane == 0) {
           tma_store_2d(&tm_out, buf, col0, row0);   // rows past M, columns past the end: clipped
           bulk_commit_group();
         }
@@ -1006,6 +1012,43 @@ __global__ void __launch_bounds__(kAdThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
+
+// Per-device side stream at the highest priority with its fork and join
+// events (created on first use, re-created if the context that owned them is
+// gone).  Callers hold g_side_mu from the fork to the join.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  SideStream& ss = g_side[dev];
+  int prio = 0;
+  if (ss.stream != nullptr && cudaStreamGetPriority(ss.stream, &prio) != cudaSuccess) {
+    (void)cudaGetLastError();
+    ss = SideStream{};
+  }
+  if (ss.stream == nullptr) {
+    int least = 0, greatest = 0;
+    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, greatest);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      ss = SideStream{};
+      return e;
+    }
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -1397,9 +1440,37 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
     if (e != cudaSuccess) return e;
   }
   e = launch_adapter(lu, st, launches);
-  if (e == cudaSuccess) e = launch_adapter(ldb, st, launches);
+  if (e != cudaSuccess) return e;
+  if (a.dx == nullptr) {
+    e = launch_adapter(ldb, st, launches);
+    if (e == cudaSuccess) e = launch_adapter(lda, st, launches);
+    return e;
+  }
+  // dx on a high-priority side stream forked after U, dB and dA^T on the
+  // caller's stream: the block scheduler gives dx every SM it can use, and the
+  // two rank-r products (which dx does not need) run on the SMs its last,
+  // partial wave leaves idle.  The caller's stream then waits for dx.
+  SideStream* side = nullptr;
+  std::unique_lock<std::mutex> lock(g_side_mu);
+  if (side_stream(&side) != cudaSuccess) {
+    lock.unlock();
+    e = launch_adapter(ldb, st, launches);
+    if (e == cudaSuccess) e = launch_adapter(lda, st, launches);
+    if (e == cudaSuccess) e = launch_fused(ldx, st, launches);
+    return e;
+  }
+  e = cudaEventRecord(side->fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+  if (e != cudaSuccess) return e;
+  const cudaError_t ex = launch_fused(ldx, side->stream, launches);
+  e = launch_adapter(ldb, st, launches);
   if (e == cudaSuccess) e = launch_adapter(lda, st, launches);
-  if (e == cudaSuccess && a.dx != nullptr) e = launch_fused(ldx, st, launches);
+  // join even after a failed launch, so the caller's stream never runs ahead
+  // of work already on the side stream
+  cudaError_t ej = cudaEventRecord(side->join, side->stream);
+  if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, side->join, 0);
+  if (e == cudaSuccess) e = ex;
+  if (e == cudaSuccess) e = ej;
   return e;
 }
 

@@ -114,6 +114,34 @@ def test_ragged_shapes(cuda_device, m, n, k, rank, dq, bias):
         r.check_backward()
 
 
+@pytest.mark.parametrize("m,n,k,rank", [
+    (300, 264, 320, 16),    # dx tile: two stored 32-column pieces, then two past the edge
+    (257, 1032, 192, 24),   # dx tile: six stored pieces, then two past the edge
+    (520, 392, 320, 16),    # pair tiles with a ragged column tail
+])
+def test_ragged_tail_repeated(cuda_device, m, n, k, rank):
+    """Repeated backward calls give the same bits every time.
+
+    The epilogue stages each 32 x 32 output piece in one of two shared buffers
+    while an earlier piece's TMA store may still read the other; a tile whose
+    last pieces lie past the output must not reuse a buffer still being read.
+    Such a race only shows under some timings, so the backward runs many times
+    (its kernels are deterministic) and every result must equal the first,
+    which is itself checked against the oracle.
+    """
+    import torch
+    Q = _Q()
+    case = WL.LinearCase(f"tail {m}x{n}x{k}", n=n, k=k, m=m, r=rank, alpha=2.0 * rank,
+                         seed=3000 + m + k, double_quant=True)
+    r = Run(case, cuda_device)
+    r.check_backward()
+    ws = Q.Workspace(cuda_device)
+    for _ in range(24):
+        dA, dB, dx = Q.linear_bwd(r.q, r.x, r.A, r.B, case.alpha, r.dy, t=r.T, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(dx, r.dx) and torch.equal(dA, r.dA) and torch.equal(dB, r.dB)
+
+
 def test_recomputed_t_matches(cuda_device):
     import torch
     case = WL.LinearCase("recompute t", n=512, k=512, m=200, r=32, alpha=64.0, seed=77)
