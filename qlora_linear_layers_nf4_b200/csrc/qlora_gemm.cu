@@ -1041,7 +1041,10 @@ cudaError_t side_stream(SideStream** out) {
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, greatest);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
-    if (e != cudaSuccess) {
+    if (e != cudaSuccess) {   // release whatever was made; the next call tries again
+      if (ss.join != nullptr) (void)cudaEventDestroy(ss.join);
+      if (ss.fork != nullptr) (void)cudaEventDestroy(ss.fork);
+      if (ss.stream != nullptr) (void)cudaStreamDestroy(ss.stream);
       ss = SideStream{};
       return e;
     }

@@ -179,16 +179,20 @@ def test_wait_check_host_validation():
 
 
 def test_bucket_encoding_conditions():
-    # The quantize kernel's fast encode indexes 64 buckets of width 1/32 over
-    # [-1, 1] and compares with the single threshold inside the bucket.  It is
-    # exact only if no bucket holds two thresholds and no threshold lies
-    # within the index rounding (2^-24) of a bucket edge.
+    # The quantize kernel's fast encode rounds 32 v + 32 to the nearest integer
+    # i (one fused multiply-add, exact before its one rounding), so bucket i of
+    # 65 covers [(i - 32.5) / 32, (i - 31.5) / 32) over v in [-1, 1], and
+    # compares v with the single threshold that may lie inside the bucket.  It
+    # is exact only if no bucket holds two thresholds and no threshold sits on
+    # a bucket edge, where a tie could pick the neighbouring bucket.
     _, th = Q.codebook()
     th = np.array(th, dtype=np.float64)
-    edges = np.arange(65) / 32.0 - 1.0
-    assert np.min(np.abs(th[:, None] - edges[None, :])) > 2.0 ** -20
-    counts = [np.sum((th >= edges[j]) & (th < edges[j] + 1 / 32)) for j in range(64)]
+    edges = (np.arange(66) - 32.5) / 32.0
+    assert edges[0] < -1.0 and edges[-1] > 1.0
+    assert np.min(np.abs(th[:, None] - edges[None, :])) > 2e-4
+    counts = [np.sum((th >= edges[j]) & (th < edges[j + 1])) for j in range(65)]
     assert max(counts) <= 1
+    assert sum(counts) == 15
 
 
 def test_sharded_double_quant_host_validation():
