@@ -104,6 +104,11 @@ cudaEvent_t prof_event() {
 namespace nf4 {
 void add_launches(int n) { g_launches += n; }
 
+bool prof_on() {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  return g_prof_on;
+}
+
 void prof_mark(cudaStream_t stream, int kernel_id, bool after) {
   std::lock_guard<std::mutex> lock(g_prof_mu);
   if (!g_prof_on) return;

@@ -137,6 +137,10 @@ enum KernelId {
 
 // When profiling is on, record an event on `stream` before / after a launch.
 void prof_mark(cudaStream_t stream, int kernel_id, bool after);
+// Whether per-kernel event profiling is on.  A launch that would otherwise
+// overlap the kernel before it (programmatic dependent launch) runs fully
+// serialised then, so each bracket times one kernel alone.
+bool prof_on();
 
 }  // namespace nf4
 

@@ -244,6 +244,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
               tma_load_2d(stage_c(s) + g * 2048, &tm_codes, &sh->full[s], (tile_n0 + 64 * g) / 2, k0);
           }
         } else {
+          if (it == p.main_steps) grid_dep_wait();
           const int r0 = (it - p.main_steps) * kTileK;
           mbar_arrive_expect_tx(&sh->full[s], kABytes + kBBytes);
           tma_load_2d(a, &tm_a2, &sh->full[s], r0, m0);
@@ -552,6 +553,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
           if (rank == 0 && a_part == 0) mbar_arrive_expect_tx(&sh->afull[s], 2 * kP2ABytes);
           tma_load_2d_pair(a, &tm_a, afull_leader, kstep(it) * kTileK, m0 + 256 * int(rank) + arow);
         } else {
+          if (it == p.main_steps) grid_dep_wait();
           const int r0 = (it - p.main_steps) * kTileK;
           if (rank == 0 && a_part == 0) mbar_arrive_expect_tx(&sh->afull[s], 2 * (kP2ABytes + kP2BBytes));
           tma_load_2d_pair(a, &tm_a2, afull_leader, r0, m0 + 256 * int(rank) + arow);
@@ -860,6 +862,7 @@ __global__ void __launch_bounds__(kAdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
+  grid_dep_launch();
 
   // TMA copies: the A tile from warp 0 and the B tile from warp 2 (one warp
   // keeps only a few TMA copies going per microsecond); each arrives on the
@@ -1303,29 +1306,48 @@ bool prepare_fused(const LinearArgs& a, int mode, const __nv_bfloat16* a2, Fused
   return true;
 }
 
-cudaError_t launch_fused(const FusedLaunch& L, cudaStream_t st, int* launches) {
-  const dim3 grid = L.grid;
+// pdl: launch as a programmatic dependent of the kernel before it on the
+// stream (which must be the producer of A2 and call grid_dep_launch); the
+// kernel reads A2 only after grid_dep_wait.
+template <typename K>
+cudaError_t launch_fused_kernel(K kernel, const FusedLaunch& L, unsigned threads, size_t smem,
+                                cudaStream_t st, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = L.grid;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
+}
+
+cudaError_t launch_fused(const FusedLaunch& L, cudaStream_t st, int* launches, bool pdl = false) {
   const int id = L.mode == kFwd ? kKFusedFwd : kKFusedDx;
   NF4_PROF_BEGIN(st, id);
+  cudaError_t e;
   if (L.pair) {
-    if (L.mode == kFwd) {
-      if (L.f16) fused_nf4_gemm_pair<kFwd, true><<<grid, kP2Threads, kP2Smem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
-      else fused_nf4_gemm_pair<kFwd, false><<<grid, kP2Threads, kP2Smem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
-    } else {
-      if (L.f16) fused_nf4_gemm_pair<kDx, true><<<grid, kP2Threads, kP2Smem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
-      else fused_nf4_gemm_pair<kDx, false><<<grid, kP2Threads, kP2Smem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
-    }
+    const unsigned t = kP2Threads;
+    if (L.mode == kFwd)
+      e = L.f16 ? launch_fused_kernel(fused_nf4_gemm_pair<kFwd, true>, L, t, kP2Smem, st, pdl)
+                : launch_fused_kernel(fused_nf4_gemm_pair<kFwd, false>, L, t, kP2Smem, st, pdl);
+    else
+      e = L.f16 ? launch_fused_kernel(fused_nf4_gemm_pair<kDx, true>, L, t, kP2Smem, st, pdl)
+                : launch_fused_kernel(fused_nf4_gemm_pair<kDx, false>, L, t, kP2Smem, st, pdl);
   } else {
-    if (L.mode == kFwd) {
-      if (L.f16) fused_nf4_gemm<kFwd, true><<<grid, kFusedThreads, kFusedSmem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
-      else fused_nf4_gemm<kFwd, false><<<grid, kFusedThreads, kFusedSmem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
-    } else {
-      if (L.f16) fused_nf4_gemm<kDx, true><<<grid, kFusedThreads, kFusedSmem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
-      else fused_nf4_gemm<kDx, false><<<grid, kFusedThreads, kFusedSmem, st>>>(L.ta, L.ta2, L.tb2, L.tc, L.to, L.p);
-    }
+    const unsigned t = kFusedThreads;
+    if (L.mode == kFwd)
+      e = L.f16 ? launch_fused_kernel(fused_nf4_gemm<kFwd, true>, L, t, kFusedSmem, st, pdl)
+                : launch_fused_kernel(fused_nf4_gemm<kFwd, false>, L, t, kFusedSmem, st, pdl);
+    else
+      e = L.f16 ? launch_fused_kernel(fused_nf4_gemm<kDx, true>, L, t, kFusedSmem, st, pdl)
+                : launch_fused_kernel(fused_nf4_gemm<kDx, false>, L, t, kFusedSmem, st, pdl);
   }
   NF4_PROF_END(st, id);
-  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) ++*launches;
   return e;
 }
@@ -1394,7 +1416,7 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
     return cudaErrorInvalidValue;
   e = launch_adapter(lt, st, launches);
   if (e != cudaSuccess) return e;
-  return launch_fused(lf, st, launches);
+  return launch_fused(lf, st, launches, /*pdl=*/!prof_on());
 }
 
 cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches) {

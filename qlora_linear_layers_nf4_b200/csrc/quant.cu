@@ -19,11 +19,6 @@ namespace nf4 {
 
 namespace {
 
-__device__ __forceinline__ float max_abs8(const float4& a, const float4& b) {
-  float m = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
-  return fmaxf(m, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
-}
-
 // Max of |x| over 8 values as the integer max of their magnitude bits: for
 // non-negative floats integer order is float order, and an Inf (0x7f800000)
 // or NaN (above it) is the largest, so one compare of the block max finds
@@ -34,11 +29,6 @@ __device__ __forceinline__ uint32_t max_abs_bits8(const float4& a, const float4&
                    max(__float_as_uint(a.z) & m, __float_as_uint(a.w) & m));
   return max(r, max(max(__float_as_uint(b.x) & m, __float_as_uint(b.y) & m),
                     max(__float_as_uint(b.z) & m, __float_as_uint(b.w) & m)));
-}
-
-__device__ __forceinline__ bool finite8(const float4& a, const float4& b) {
-  return isfinite(a.x) && isfinite(a.y) && isfinite(a.z) && isfinite(a.w) && isfinite(b.x) &&
-         isfinite(b.y) && isfinite(b.z) && isfinite(b.w);
 }
 
 // Fast encode.  v = RN(w / a) is formed without a division: y = RN(1/a) once

@@ -154,6 +154,18 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Programmatic dependent launch.  grid_dep_launch: this CTA no longer holds
+// back the next kernel on the stream (if that kernel was launched as a
+// programmatic dependent).  grid_dep_wait: block until every prerequisite
+// grid has completed and its memory operations are visible; a no-op in a
+// kernel that was launched without the attribute.
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Orders this thread's earlier shared::cluster stores before its later
 // operations, for observers anywhere in the cluster.
 __device__ __forceinline__ void fence_cluster() {
