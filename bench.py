@@ -744,24 +744,57 @@ def measure_rows(args, dev, flush, pk, pk_kind, barrier):
     del outs_m, qm
     torch.cuda.empty_cache()
 
-    # ---- the seven targets of one decoder block, fwd + bwd each (long kernels: eager)
+    # ---- the seven targets of one decoder block, fwd + bwd each (long kernels: eager).
+    # The block's forward runs its targets in layer order and its backward in
+    # reverse; q, k, v (which read the same activations) and gate, up are
+    # independent of one another, so each group runs on parallel streams, as
+    # a training step schedules them.  Every target has its own workspace.
     if not args.no_block:
         ws_q = Q.Workspace(dev)
-        layers = []
+        layers = {}
         for case in WL.BLOCK:
             inp = WL.draw_linear(case)
             qb = Q.quantize(torch.from_numpy(inp.w).to(dev), 64, True, workspace=ws_q)
             x, A, B, dy = (bf16_dev(v, dev) for v in (inp.x, inp.a, inp.b, inp.dy))
-            layers.append((case, qb, x, A, B, dy,
-                           torch.empty((case.m, case.n), dtype=torch.bfloat16, device=dev),
-                           torch.empty((case.m, case.r), dtype=torch.bfloat16, device=dev),
-                           torch.empty((case.m, case.k), dtype=torch.bfloat16, device=dev)))
-        wsb = Q.Workspace(dev)
+            layers[case.name.split()[1]] = (
+                case, qb, x, A, B, dy,
+                torch.empty((case.m, case.n), dtype=torch.bfloat16, device=dev),
+                torch.empty((case.m, case.r), dtype=torch.bfloat16, device=dev),
+                torch.empty((case.m, case.k), dtype=torch.bfloat16, device=dev),
+                Q.Workspace(dev))
+        groups = [["q_proj", "k_proj", "v_proj"], ["o_proj"], ["gate_proj", "up_proj"], ["down_proj"]]
+        assert sorted(n for g in groups for n in g) == sorted(layers)
+        side = [torch.cuda.Stream(device=dev) for _ in range(3)]
+
+        def fwd(name):
+            case, qb, x, A, B, dy, y, T, dx, wsl = layers[name]
+            Q.linear_fwd(qb, x, A, B, case.alpha, out=y, t_out=T, workspace=wsl)
+
+        def bwd(name):
+            case, qb, x, A, B, dy, y, T, dx, wsl = layers[name]
+            Q.linear_bwd(qb, x, A, B, case.alpha, dy, t=T, dx=dx, workspace=wsl)
+
+        def run_group(fn, group):
+            if len(group) == 1:
+                fn(group[0])
+                return
+            main = torch.cuda.current_stream()
+            start = torch.cuda.Event()
+            start.record(main)
+            for st, name in zip(side, group):
+                st.wait_event(start)
+                with torch.cuda.stream(st):
+                    fn(name)
+            for st in side[:len(group)]:
+                done = torch.cuda.Event()
+                done.record(st)
+                main.wait_event(done)
 
         def block_step():
-            for case, qb, x, A, B, dy, y, T, dx in layers:
-                Q.linear_fwd(qb, x, A, B, case.alpha, out=y, t_out=T, workspace=wsb)
-                Q.linear_bwd(qb, x, A, B, case.alpha, dy, t=T, dx=dx, workspace=wsb)
+            for g in groups:
+                run_group(fwd, g)
+            for g in reversed(groups):
+                run_group(bwd, g)
 
         flops = sum(linear_flops(c.m, c.n, c.k, c.r) for c in WL.BLOCK)
         bsteps = max(3, min(args.steps, 10))
@@ -771,7 +804,8 @@ def measure_rows(args, dev, flush, pk, pk_kind, barrier):
         out["decoder_block_7_targets_fwd_bwd"] = {
             "TFLOP/s": tf, "ms_per_block": ms / bsteps, "flops": flops, "frac_peak": tf / peak,
             "peak": peak, "peak_source": f"{pk_kind} {peak_name}: {why}",
-            "method": "eager steps, L2 flushed before each"}
+            "method": "eager steps, L2 flushed before each; forward in layer order, backward in reverse; "
+                      "q/k/v and gate/up on parallel streams"}
     return out
 
 

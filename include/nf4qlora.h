@@ -339,11 +339,12 @@ NF4_API nf4_status qlora_linear_fwd(const nf4_weight* w, const void* x, int64_t 
  * T written by the forward's t_out, or NULL to recompute it.
  *   workspace      >= nf4_workspace_bytes(NF4_OP_LINEAR_BWD, M, N, K, r, 64, dq).
  * Streams: with BF16 / F16 and dx given, dx runs on a high-priority stream the
- * library keeps per device (made on the first such call), forked from `stream`
- * after U and joined back with events before the call returns, so work the
- * caller enqueues on `stream` afterwards sees every output; `stream` must
- * belong to the current device.  Calls from several host threads on one
- * device serialise on a lock while they enqueue.
+ * library keeps per device and calling stream (made on the first such call;
+ * up to 8 calling streams per device have their own, more share them), forked
+ * from `stream` after U and joined back with events before the call returns,
+ * so work the caller enqueues on `stream` afterwards sees every output;
+ * `stream` must belong to the current device.  Calls from several host
+ * threads serialise on a lock while they enqueue.
  */
 NF4_API nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const void* A,
                             const void* B, int r, float alpha, int compute_dtype,

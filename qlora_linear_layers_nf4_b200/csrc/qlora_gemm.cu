@@ -1016,27 +1016,41 @@ __global__ void __launch_bounds__(kAdThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
-// Per-device side stream at the highest priority with its fork and join
-// events (created on first use, re-created if the context that owned them is
-// gone).  Callers hold g_side_mu from the fork to the join.
+// High-priority side streams with their fork and join events, per device and
+// per calling stream (up to kSideSlots calling streams each; more share the
+// slots round robin, which only serialises their side work).  Created on
+// first use, re-created if the context that owned them is gone.  Callers hold
+// g_side_mu from the fork to the join.
 struct SideStream {
+  cudaStream_t owner = nullptr;   // the calling stream this slot serves
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr;
   cudaEvent_t join = nullptr;
 };
+constexpr int kSideSlots = 8;
 std::mutex g_side_mu;
-SideStream g_side[64];
+SideStream g_side[64][kSideSlots];
+int g_side_next[64];
 
-cudaError_t side_stream(SideStream** out) {
+cudaError_t side_stream(cudaStream_t caller, SideStream** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  SideStream& ss = g_side[dev];
+  SideStream* slots = g_side[dev];
+  int pick = -1;
+  for (int i = 0; i < kSideSlots && pick < 0; ++i)
+    if (slots[i].stream != nullptr && slots[i].owner == caller) pick = i;
+  for (int i = 0; i < kSideSlots && pick < 0; ++i)
+    if (slots[i].stream == nullptr) pick = i;
+  if (pick < 0) pick = g_side_next[dev]++ % kSideSlots;
+  SideStream& ss = slots[pick];
+  ss.owner = caller;
   int prio = 0;
   if (ss.stream != nullptr && cudaStreamGetPriority(ss.stream, &prio) != cudaSuccess) {
     (void)cudaGetLastError();
     ss = SideStream{};
+    ss.owner = caller;
   }
   if (ss.stream == nullptr) {
     int least = 0, greatest = 0;
@@ -1477,7 +1491,7 @@ cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t st, int
   // partial wave leaves idle.  The caller's stream then waits for dx.
   SideStream* side = nullptr;
   std::unique_lock<std::mutex> lock(g_side_mu);
-  if (side_stream(&side) != cudaSuccess) {
+  if (side_stream(st, &side) != cudaSuccess) {
     lock.unlock();
     e = launch_adapter(ldb, st, launches);
     if (e == cudaSuccess) e = launch_adapter(lda, st, launches);

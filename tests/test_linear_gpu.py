@@ -142,6 +142,31 @@ def test_ragged_tail_repeated(cuda_device, m, n, k, rank):
         assert torch.equal(dx, r.dx) and torch.equal(dA, r.dA) and torch.equal(dB, r.dB)
 
 
+def test_backward_on_parallel_streams(cuda_device):
+    """Backward calls from three streams at once (each with its own workspace)
+    give the bits of the same calls made one after another: each calling
+    stream forks dx onto its own side stream and joins it back."""
+    import torch
+    Q = _Q()
+    runs = [Run(WL.LinearCase(f"streams {i}", n=1024 + 256 * i, k=768, m=600, r=32, alpha=64.0,
+                              seed=4100 + i), cuda_device) for i in range(3)]
+    for r in runs:
+        r.check_backward()
+    streams = [torch.cuda.Stream(device=cuda_device) for _ in runs]
+    wss = [Q.Workspace(cuda_device) for _ in runs]
+    outs = [None] * len(runs)
+    torch.cuda.synchronize()
+    for _ in range(4):
+        for i, (r, st) in enumerate(zip(runs, streams)):
+            with torch.cuda.stream(st):
+                outs[i] = Q.linear_bwd(r.q, r.x, r.A, r.B, r.case.alpha, r.dy, t=r.T, workspace=wss[i])
+        torch.cuda.synchronize()
+        for r, (dA, dB, dx) in zip(runs, outs):
+            assert torch.equal(dx, r.dx) and torch.equal(dA, r.dA) and torch.equal(dB, r.dB)
+    for ws in wss:
+        assert ws.read_status() == 0
+
+
 def test_recomputed_t_matches(cuda_device):
     import torch
     case = WL.LinearCase("recompute t", n=512, k=512, m=200, r=32, alpha=64.0, seed=77)
