@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the hash of the kernel source it was taken on; reported as null once the
 # source changes.
 NCU_TRAFFIC = {
-    # forward 124.3 MB, dx 178.8 MB per launch
-    "f29217272332d356": {"fwd": 124_325_632, "dx": 178_798_080},
+    # forward 125.3 MB, dx 178.7 MB per launch
+    "5658984bc2757e50": {"fwd": 69_511_424 + 55_790_080, "dx": 159_868_928 + 18_873_600},
 }
 
 
