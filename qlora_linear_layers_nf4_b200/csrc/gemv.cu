@@ -81,7 +81,8 @@ struct GemvParams {
 //   bs     [128 W rows][r] bf16 (this tile's rows of B)
 //   scales [128 rows][kGvMaxBlocks] fp32                 8 KB
 //   recv   [slice][128 / S rows][NP] fp32: partials pushed by the cluster
-//   tpart  [r_pad][NP] fp32: this slice's x A^T
+//   tpart  [t_parts][r_pad][NP] fp32: this slice's x A^T, in t_parts partial
+//          sums over interleaved K blocks
 //   red    [block phase - 1][128][NP] fp32: in-CTA partials (over codes and
 //          xs once they are consumed, when they are large enough)
 //   bars   [G] TMA groups, B tile, recv
@@ -91,7 +92,8 @@ struct GemvLayout {
 
 __host__ __device__ constexpr size_t align1k(size_t v) { return (v + 1023) & ~size_t(1023); }
 
-__host__ __device__ inline GemvLayout gemv_layout(int bps, int np, int r_pad, int r, int phases) {
+__host__ __device__ inline GemvLayout gemv_layout(int bps, int np, int r_pad, int r, int phases,
+                                                  int t_parts) {
   const int groups = (bps + kGvGroup - 1) / kGvGroup;
   const int blocks = groups * kGvGroup;
   GemvLayout L{};
@@ -102,7 +104,7 @@ __host__ __device__ inline GemvLayout gemv_layout(int bps, int np, int r_pad, in
   L.scales = align1k(L.bs + size_t(kGvRows) * r * 2);
   L.recv = align1k(L.scales + size_t(kGvRows) * kGvMaxBlocks * 4);
   L.tpart = L.recv + size_t(kGvRows) * np * 4;
-  size_t end = align1k(L.tpart + size_t(r_pad) * np * 4);
+  size_t end = align1k(L.tpart + size_t(t_parts) * r_pad * np * 4);
   const size_t red_bytes = size_t(phases - 1) * kGvRows * np * 4;
   if (red_bytes <= L.as - L.codes) {
     L.red = L.codes;
@@ -200,7 +202,8 @@ __device__ __forceinline__ void frag_pair(const uint4& lo, const uint4& hi, int 
 // MMA row g + 8 is W row 2g + 1.  In a half-warp the four rows a code load
 // touches then differ in bits 1..2 of the row, which the 128-byte swizzle
 // turns into four different 32-byte bank groups: the loads are conflict-free.
-template <int NT8, int RG, bool F16>
+// TP: the x A^T of a slice as TP partial sums over interleaved K blocks (1, 2 or 4).
+template <int NT8, int RG, bool F16, int TP>
 __global__ void __launch_bounds__(kGvThreads, 1)
     nf4_gemv(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
              const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -211,7 +214,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(1024) uint32_t lut[256 * 32];      // [entry][lane] copies
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const GemvLayout L = gemv_layout(p.blocks_per_slice, NP, p.r_pad, p.r, kPhases);
+  const GemvLayout L = gemv_layout(p.blocks_per_slice, NP, p.r_pad, p.r, kPhases, TP);
   uint8_t* codes = smem + L.codes;
   uint8_t* xs = smem + L.xs;
   uint8_t* as = smem + L.as;
@@ -219,6 +222,15 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   float* scales = reinterpret_cast<float*>(smem + L.scales);
   float* recv = reinterpret_cast<float*>(smem + L.recv);
   float* tpart = reinterpret_cast<float*>(smem + L.tpart);
+  // x A^T partial sums: r_pad / 16 row groups times t_parts K-block parts
+  // over the four adapter warps (r_pad / 16 * t_parts <= 4)
+  constexpr int t_parts = TP;
+  const int t_stride = p.r_pad * NP;
+  auto t_sum = [&](int i) {   // the parts of entry i, summed in part order
+    float v = tpart[i];
+    for (int k = 1; k < t_parts; ++k) v += tpart[k * t_stride + i];
+    return v;
+  };
   float* red = reinterpret_cast<float*>(smem + L.red);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);   // [group], B rows, recv
   uint64_t* bar_b = &bar[kGvMaxGroups];
@@ -409,13 +421,18 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       }
     }
   } else {
-    // ---- adapter rows j0 + g and j0 + g + 8 of x A^T over this K slice
-    const int j0 = (warp - kGvWWarps) * 16;
-    if (j0 < p.r) {
+    // ---- adapter rows j0 + g and j0 + g + 8 of x A^T over the K blocks
+    // part, part + parts, ... of this slice: the four adapter warps split the
+    // r_pad / 16 row groups and, when there are fewer than four, the K
+    // blocks, so no single warp walks every block alone.
+    const int aw = warp - kGvWWarps;
+    const int j0 = (aw / t_parts) * 16;
+    const int part = aw % t_parts;
+    if (j0 < p.r_pad) {
       float ta[NT8][4];
 #pragma unroll
       for (int t = 0; t < NT8; ++t) ta[t][0] = ta[t][1] = ta[t][2] = ta[t][3] = 0.0f;
-      for (int b = 0; b < nblk; ++b) {
+      for (int b = part; b < nblk; b += t_parts) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[b / kGvGroup], 0, &abort_flag, p.status));
         if (!ok) break;
         const uint8_t* at = as + b * abytes;
@@ -441,12 +458,13 @@ __global__ void __launch_bounds__(kGvThreads, 1)
           }
         }
       }
+      float* tp = tpart + part * t_stride;
 #pragma unroll
       for (int t = 0; t < NT8; ++t) {
-        tpart[(j0 + g) * NP + 8 * t + 2 * q] = ta[t][0];
-        tpart[(j0 + g) * NP + 8 * t + 2 * q + 1] = ta[t][1];
-        tpart[(j0 + g + 8) * NP + 8 * t + 2 * q] = ta[t][2];
-        tpart[(j0 + g + 8) * NP + 8 * t + 2 * q + 1] = ta[t][3];
+        tp[(j0 + g) * NP + 8 * t + 2 * q] = ta[t][0];
+        tp[(j0 + g) * NP + 8 * t + 2 * q + 1] = ta[t][1];
+        tp[(j0 + g + 8) * NP + 8 * t + 2 * q] = ta[t][2];
+        tp[(j0 + g + 8) * NP + 8 * t + 2 * q + 1] = ta[t][3];
       }
     }
   }
@@ -497,8 +515,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         for (int t = 0; t < NT8; ++t) {
           const int m = 8 * t + g;
           const int ja = j0 + 2 * q, jb = j0 + 2 * q + 8;
-          tfr[t][0] = pack2_rn<F16>(p.s * tpart[ja * NP + m], p.s * tpart[(ja + 1) * NP + m]);
-          tfr[t][1] = pack2_rn<F16>(p.s * tpart[jb * NP + m], p.s * tpart[(jb + 1) * NP + m]);
+          tfr[t][0] = pack2_rn<F16>(p.s * t_sum(ja * NP + m), p.s * t_sum((ja + 1) * NP + m));
+          tfr[t][1] = pack2_rn<F16>(p.s * t_sum(jb * NP + m), p.s * t_sum((jb + 1) * NP + m));
         }
         // B columns j >= r hold no adapter: masked to 0 (tpart rows r .. r_pad-1
         // are 0 too, from the zero-filled A rows)
@@ -562,7 +580,12 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         const int m = i / p.r, j = i % p.r;
         const uint32_t off = uint32_t((j * NP + m) * 4);
         float v = 0.0f;
-        for (int sl = 0; sl < S; ++sl) v += ld_shared_cluster_f32(mapa_shared(tbase + off, uint32_t(sl)));
+        for (int sl = 0; sl < S; ++sl) {
+          float vs = ld_shared_cluster_f32(mapa_shared(tbase + off, uint32_t(sl)));
+          for (int k = 1; k < t_parts; ++k)
+            vs += ld_shared_cluster_f32(mapa_shared(tbase + off + uint32_t(k * t_stride * 4), uint32_t(sl)));
+          v += vs;
+        }
         p.t_out[i] = from_f32<F16>(p.s * v);
       }
     }
@@ -587,12 +610,19 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   const int phases = kGvWWarps / (8 / rg);
   const int np = 8 * nt8;
   const int r_pad = (a.r + 15) / 16 * 16;
+  // With at most 8 tokens and one or two adapter row groups, the x A^T of a
+  // slice is split over the four adapter warps by K block as well, so it
+  // finishes with the weight rows (more tokens keep the W warps busier).
+  const int t_groups = r_pad / 16;
+  const int t_parts = (nt8 == 1 && t_groups <= 2) ? 4 / t_groups : 1;
   // K slices: one wave of one CTA per SM where possible, and everything a CTA
   // reads fits in its shared memory at once.
   int slices = 1;
   while (slices < kGvMaxSlices && tiles * slices * 2 <= 148 && slices * 2 <= kb) slices *= 2;
   int bps = (kb + slices - 1) / slices;
-  auto fits = [&](int b) { return b <= kGvMaxBlocks && gemv_layout(b, np, r_pad, a.r, phases).total <= kGvMaxDynSmem; };
+  auto fits = [&](int b) {
+    return b <= kGvMaxBlocks && gemv_layout(b, np, r_pad, a.r, phases, t_parts).total <= kGvMaxDynSmem;
+  };
   while (!fits(bps) && slices < kGvMaxSlices) {
     slices *= 2;
     bps = (kb + slices - 1) / slices;
@@ -632,7 +662,7 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   p.t_out = static_cast<__nv_bfloat16*>(a.t_out);
   p.status = a.status;
 
-  const size_t smem = gemv_layout(bps, np, r_pad, a.r, phases).total;
+  const size_t smem = gemv_layout(bps, np, r_pad, a.r, phases, t_parts).total;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(tiles), unsigned(slices), 1);
   cfg.blockDim = dim3(kGvThreads, 1, 1);
@@ -651,13 +681,19 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   cfg.numAttrs = 2;
   // The shared-memory opt-in is set once per instantiation (the maximum the
   // decode path can ask for), not on every call.
-  auto kernel_for = [](int n8, bool f16) {
-    if (f16) return n8 == 1 ? nf4_gemv<1, 2, true> : (n8 == 2 ? nf4_gemv<2, 2, true> : nf4_gemv<4, 1, true>);
-    return n8 == 1 ? nf4_gemv<1, 2, false> : (n8 == 2 ? nf4_gemv<2, 2, false> : nf4_gemv<4, 1, false>);
+  auto kernel_for = [](int n8, bool f16, int tp) {
+    if (f16) {
+      if (n8 == 1) return tp == 4 ? nf4_gemv<1, 2, true, 4> : (tp == 2 ? nf4_gemv<1, 2, true, 2> : nf4_gemv<1, 2, true, 1>);
+      return n8 == 2 ? nf4_gemv<2, 2, true, 1> : nf4_gemv<4, 1, true, 1>;
+    }
+    if (n8 == 1) return tp == 4 ? nf4_gemv<1, 2, false, 4> : (tp == 2 ? nf4_gemv<1, 2, false, 2> : nf4_gemv<1, 2, false, 1>);
+    return n8 == 2 ? nf4_gemv<2, 2, false, 1> : nf4_gemv<4, 1, false, 1>;
   };
-  static PerDeviceOnce attr_done[6];
-  const int slot = (nt8 == 1 ? 0 : (nt8 == 2 ? 1 : 2)) + (a.f16 ? 3 : 0);
-  auto* kernel = kernel_for(nt8, a.f16 != 0);
+  // one slot per instantiation: (tokens, parts) in {(8, 4), (8, 2), (8, 1), (16, 1), (32, 1)} x dtype
+  static PerDeviceOnce attr_done[10];
+  const int kind = nt8 == 1 ? (t_parts == 4 ? 0 : (t_parts == 2 ? 1 : 2)) : (nt8 == 2 ? 3 : 4);
+  const int slot = kind + (a.f16 ? 5 : 0);
+  auto* kernel = kernel_for(nt8, a.f16 != 0, t_parts);
   cudaError_t e = cudaSuccess;
   const int dev = PerDeviceOnce::current();
   if (!attr_done[slot].done(dev)) {

@@ -187,10 +187,14 @@ def test_decode_shapes(cuda_device, case):
 
 # Decode with 17..32 tokens takes the widest decode instantiation (four 8-token
 # MMA column groups); r = 8 and r = 64 are the smallest and largest adapter the
-# decode kernel takes in one K step of its adapter warps.
+# decode kernel takes in one K step of its adapter warps.  With at most 8 tokens
+# the x A^T of a slice is split over the adapter warps by K block: four parts
+# for one 16-row adapter group (r <= 16), two for two (r = 24, 32), none for
+# three or four (r = 48, 64).
 @pytest.mark.parametrize("m,rank,dq", [
     (17, 16, True), (24, 16, True), (32, 16, True), (32, 16, False),
     (5, 8, True), (32, 8, True), (9, 64, True), (32, 64, False),
+    (4, 32, True), (8, 24, False), (3, 48, True), (1, 64, True),
 ])
 def test_decode_wide_and_rank_edges(cuda_device, m, rank, dq):
     case = WL.LinearCase(f"decode 4096x4096 M={m} r={rank}", n=4096, k=4096, m=m, r=rank,
