@@ -299,8 +299,10 @@ NF4_API nf4_status nf4_dequantize(const nf4_weight* w, int out_dtype, void* out,
  *   y = x W'^T + s (x A^T) B^T (+ bias),  s = alpha / r,
  * W' the dequantized base rounded to compute_dtype, operands in
  * compute_dtype, fp32 accumulation, y rounded to compute_dtype.
- *   w              N = w->rows (out), K = w->cols (in); block_size 64;
- *                  K % 64 == 0, N % 8 == 0.
+ *   w              N = w->rows (out), K = w->cols (in); block_size a power
+ *                  of two from 64 to 4096 (others: NF4_ERR_UNSUPPORTED);
+ *                  K % 64 == 0, N % 8 == 0.  Blocks run over the flattened
+ *                  weight, so K need not be a multiple of the block size.
  *   x              [M, K] compute_dtype; M >= 1.
  *   A, B           [r, K] and [N, r] compute_dtype; 8 <= r <= 256, r % 8 == 0.
  *   compute_dtype  NF4_BF16, NF4_F16 or NF4_F32.  NF4_F32 is the pages'
@@ -358,11 +360,13 @@ NF4_API nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t 
  * equation 6.3.6 -- the merged weight stays in BF16, it is not requantized):
  *   out[n, k] = w'[n, k] + s (B A)[n, k],  s = alpha / r,
  * w' = fp32(L[code] * scale) the fp32 dequant, B A accumulated in fp32, the sum
- * rounded once to fp32 (one FMA) and then, for NF4_BF16, to bf16 (nearest,
- * ties to even).
- *   w          block_size 64; cols % 64 == 0, rows % 8 == 0.
+ * rounded once to fp32 (one FMA) and then, for NF4_BF16 or NF4_F16, to that
+ * type (nearest, ties to even; beyond the f16 range, +-inf).
+ *   w          block_size a power of two from 64 to 4096; cols % 64 == 0,
+ *              rows % 8 == 0.
  *   A, B       [r, K] and [N, r] bf16; 8 <= r <= 256, r % 8 == 0.
- *   out_dtype  NF4_BF16 or NF4_F32; out has rows * cols elements, written.
+ *   out_dtype  NF4_BF16, NF4_F16 or NF4_F32; out has rows * cols elements,
+ *              written.
  *   workspace  >= nf4_workspace_bytes(NF4_OP_MERGE, 0, N, K, r, 64, dq): the
  *              status word only.
  * Same validation, ownership and error rules as the linear entry points.

@@ -326,7 +326,8 @@ def merge(q: dict, a, b, alpha: float, out_dtype: str = "bf16") -> np.ndarray:
 
     W' is the fp32 dequant; B A and the sum are exact in fp64.  out_dtype
     "f64" returns that sum, "f32" its round to fp32, "bf16" the uint16 bits of
-    the fp32 value rounded to bf16 (R16).
+    the fp32 value rounded to bf16, "f16" the fp32 value rounded to f16 (R16;
+    the f16 output is the pages' F16 compute dtype applied to the merge).
     """
     w = dequantize(q, "f32").astype(np.float64)
     a = np.asarray(a, dtype=np.float64)
@@ -340,6 +341,9 @@ def merge(q: dict, a, b, alpha: float, out_dtype: str = "bf16") -> np.ndarray:
         return m32
     if out_dtype == "bf16":
         return bf16_round(m32).reshape(merged.shape)
+    if out_dtype == "f16":
+        with np.errstate(over="ignore"):   # beyond the f16 range: +-inf, as IEEE rounding gives
+            return m32.astype(np.float16)
     raise ValueError(out_dtype)
 
 

@@ -56,7 +56,8 @@ nf4_status check_linear(const nf4_weight* w, const void* x, int64_t M, const voi
   if (compute_dtype != NF4_BF16 && compute_dtype != NF4_F16 && compute_dtype != NF4_F32)
     return NF4_ERR_INVALID_ARG;
   if (M < 1 || w->rows < 1 || w->cols < 1) return NF4_ERR_SHAPE;
-  if (w->block_size != 64) return NF4_ERR_UNSUPPORTED;
+  if (w->block_size < 1) return NF4_ERR_SHAPE;
+  if (nf4::log2_block(w->block_size) < 0) return NF4_ERR_UNSUPPORTED;   // 64, 128, ..., 4096
   if (w->cols % 64 != 0 || w->rows % 8 != 0) return NF4_ERR_SHAPE;
   if (M > (int64_t(1) << 31) || w->rows > (int64_t(1) << 31) || w->cols > (int64_t(1) << 31))
     return NF4_ERR_SHAPE;
@@ -455,9 +456,7 @@ nf4_status nf4_merge(const nf4_weight* w, const void* A, const void* B, int r, f
   // the linear checks with a stand-in x (the merge has no activations)
   nf4_status s = check_linear(w, A, 1, A, B, r, alpha, NF4_BF16);
   if (s != NF4_OK) return s;
-  if (out_dtype != NF4_BF16 && out_dtype != NF4_F32) {
-    return out_dtype == NF4_F16 ? NF4_ERR_UNSUPPORTED : NF4_ERR_INVALID_ARG;
-  }
+  if (out_dtype != NF4_BF16 && out_dtype != NF4_F32 && out_dtype != NF4_F16) return NF4_ERR_INVALID_ARG;
   if (out == nullptr) return NF4_ERR_INVALID_ARG;
   if (!aligned16(out)) return NF4_ERR_ALIGNMENT;
   if (workspace == nullptr || !aligned16(workspace)) return NF4_ERR_WORKSPACE;
@@ -465,7 +464,8 @@ nf4_status nf4_merge(const nf4_weight* w, const void* A, const void* B, int r, f
     return NF4_ERR_WORKSPACE;
   uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + nf4::kWsStatus);
   int launches = 0;
-  const cudaError_t e = nf4::launch_merge(*w, A, B, r, alpha, out_dtype == NF4_F32 ? 1 : 0, out,
+  const int kind = out_dtype == NF4_F32 ? nf4::kMergeF32 : (out_dtype == NF4_F16 ? nf4::kMergeF16 : nf4::kMergeBf16);
+  const cudaError_t e = nf4::launch_merge(*w, A, B, r, alpha, kind, out,
                                           status, static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches);
 }

@@ -45,6 +45,7 @@ struct F32Operand {
   const uint8_t* absmax_q;
   const float* absmax_scale;
   int dq;
+  int bs_shift;            // log2 of the NF4 block size (6 .. 12)
   int64_t wcols;           // W's row length; kmajor: (i, kk) = W[i, kk], else W[kk, i]
 };
 
@@ -82,7 +83,8 @@ __device__ __forceinline__ void load_slice(const F32Operand& o, int64_t i0, int6
   v[0] = v[1] = v[2] = v[3] = 0.0f;
   if (o.nf4) {
     // four consecutive elements along a row of W: two code bytes, one scale
-    // block (the row length and the column are multiples of 4, the block 64)
+    // block (the row length and the column are multiples of 4, the block a
+    // power of two of at least 64 elements)
     bool ok;
     int64_t e;
     if (o.kmajor) {
@@ -94,7 +96,7 @@ __device__ __forceinline__ void load_slice(const F32Operand& o, int64_t i0, int6
     }
     if (!ok) return;
     const uint16_t two = *reinterpret_cast<const uint16_t*>(o.codes + (e >> 1));
-    const int64_t blk = e >> 6;
+    const int64_t blk = e >> o.bs_shift;
     const float scale =
         o.dq ? __fmul_rn(float(o.absmax_q[blk]), *o.absmax_scale) : o.absmax[blk];
     const uint32_t b0 = two & 0xffu, b1 = two >> 8;
@@ -249,6 +251,7 @@ F32Operand nf4_weight_operand(const nf4_weight* w, bool kmajor, int64_t extent) 
   o.absmax_q = w->absmax_q;
   o.absmax_scale = w->absmax_scale;
   o.dq = w->double_quant ? 1 : 0;
+  o.bs_shift = log2_block(w->block_size);
   o.wcols = w->cols;
   return o;
 }

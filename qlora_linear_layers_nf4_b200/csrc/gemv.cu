@@ -57,7 +57,8 @@ constexpr size_t kGvMaxDynSmem = 194u * 1024u;
 
 struct GemvParams {
   int M, N, K, r;
-  int kb_per_row;       // K / 64
+  int kb_per_row;       // K / 64: 64-element chunks per W row
+  int bs_shift;         // log2 of the NF4 block size (6 .. 12)
   int blocks_per_slice;
   int vec_scales;       // 16-byte aligned scale rows: vector loads
   int slices;
@@ -316,8 +317,10 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     for (int j = 0; j < kScaleRegs; ++j) {
       const int b = (threadIdx.x >> 7) + kScaleSteps * j;
       uint32_t v = 0;
-      if (b < nblk && swr < p.N)
-        v = dq ? uint32_t(__ldg(p.absmax_q + sidx0 + b)) : __float_as_uint(__ldg(p.absmax + sidx0 + b));
+      if (b < nblk && swr < p.N) {
+        const int64_t si = chunk_block(swr, p.K, kb0 + b, p.bs_shift);
+        v = dq ? uint32_t(__ldg(p.absmax_q + si)) : __float_as_uint(__ldg(p.absmax + si));
+      }
       sc_raw[j] = v;
     }
   }
@@ -644,10 +647,11 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   p.K = int(a.K);
   p.r = a.r;
   p.kb_per_row = kb;
+  p.bs_shift = log2_block(a.w->block_size);
   p.blocks_per_slice = bps;
   // a row's 16 scales of a slice start on a 16-byte boundary (u8) or a
   // 16-byte boundary of fp32 (four vectors) for every row and slice
-  p.vec_scales = bps == kGvMaxBlocks &&
+  p.vec_scales = bps == kGvMaxBlocks && a.w->block_size == 64 &&
                  (a.w->double_quant ? (kb % 16 == 0 && (reinterpret_cast<uintptr_t>(a.w->absmax_q) & 15u) == 0)
                                     : (kb % 4 == 0 && (reinterpret_cast<uintptr_t>(a.w->absmax) & 15u) == 0));
   p.slices = slices;

@@ -78,6 +78,13 @@ struct LinearArgs {
 
 size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, int r);
 
+// log2 of a block size the GEMM paths take (a power of two, 64 .. 4096), else -1.
+inline int log2_block(int64_t bs) {
+  for (int s = 6; s <= 12; ++s)
+    if (bs == (int64_t(1) << s)) return s;
+  return -1;
+}
+
 // 2-D TMA map over a row-major matrix (`inner` elements per row, `outer`
 // rows; bf16 or u8), optional 128-byte swizzle.  False if it cannot be encoded.
 bool make_map_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
@@ -110,8 +117,12 @@ cudaError_t launch_wait_timeout_check(uint32_t* status, uint64_t limit_ns, uint3
                                       cudaStream_t st, int* launches);
 
 // Dense merge W' + s B A (merge.cu).
+// Output types of the merge.
+constexpr int kMergeBf16 = 0;
+constexpr int kMergeF32 = 1;
+constexpr int kMergeF16 = 2;
 cudaError_t launch_merge(const nf4_weight& w, const void* A, const void* B, int r, float alpha,
-                         int out_f32, void* out, uint32_t* status, cudaStream_t st, int* launches);
+                         int out_kind, void* out, uint32_t* status, cudaStream_t st, int* launches);
 
 }  // namespace nf4
 

@@ -19,6 +19,7 @@
 // the contraction is a small fraction of its time.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kernels.h"
 #include "nf4_common.cuh"
@@ -44,10 +45,10 @@ constexpr uint32_t kMgABytes = (kMgCols / 64) * 64 * 128; // 64 r x kMgCols k (b
 constexpr uint32_t kMgChunkBytes = kMgBBytes + kMgABytes;
 
 struct MergeParams {
-  int N, K, r, chunks, kb_per_row;
+  int N, K, r, chunks, bs_shift;
   float s;
   int double_quant;
-  int out_f32;
+  int out_kind;        // kMergeBf16, kMergeF32 or kMergeF16
   const uint8_t* codes;
   const uint8_t* absmax_q;
   const float* absmax;
@@ -67,6 +68,14 @@ struct MergeShared {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// Two merged values as one 32-bit word of the 2-byte output type.
+__device__ __forceinline__ uint32_t pack_out2(bool f16, float lo, float hi) {
+  return f16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 
 // Bytes of the operand region: every r chunk, and at least the output staging.
@@ -172,7 +181,7 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         if (kh + 64 * j >= p.K) continue;
-        const int64_t blk = int64_t(n) * p.kb_per_row + (kh + 64 * j) / 64;
+        const int64_t blk = chunk_block(n, p.K, (kh + 64 * j) / 64, p.bs_shift);
         scale[j] = p.double_quant ? __fmul_rn(float(__ldg(p.absmax_q + blk)), s_g) : __ldg(p.absmax + blk);
       }
     }
@@ -182,6 +191,7 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
     tc_fence_after();
     if (ok) {
       const float* lut = sh->lut + lane;
+      const bool f16 = p.out_kind == kMergeF16;
       uint8_t* stage = smem + (warp - 2) * 2 * kMgStageBytes;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -211,7 +221,7 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
         uint8_t* buf = stage + (c & 1) * kMgStageBytes;
         if (lane == 0 && c >= 2) bulk_wait_group_read<1>();
         __syncwarp();
-        if (p.out_f32) {       // 128-byte rows, 128-byte swizzle: chunk j at j ^ (lane & 7)
+        if (p.out_kind == kMergeF32) {   // 128-byte rows, 128-byte swizzle: chunk j at j ^ (lane & 7)
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             *reinterpret_cast<float4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
@@ -220,8 +230,8 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
-                make_uint4(pack_bf16x2(m[8 * j], m[8 * j + 1]), pack_bf16x2(m[8 * j + 2], m[8 * j + 3]),
-                           pack_bf16x2(m[8 * j + 4], m[8 * j + 5]), pack_bf16x2(m[8 * j + 6], m[8 * j + 7]));
+                make_uint4(pack_out2(f16, m[8 * j], m[8 * j + 1]), pack_out2(f16, m[8 * j + 2], m[8 * j + 3]),
+                           pack_out2(f16, m[8 * j + 4], m[8 * j + 5]), pack_out2(f16, m[8 * j + 6], m[8 * j + 7]));
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -253,7 +263,7 @@ size_t merge_smem_bytes(int chunks) {
 }
 
 cudaError_t launch_merge(const nf4_weight& w, const void* A, const void* B, int r, float alpha,
-                         int out_f32, void* out, uint32_t* status, cudaStream_t st, int* launches) {
+                         int out_kind, void* out, uint32_t* status, cudaStream_t st, int* launches) {
   static PerDeviceOnce attr_done;
   const int dev = PerDeviceOnce::current();
   if (!attr_done.done(dev)) {
@@ -270,18 +280,21 @@ cudaError_t launch_merge(const nf4_weight& w, const void* A, const void* B, int 
   // (MN-major); out [N, K]: 32 x 128 boxes in the staging layout.
   bool ok = make_map_2d(&tb, B, true, uint64_t(r), uint64_t(N), 64, kMgRows, true);
   ok = ok && make_map_2d(&ta, A, true, uint64_t(K), uint64_t(r), 64, 64, true);
-  ok = ok && (out_f32 ? make_map_2d_f32(&to, out, uint64_t(K), uint64_t(N), 32, 32, CU_TENSOR_MAP_SWIZZLE_128B)
-                      : make_map_2d_bf16(&to, out, uint64_t(K), uint64_t(N), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
+  // (the store copies bytes: a bf16 map serves the f16 output as well)
+  ok = ok && (out_kind == kMergeF32
+                  ? make_map_2d_f32(&to, out, uint64_t(K), uint64_t(N), 32, 32, CU_TENSOR_MAP_SWIZZLE_128B)
+                  : make_map_2d_bf16(&to, out, uint64_t(K), uint64_t(N), 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
   if (!ok) return cudaErrorInvalidValue;
   MergeParams p;
   p.N = int(N);
   p.K = int(K);
   p.r = r;
   p.chunks = (r + 63) / 64;
-  p.kb_per_row = int(K / 64);
+  p.bs_shift = log2_block(w.block_size);
+  if (p.bs_shift < 0) return cudaErrorInvalidValue;
   p.s = alpha / float(r);
   p.double_quant = w.double_quant;
-  p.out_f32 = out_f32;
+  p.out_kind = out_kind;
   p.codes = w.codes;
   p.absmax_q = w.absmax_q;
   p.absmax = w.absmax;

@@ -56,6 +56,14 @@ __device__ __forceinline__ float level(int c) {
   return __uint_as_float(kLevelBitsDev[c]);
 }
 
+// Block index of the 64-element chunk `chunk` (along the row) of W row `row`:
+// blocks run over the row-major flattened tensor and hold 2^bs_shift >= 64
+// elements, so a 64-aligned chunk never straddles two blocks.
+__host__ __device__ __forceinline__ int64_t chunk_block(int64_t row, int64_t cols, int64_t chunk,
+                                                        int bs_shift) {
+  return (row * cols + chunk * 64) >> bs_shift;
+}
+
 __device__ __forceinline__ void report(uint32_t* status, uint32_t code) {
   if (status != nullptr) atomicCAS(status, 0u, code);
 }

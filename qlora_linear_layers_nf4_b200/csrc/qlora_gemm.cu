@@ -159,7 +159,8 @@ struct FusedParams {
   int main_steps;    // fwd: K / 64; dx: ceil(N / 64)
   int adapter_steps; // ceil(r / 64)
   int out_cols;      // N (fwd) or K (dx)
-  int kb_per_row;    // K / 64 NF4 blocks per W row
+  int kb_per_row;    // K / 64: 64-element chunks per W row
+  int bs_shift;      // log2 of the NF4 block size (6 .. 12)
   int double_quant;
   int f16;           // operands and outputs in f16 (else bf16)
   const uint8_t* absmax_q;
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       if (row >= p.N) return 0.0f;
       const int bcol = (MODE == kFwd) ? it : block_col0;
       if (MODE == kDx && bcol >= p.kb_per_row) return 0.0f;
-      return load_scale(p.absmax_q, p.absmax, s_g, dq, row * p.kb_per_row + bcol);
+      return load_scale(p.absmax_q, p.absmax, s_g, dq, chunk_block(row, p.K, bcol, p.bs_shift));
     };
     float next_scale = p.main_steps > 0 ? scale_at(0) : 0.0f;
     for (int it = 0; it < p.main_steps; ++it) {
@@ -672,7 +673,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP2Threads, 1)
       if (wr >= p.N) return 0.0f;
       const int bcol = (MODE == kFwd) ? ks : block_col0;
       if (MODE == kDx && bcol >= p.kb_per_row) return 0.0f;
-      return load_scale(p.absmax_q, p.absmax, s_g, dq, wr * p.kb_per_row + bcol);
+      return load_scale(p.absmax_q, p.absmax, s_g, dq, chunk_block(wr, p.K, bcol, p.bs_shift));
     };
     // scales of the next four steps in flight (a small register ring)
     float sc[4];
@@ -1246,6 +1247,7 @@ FusedParams fused_params(const LinearArgs& a, int mode) {
   p.adapter_steps = int(cdiv(a.r, 64));
   p.out_cols = mode == kFwd ? int(a.N) : int(a.K);
   p.kb_per_row = int(a.K / 64);
+  p.bs_shift = log2_block(a.w->block_size);
   p.double_quant = a.w->double_quant;
   p.f16 = a.f16;
   p.absmax_q = a.w->absmax_q;

@@ -286,9 +286,10 @@ def dequantize(q: QuantizedWeight, out_dtype: str = "f32", stream=None):
 
 def merge(q: QuantizedWeight, A, B, alpha: float, out_dtype: str = "bf16", out=None,
           workspace: Workspace | None = None, stream=None):
-    """Dense merged weight dequant(W) + (alpha/r) B A, [rows, cols] in bf16 or f32."""
+    """Dense merged weight dequant(W) + (alpha/r) B A, [rows, cols] in bf16, f16 or f32."""
     import torch
-    dt = {"f32": (NF4_F32, torch.float32), "bf16": (NF4_BF16, torch.bfloat16)}[out_dtype]
+    dt = {"f32": (NF4_F32, torch.float32), "bf16": (NF4_BF16, torch.bfloat16),
+          "f16": (NF4_F16, torch.float16)}[out_dtype]
     if A.dim() != 2:
         raise ValueError("A must be 2-D ([r, K])")
     r = A.shape[0]

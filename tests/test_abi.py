@@ -126,7 +126,12 @@ def test_linear_host_validation():
     assert _fwd(_cw(), M=0) == 2
     assert _fwd(_cw(cols=4000)) == 2              # K % 64
     assert _fwd(_cw(rows=4092)) == 2              # N % 8
-    assert _fwd(_cw(bs=128)) == 4                 # GEMMs take block 64
+    assert _fwd(_cw(bs=128), wsb=0) == 5          # powers of two from 64 to 4096 pass the checks
+    assert _fwd(_cw(bs=4096), wsb=0) == 5
+    assert _fwd(_cw(bs=32)) == 4                  # below 64: a K step would hold two blocks
+    assert _fwd(_cw(bs=96)) == 4                  # not a power of two
+    assert _fwd(_cw(bs=8192)) == 4
+    assert _fwd(_cw(bs=0)) == 2
     assert _fwd(_cw(), x=FAKE + 2) == 3
     assert _fwd(_cw(), y=None) == 1
     assert _fwd(_cw(), wsb=0) == 5
@@ -142,12 +147,13 @@ def test_merge_host_validation():
         ctypes.byref(cw), FAKE, FAKE, r, 32.0, dt, out, FAKE, wsb, None)
     assert m(_cw(), r=4) == 1                     # r < 8
     assert m(_cw(), r=264) == 1                   # r > 256
-    assert m(_cw(), dt=2) == 4                    # f16 output: not in this build
+    assert m(_cw(), dt=2, wsb=0) == 5             # f16 output passes the dtype check
     assert m(_cw(), dt=7) == 1
     assert m(_cw(), out=None) == 1
     assert m(_cw(), out=FAKE + 2) == 3
     assert m(_cw(cols=4000)) == 2                 # K % 64
-    assert m(_cw(bs=128)) == 4                    # block 64 only
+    assert m(_cw(bs=256), wsb=0) == 5             # powers of two from 64 to 4096
+    assert m(_cw(bs=192)) == 4
     assert m(_cw(), wsb=0) == 5
 
 

@@ -49,8 +49,8 @@ def _run(case, dev, zero_w=False, bias=False, rows=None, t_from_fwd=True):
     from qlora_linear_layers_nf4_b200 import nf4qlora as Q
     inp = WL.draw_linear(case)
     w = np.zeros_like(inp.w) if zero_w else inp.w
-    ref_q = O.quantize(w, 64, double=case.double_quant)
-    q = Q.quantize(torch.from_numpy(w).to(dev), 64, case.double_quant)
+    ref_q = O.quantize(w, case.block_size, double=case.double_quant)
+    q = Q.quantize(torch.from_numpy(w).to(dev), case.block_size, case.double_quant)
     f32 = inp.extra["f32"]
     x, A, B, dy = (torch.from_numpy(np.ascontiguousarray(f32[k])).to(dev) for k in ("x", "a", "b", "dy"))
     bias_t = bias_np = None
@@ -105,6 +105,15 @@ def test_f32_shapes(cuda_device, m, n, k, rank, dq, bias):
     case = WL.LinearCase(f"f32 {m}x{n}x{k} r={rank}", n=n, k=k, m=m, r=rank, alpha=2.0 * rank,
                          seed=5000 + m + n + k + rank, double_quant=dq)
     _run(case, cuda_device, bias=bias)
+    _run(case, cuda_device, zero_w=True)
+
+
+@pytest.mark.parametrize("bs", [128, 1024])
+def test_f32_block_sizes(cuda_device, bs):
+    """Blocks of 128 and 1024 over the flattened weight (they straddle rows of 320)."""
+    case = WL.LinearCase(f"f32 block {bs}", n=264, k=320, m=100, r=16, alpha=32.0,
+                         seed=5200 + bs, block_size=bs, double_quant=True)
+    _run(case, cuda_device, bias=True)
     _run(case, cuda_device, zero_w=True)
 
 

@@ -167,6 +167,28 @@ def test_backward_on_parallel_streams(cuda_device):
         assert ws.read_status() == 0
 
 
+# Block sizes other than 64: powers of two up to 4096, over the flattened weight
+# (a block may straddle rows when K is not a multiple of it).  Each case runs
+# the pair GEMM (M > 256), the single-CTA GEMM (32 < M <= 256) or the decode
+# path (M <= 32), forward and backward, with the adapter-only check too.
+@pytest.mark.parametrize("m,n,k,bs,dq", [
+    (520, 512, 512, 128, True),      # pair tiles
+    (300, 264, 320, 256, False),     # ragged pair tiles; blocks of 256 straddle rows of 320
+    (200, 512, 768, 128, True),      # single-CTA tiles
+    (96, 256, 4096, 4096, True),     # one block per row
+    (1, 1024, 1024, 128, True),      # decode
+    (16, 512, 4096, 256, False),     # decode, 16 tokens
+    (5, 256, 192, 128, True),        # decode, blocks straddle rows of 192
+])
+def test_block_sizes(cuda_device, m, n, k, bs, dq):
+    case = WL.LinearCase(f"block {bs} {m}x{n}x{k}", n=n, k=k, m=m, r=16, alpha=32.0,
+                         seed=6000 + m + n + k + bs, block_size=bs, double_quant=dq)
+    for zero_w in (False, True):
+        r = Run(case, cuda_device, zero_w=zero_w)
+        r.check_forward()
+        r.check_backward()
+
+
 def test_recomputed_t_matches(cuda_device):
     import torch
     case = WL.LinearCase("recompute t", n=512, k=512, m=200, r=32, alpha=64.0, seed=77)

@@ -5,7 +5,8 @@ Bound per element (both outputs are one rounding of an fp32 value):
   fp32: |gpu - exact| <= 2^-23 |exact| + (r + 2) 2^-24 s (|B| |A|)
         (the fp32 rounding of the sum plus the fp32 accumulation of r exact
         bf16 x bf16 products);
-  bf16: |gpu - exact| <= ulp_bf16(exact) + the fp32 bound above.
+  bf16: |gpu - exact| <= ulp_bf16(exact) + the fp32 bound above;
+  f16:  |gpu - exact| <= ulp_f16(exact) + the fp32 bound above (normal range).
 With B = 0 the merge is the plain dequant and must match it bit for bit.
 """
 import numpy as np
@@ -39,8 +40,10 @@ def _run(case, dev, zero_w=False, zero_b=False, rows=None):
     ws = Q.Workspace(dev)
     out_bf = Q.merge(q, A, B, case.alpha, "bf16", workspace=ws)
     out_f32 = Q.merge(q, A, B, case.alpha, "f32", workspace=ws)
+    out_h = Q.merge(q, A, B, case.alpha, "f16", workspace=ws)
     torch.cuda.synchronize()
     assert ws.read_status() == 0
+    _run.last_f16 = out_h
     return inp, ref_q, b, out_bf, out_f32
 
 
@@ -61,6 +64,14 @@ def _check(case, inp, ref_q, b_bits, out_bf, out_f32, rows=None):
     want_bits = O.merge(qsel, a, b[sel], case.alpha, "bf16")
     got_bits = out_bf.cpu().view(__import__("torch").int16).numpy()[sel].view(np.uint16)
     assert np.mean(got_bits == want_bits) > 0.999
+    # the f16 output of the same call: one f16 ulp plus the fp32 bound, and
+    # almost always the f16 rounding of the oracle's fp32 value
+    gh = _run.last_f16.cpu().numpy()[sel]
+    assert np.all(np.isfinite(gh))
+    ulp_h = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact), 2.0 ** -14))) - 10)
+    assert np.all(np.abs(gh.astype(np.float64) - exact) <= ulp_h + bound32), "f16 outside one ulp"
+    want_h = O.merge(qsel, a, b[sel], case.alpha, "f16")
+    assert np.mean(gh.view(np.uint16) == want_h.view(np.uint16)) > 0.999
 
 
 def _rows_of(q, rows):
@@ -106,6 +117,16 @@ def test_b_zero_is_the_dequant_bit_for_bit(cuda_device):
                           O.dequantize(ref_q, "f32").view(np.uint32))
     assert np.array_equal(out_bf.cpu().view(torch.int16).numpy().view(np.uint16),
                           O.dequantize(ref_q, "bf16"))
+    assert np.array_equal(_run.last_f16.cpu().numpy().view(np.uint16),
+                          O.dequantize(ref_q, "f16").view(np.uint16))
+
+
+@pytest.mark.parametrize("bs,k", [(128, 512), (256, 320), (1024, 4096)])
+def test_block_sizes(cuda_device, bs, k):
+    """Blocks of 128 to 1024 elements (straddling rows when K is not a multiple)."""
+    case = WL.LinearCase(f"merge block {bs}", n=264, k=k, m=1, r=32, alpha=64.0, seed=2100 + bs,
+                         block_size=bs)
+    _check(case, *_run(case, cuda_device))
 
 
 def test_zero_base_leaves_the_update(cuda_device):

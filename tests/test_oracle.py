@@ -544,3 +544,21 @@ def test_double_quant_of_a_part_uses_the_whole_max():
     q_default, s_default = O.double_quant(a)
     q_given, s_given = O.double_quant(a, g=a.max())
     assert np.array_equal(q_default, q_given) and s_default == s_given
+
+
+def test_merge_f16_is_the_f16_rounding_of_the_fp32_merge():
+    """The merge's f16 output (R16 with the F16 compute dtype) is the
+    round-to-nearest-even f16 of the fp32 merged value, overflow to inf."""
+    import torch
+    rng = np.random.default_rng(77)
+    w = (rng.standard_normal((8, 128)) * 0.02).astype(np.float32)
+    w[0, :64] *= 5e6                  # one block whose merged values pass 65504
+    q = O.quantize(w, 64, double=False)
+    a = rng.standard_normal((8, 128)) * 0.1
+    b = rng.standard_normal((8, 8)) * 0.01
+    m32 = O.merge(q, a, b, 16.0, "f32")
+    want = torch.from_numpy(m32).half().numpy()
+    got = O.merge(q, a, b, 16.0, "f16")
+    assert got.dtype == np.float16
+    assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+    assert np.isinf(got[0, :64]).any()
