@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the hash of the kernel source it was taken on; reported as null once the
 # source changes.
 NCU_TRAFFIC = {
-    # forward 125.3 MB, dx 178.7 MB per launch
-    "5658984bc2757e50": {"fwd": 69_511_424 + 55_790_080, "dx": 159_868_928 + 18_873_600},
+    # forward 126.1 MB, dx 177.2 MB per launch
+    "b6c61cf6b609ba98": {"fwd": 70_948_864 + 55_177_728, "dx": 157_914_880 + 19_273_728},
 }
 
 
