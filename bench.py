@@ -658,7 +658,8 @@ def measure_rows(args, dev, flush, pk, pk_kind, barrier):
 
         nbytes = (case.n * case.k // 2 + case.n * case.k // 64 + 4 + 2 * case.r * case.k
                   + 2 * case.n * case.r + 2 * case.m * (case.k + case.n))
-        row(f"decode_fwd_M{case.m}", [fcall(cw) for cw in cws], nbytes, RD * nbytes, replays=20)
+        # 128 calls per graph (each weight twice, 63 others in between)
+        row(f"decode_fwd_M{case.m}", [fcall(cw) for cw in cws + cws], nbytes, RD * nbytes, replays=20)
     del qws
     torch.cuda.empty_cache()
 

@@ -346,7 +346,11 @@ NF4_API nf4_status qlora_linear_fwd(const nf4_weight* w, const void* x, int64_t 
  * from `stream` after U and joined back with events before the call returns,
  * so work the caller enqueues on `stream` afterwards sees every output;
  * `stream` must belong to the current device.  Calls from several host
- * threads serialise on a lock while they enqueue.
+ * threads serialise on a lock while they enqueue.  The fork and join are
+ * ordinary event dependencies, so a backward call enqueued while `stream` is
+ * being captured into a CUDA graph becomes part of the graph, side branch
+ * included (the side stream is made on the first call, so make one call
+ * before capturing).
  */
 NF4_API nf4_status qlora_linear_bwd(const nf4_weight* w, const void* x, int64_t M, const void* A,
                             const void* B, int r, float alpha, int compute_dtype,

@@ -189,6 +189,39 @@ def test_block_sizes(cuda_device, m, n, k, bs, dq):
         r.check_backward()
 
 
+def test_forward_backward_in_a_cuda_graph(cuda_device):
+    """A training step's forward and backward captured in a CUDA graph (the
+    backward forks dx onto its side stream inside the capture) replays to the
+    bits of the same calls made eagerly."""
+    import torch
+    Q = _Q()
+    case = WL.LinearCase("graph", n=1024, k=768, m=600, r=32, alpha=64.0, seed=4200)
+    r = Run(case, cuda_device)
+    ws = Q.Workspace(cuda_device)
+    y = torch.empty_like(r.y)
+    T = torch.empty_like(r.T)
+    dA, dB, dx = torch.empty_like(r.dA), torch.empty_like(r.dB), torch.empty_like(r.dx)
+    st = torch.cuda.Stream(device=cuda_device)
+
+    def step():
+        Q.linear_fwd(r.q, r.x, r.A, r.B, case.alpha, out=y, t_out=T, workspace=ws)
+        Q.linear_bwd(r.q, r.x, r.A, r.B, case.alpha, r.dy, t=T, dA=dA, dB=dB, dx=dx, workspace=ws)
+
+    with torch.cuda.stream(st):
+        step()                      # warm-up outside the capture (workspace, side stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        step()
+    for out in (y, T, dA, dB, dx):
+        out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert ws.read_status() == 0
+    for got, want in ((y, r.y), (T, r.T), (dA, r.dA), (dB, r.dB), (dx, r.dx)):
+        assert torch.equal(got, want)
+
+
 def test_recomputed_t_matches(cuda_device):
     import torch
     case = WL.LinearCase("recompute t", n=512, k=512, m=200, r=32, alpha=64.0, seed=77)
