@@ -71,6 +71,7 @@ struct GemvParams {
   const __nv_bfloat16* bias;
   __nv_bfloat16* y;
   __nv_bfloat16* t_out;
+  const __nv_bfloat16* t_in;   // TP == 0: T = s x A^T [M, r] from the kernel before
   uint32_t* status;
 };
 
@@ -203,7 +204,10 @@ __device__ __forceinline__ void frag_pair(const uint4& lo, const uint4& hi, int 
 // MMA row g + 8 is W row 2g + 1.  In a half-warp the four rows a code load
 // touches then differ in bits 1..2 of the row, which the 128-byte swizzle
 // turns into four different 32-byte bank groups: the loads are conflict-free.
-// TP: the x A^T of a slice as TP partial sums over interleaved K blocks (1, 2 or 4).
+// TP: the x A^T of a slice as TP partial sums over interleaved K blocks (1, 2
+// or 4); TP == 0: T = s x A^T comes finished from the kernel before (larger
+// r, whose A tiles would not fit beside the weight tiles), read after the
+// dependency wait, and slice 0 adds the whole T B^T.
 template <int NT8, int RG, bool F16, int TP>
 __global__ void __launch_bounds__(kGvThreads, 1)
     nf4_gemv(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
@@ -215,7 +219,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(1024) uint32_t lut[256 * 32];      // [entry][lane] copies
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const GemvLayout L = gemv_layout(p.blocks_per_slice, NP, p.r_pad, p.r, kPhases, TP);
+  constexpr bool kTGiven = TP == 0;
+  const GemvLayout L = gemv_layout(p.blocks_per_slice, NP, kTGiven ? 0 : p.r_pad, p.r, kPhases, TP);
   uint8_t* codes = smem + L.codes;
   uint8_t* xs = smem + L.xs;
   uint8_t* as = smem + L.as;
@@ -251,7 +256,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   const uint32_t xbytes = uint32_t(NP) * 128u;
   const uint32_t abytes = uint32_t(p.r_pad) * 128u;
   const int band = kGvRows / S;                // rows of the tile this CTA finishes
-  const bool pull_t = p.t_out != nullptr && blockIdx.x == 0;   // uniform over the cluster
+  const bool pull_t = !kTGiven && p.t_out != nullptr && blockIdx.x == 0;   // uniform over the cluster
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -338,6 +343,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       } else if (part == 1) {
         mbar_arrive_expect_tx(&bar[grp], xbytes * kGvGroup);
         tma_load_3d(xs + b * xbytes, &tm_x, &bar[grp], 0, 0, kb);
+      } else if (kTGiven) {
+        mbar_arrive(&bar[grp]);   // no A tiles: T comes finished
       } else {
         mbar_arrive_expect_tx(&bar[grp], abytes * kGvGroup);
         tma_load_3d(as + b * abytes, &tm_a, &bar[grp], 0, 0, kb);
@@ -429,9 +436,9 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     // r_pad / 16 row groups and, when there are fewer than four, the K
     // blocks, so no single warp walks every block alone.
     const int aw = warp - kGvWWarps;
-    const int j0 = (aw / t_parts) * 16;
-    const int part = aw % t_parts;
-    if (j0 < p.r_pad) {
+    const int j0 = kTGiven ? p.r_pad : (aw / (kTGiven ? 1 : t_parts)) * 16;
+    const int part = aw % (kTGiven ? 1 : t_parts);
+    if (!kTGiven && j0 < p.r_pad) {
       float ta[NT8][4];
 #pragma unroll
       for (int t = 0; t < NT8; ++t) ta[t][0] = ta[t][1] = ta[t][2] = ta[t][3] = 0.0f;
@@ -511,15 +518,22 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     // the tile's B rows (bf16 in shared memory) as A and s T_slice rounded to
     // the compute type as B.
     ok = __all_sync(0xffffffffu, ok && mbar_wait(bar_b, 0, &abort_flag, p.status));
-    if (ok) {
+    if (ok && (!kTGiven || slice == 0)) {
       for (int j0 = 0; j0 < p.r_pad; j0 += 16) {
         uint32_t tfr[NT8][2];
 #pragma unroll
         for (int t = 0; t < NT8; ++t) {
           const int m = 8 * t + g;
           const int ja = j0 + 2 * q, jb = j0 + 2 * q + 8;
-          tfr[t][0] = pack2_rn<F16>(p.s * t_sum(ja * NP + m), p.s * t_sum((ja + 1) * NP + m));
-          tfr[t][1] = pack2_rn<F16>(p.s * t_sum(jb * NP + m), p.s * t_sum((jb + 1) * NP + m));
+          if (kTGiven) {
+            // two consecutive adapter columns of token m (r is a multiple of 8)
+            const uint32_t* trow = reinterpret_cast<const uint32_t*>(p.t_in + int64_t(m) * p.r);
+            tfr[t][0] = (m < p.M && ja < p.r) ? __ldg(trow + (ja >> 1)) : 0u;
+            tfr[t][1] = (m < p.M && jb < p.r) ? __ldg(trow + (jb >> 1)) : 0u;
+          } else {
+            tfr[t][0] = pack2_rn<F16>(p.s * t_sum(ja * NP + m), p.s * t_sum((ja + 1) * NP + m));
+            tfr[t][1] = pack2_rn<F16>(p.s * t_sum(jb * NP + m), p.s * t_sum((jb + 1) * NP + m));
+          }
         }
         // B columns j >= r hold no adapter: masked to 0 (tpart rows r .. r_pad-1
         // are 0 too, from the zero-filled A rows)
@@ -604,7 +618,8 @@ bool decode_supported(int64_t M, int64_t N, int64_t K, int r) {
   return M >= 1 && M <= 32 && r <= kGvMaxR;
 }
 
-cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches) {
+cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches,
+                              const void* t_given, bool dry_run) {
   (void)sms;
   const int kb = int(a.K / 64);
   const int tiles = int((a.N + kGvRows - 1) / kGvRows);
@@ -617,14 +632,15 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   // slice is split over the four adapter warps by K block as well, so it
   // finishes with the weight rows (more tokens keep the W warps busier).
   const int t_groups = r_pad / 16;
-  const int t_parts = (nt8 == 1 && t_groups <= 2) ? 4 / t_groups : 1;
+  const int t_parts = t_given != nullptr ? 0 : ((nt8 == 1 && t_groups <= 2) ? 4 / t_groups : 1);
+  const int lay_r = t_given != nullptr ? 0 : r_pad;   // A tile rows held in shared memory
   // K slices: one wave of one CTA per SM where possible, and everything a CTA
   // reads fits in its shared memory at once.
   int slices = 1;
   while (slices < kGvMaxSlices && tiles * slices * 2 <= 148 && slices * 2 <= kb) slices *= 2;
   int bps = (kb + slices - 1) / slices;
   auto fits = [&](int b) {
-    return b <= kGvMaxBlocks && gemv_layout(b, np, r_pad, a.r, phases, t_parts).total <= kGvMaxDynSmem;
+    return b <= kGvMaxBlocks && gemv_layout(b, np, lay_r, a.r, phases, t_parts).total <= kGvMaxDynSmem;
   };
   while (!fits(bps) && slices < kGvMaxSlices) {
     slices *= 2;
@@ -664,9 +680,10 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   p.bias = static_cast<const __nv_bfloat16*>(a.bias);
   p.y = static_cast<__nv_bfloat16*>(a.y);
   p.t_out = static_cast<__nv_bfloat16*>(a.t_out);
+  p.t_in = static_cast<const __nv_bfloat16*>(t_given);
   p.status = a.status;
 
-  const size_t smem = gemv_layout(bps, np, r_pad, a.r, phases, t_parts).total;
+  const size_t smem = gemv_layout(bps, np, lay_r, a.r, phases, t_parts).total;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(tiles), unsigned(slices), 1);
   cfg.blockDim = dim3(kGvThreads, 1, 1);
@@ -687,17 +704,26 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   // decode path can ask for), not on every call.
   auto kernel_for = [](int n8, bool f16, int tp) {
     if (f16) {
-      if (n8 == 1) return tp == 4 ? nf4_gemv<1, 2, true, 4> : (tp == 2 ? nf4_gemv<1, 2, true, 2> : nf4_gemv<1, 2, true, 1>);
-      return n8 == 2 ? nf4_gemv<2, 2, true, 1> : nf4_gemv<4, 1, true, 1>;
+      if (n8 == 1)
+        return tp == 4 ? nf4_gemv<1, 2, true, 4>
+                       : (tp == 2 ? nf4_gemv<1, 2, true, 2> : (tp == 1 ? nf4_gemv<1, 2, true, 1> : nf4_gemv<1, 2, true, 0>));
+      if (n8 == 2) return tp == 1 ? nf4_gemv<2, 2, true, 1> : nf4_gemv<2, 2, true, 0>;
+      return tp == 1 ? nf4_gemv<4, 1, true, 1> : nf4_gemv<4, 1, true, 0>;
     }
-    if (n8 == 1) return tp == 4 ? nf4_gemv<1, 2, false, 4> : (tp == 2 ? nf4_gemv<1, 2, false, 2> : nf4_gemv<1, 2, false, 1>);
-    return n8 == 2 ? nf4_gemv<2, 2, false, 1> : nf4_gemv<4, 1, false, 1>;
+    if (n8 == 1)
+      return tp == 4 ? nf4_gemv<1, 2, false, 4>
+                     : (tp == 2 ? nf4_gemv<1, 2, false, 2> : (tp == 1 ? nf4_gemv<1, 2, false, 1> : nf4_gemv<1, 2, false, 0>));
+    if (n8 == 2) return tp == 1 ? nf4_gemv<2, 2, false, 1> : nf4_gemv<2, 2, false, 0>;
+    return tp == 1 ? nf4_gemv<4, 1, false, 1> : nf4_gemv<4, 1, false, 0>;
   };
-  // one slot per instantiation: (tokens, parts) in {(8, 4), (8, 2), (8, 1), (16, 1), (32, 1)} x dtype
-  static PerDeviceOnce attr_done[10];
-  const int kind = nt8 == 1 ? (t_parts == 4 ? 0 : (t_parts == 2 ? 1 : 2)) : (nt8 == 2 ? 3 : 4);
-  const int slot = kind + (a.f16 ? 5 : 0);
+  // one slot per instantiation: (tokens, parts) in {(8, 4), (8, 2), (8, 1), (8, T given),
+  // (16, 1), (16, T given), (32, 1), (32, T given)} x dtype
+  static PerDeviceOnce attr_done[16];
+  const int kind = nt8 == 1 ? (t_parts == 4 ? 0 : (t_parts == 2 ? 1 : (t_parts == 1 ? 2 : 3)))
+                            : (nt8 == 2 ? (t_parts == 1 ? 4 : 5) : (t_parts == 1 ? 6 : 7));
+  const int slot = kind + (a.f16 ? 8 : 0);
   auto* kernel = kernel_for(nt8, a.f16 != 0, t_parts);
+  if (dry_run) return cudaSuccess;
   cudaError_t e = cudaSuccess;
   const int dev = PerDeviceOnce::current();
   if (!attr_done[slot].done(dev)) {

@@ -103,7 +103,12 @@ bool make_map_3d(CUtensorMap* map, const void* base, bool bf16, uint64_t d0, uin
 
 // Decode-shape forward (gemv.cu): one kernel for M <= 32 tokens.
 bool decode_supported(int64_t M, int64_t N, int64_t K, int r);
-cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
+// t_given: T = s x A^T [M, r] written by the kernel just before on the stream
+// (then the decode kernel is its programmatic dependent and holds no A tiles),
+// or null to compute it inside.  dry_run: check that the launch would go
+// ahead (cudaErrorNotSupported if the shape does not fit), launch nothing.
+cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches,
+                              const void* t_given = nullptr, bool dry_run = false);
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 // The F32 compute dtype (f32_gemm.cu): fp32 operands and outputs, CUDA-core fp32 FMAs.

@@ -863,7 +863,14 @@ __global__ void __launch_bounds__(kAdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
+  // A kernel launched as this one's programmatic dependent (the forward GEMM
+  // or the decode GEMV after T) may start on the SMs this grid leaves free; it
+  // waits for this grid's completion before it reads the result.  When this
+  // grid is itself launched as a dependent (T before a decode GEMV), nothing
+  // is read or written before the kernel ahead of it has completed; otherwise
+  // the wait returns at once.
   grid_dep_launch();
+  grid_dep_wait();
 
   // TMA copies: the A tile from warp 0 and the B tile from warp 2 (one warp
   // keeps only a few TMA copies going per microsecond); each arrives on the
@@ -1213,19 +1220,21 @@ bool prepare_adapter(const AdapterJob& j, uint32_t* status, AdapterLaunch* L) {
   return true;
 }
 
-cudaError_t launch_adapter(const AdapterLaunch& L, cudaStream_t st, int* launches) {
+cudaError_t launch_adapter(const AdapterLaunch& L, cudaStream_t st, int* launches, bool pdl = false) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = L.grid;
   cfg.blockDim = dim3(kAdThreads, 1, 1);
   cfg.dynamicSmemBytes = L.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = L.grid.y;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   NF4_PROF_BEGIN(st, L.prof_id);
   cudaError_t e = cudaLaunchKernelEx(&cfg, adapter_gemm, L.ma, L.mb, L.p);
   NF4_PROF_END(st, L.prof_id);
@@ -1418,14 +1427,32 @@ size_t linear_workspace_bytes(bool backward, int64_t M, int64_t N, int64_t K, in
 // first is enqueued, so a call that fails on the host enqueues nothing.
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches) {
   (void)sms;
-  if (decode_supported(a.M, a.N, a.K, a.r)) {
-    const cudaError_t d = launch_decode_fwd(a, sms, st, launches);
-    if (d != cudaErrorNotSupported) return d;
-  }
-  cudaError_t e = set_attrs();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   uint8_t* ws = a.ws + kWsHeader;
   __nv_bfloat16* T = a.t_out ? static_cast<__nv_bfloat16*>(a.t_out) : reinterpret_cast<__nv_bfloat16*>(ws);
+  if (decode_supported(a.M, a.N, a.K, a.r)) {
+    // With r > 32 the A tiles of a K slice would crowd the weight tiles out of
+    // shared memory: T comes from the adapter kernel first, and the decode
+    // kernel (its programmatic dependent) reads it.
+    const bool t_first = a.r > 32;
+    e = launch_decode_fwd(a, sms, st, launches, t_first ? T : nullptr, /*dry_run=*/true);
+    if (e == cudaSuccess) {
+      if (t_first) {
+        AdapterLaunch lt0;
+        e = set_attrs();
+        if (e != cudaSuccess) return e;
+        if (!prepare_adapter(job_T(a, T), a.status, &lt0)) return cudaErrorInvalidValue;
+        // a programmatic dependent of the kernel before (a previous decode
+        // call's tail overlaps its set-up), unless the per-kernel brackets are on
+        e = launch_adapter(lt0, st, launches, /*pdl=*/!prof_on());
+        if (e != cudaSuccess) return e;
+      }
+      return launch_decode_fwd(a, sms, st, launches, t_first ? T : nullptr, false);
+    }
+    if (e != cudaErrorNotSupported) return e;
+  }
+  e = set_attrs();
+  if (e != cudaSuccess) return e;
   AdapterLaunch lt;
   FusedLaunch lf;
   if (!prepare_adapter(job_T(a, T), a.status, &lt) || !prepare_fused(a, kFwd, T, &lf))
