@@ -610,12 +610,103 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   }
 }
 
+// T = s x A^T for a decode call (M <= 32 tokens, r <= 64) when the decode
+// kernel takes T finished: one CTA per adapter row j and group of up to 8
+// tokens, each thread a strided share of the K range for every token, fp32
+// products and sums (fixed order: the thread's own K share, then a shuffle
+// tree, then the warps in order), rounded once to the compute type.
+// Launched as a programmatic dependent: x may be the previous kernel's output.
+constexpr int kDtThreads = 256;
+constexpr int kDtTokens = 8;
+template <bool F16>
+__global__ void __launch_bounds__(kDtThreads) decode_t_kernel(
+    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ A, int M, int K, int r,
+    float s, __nv_bfloat16* __restrict__ T) {
+  constexpr int MT = kDtTokens;
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int j = blockIdx.x;
+  const int m0 = blockIdx.y * MT;
+  x += int64_t(m0) * K;
+  T += int64_t(m0) * r;
+  M = min(MT, M - m0);
+  float acc[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+  const uint4* arow = reinterpret_cast<const uint4*>(A + int64_t(j) * K);
+  for (int k8 = threadIdx.x; k8 < K / 8; k8 += kDtThreads) {
+    const uint4 av = __ldg(arow + k8);
+    const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+    float af[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&aw[e]);
+      af[2 * e] = to_f32<F16>(h[0]);
+      af[2 * e + 1] = to_f32<F16>(h[1]);
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (m >= M) break;
+      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + int64_t(m) * K) + k8);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&xw[e]);
+        acc[m] = fmaf(to_f32<F16>(h[0]), af[2 * e], acc[m]);
+        acc[m] = fmaf(to_f32<F16>(h[1]), af[2 * e + 1], acc[m]);
+      }
+    }
+  }
+  __shared__ float part[kDtThreads / 32][MT];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    if (m >= M) break;
+    float v = acc[m];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) part[warp][m] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < M) {
+    float v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kDtThreads / 32; ++w) v += part[w][threadIdx.x];
+    T[int64_t(threadIdx.x) * r + j] = from_f32<F16>(s * v);
+  }
+}
+
 }  // namespace
 
 bool decode_supported(int64_t M, int64_t N, int64_t K, int r) {
   (void)N;
   (void)K;
   return M >= 1 && M <= 32 && r <= kGvMaxR;
+}
+
+cudaError_t launch_decode_t(const LinearArgs& a, void* T, cudaStream_t st, int* launches, bool pdl) {
+  if (a.M < 1 || a.M > 32 || a.r < 1 || a.K % 8 != 0) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(a.r), unsigned((a.M + kDtTokens - 1) / kDtTokens), 1);
+  cfg.blockDim = dim3(kDtThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const auto* x = static_cast<const __nv_bfloat16*>(a.x);
+  const auto* A = static_cast<const __nv_bfloat16*>(a.A);
+  auto* t = static_cast<__nv_bfloat16*>(T);
+  const int M = int(a.M), K = int(a.K), r = a.r;
+  NF4_PROF_BEGIN(st, kKAdapterT);
+  cudaError_t e;
+  e = a.f16 ? cudaLaunchKernelEx(&cfg, decode_t_kernel<true>, x, A, M, K, r, a.s, t)
+            : cudaLaunchKernelEx(&cfg, decode_t_kernel<false>, x, A, M, K, r, a.s, t);
+  NF4_PROF_END(st, kKAdapterT);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int* launches,

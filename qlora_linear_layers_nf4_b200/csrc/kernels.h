@@ -109,6 +109,9 @@ bool decode_supported(int64_t M, int64_t N, int64_t K, int r);
 // ahead (cudaErrorNotSupported if the shape does not fit), launch nothing.
 cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches,
                               const void* t_given = nullptr, bool dry_run = false);
+// T = s x A^T [M, r] in the compute type for a decode call (M <= 32), the
+// T the decode kernel takes finished; pdl: launch as a programmatic dependent.
+cudaError_t launch_decode_t(const LinearArgs& a, void* T, cudaStream_t stream, int* launches, bool pdl);
 cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 cudaError_t launch_linear_bwd(const LinearArgs& a, int sms, cudaStream_t stream, int* launches);
 // The F32 compute dtype (f32_gemm.cu): fp32 operands and outputs, CUDA-core fp32 FMAs.

@@ -1438,13 +1438,9 @@ cudaError_t launch_linear_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
     e = launch_decode_fwd(a, sms, st, launches, t_first ? T : nullptr, /*dry_run=*/true);
     if (e == cudaSuccess) {
       if (t_first) {
-        AdapterLaunch lt0;
-        e = set_attrs();
-        if (e != cudaSuccess) return e;
-        if (!prepare_adapter(job_T(a, T), a.status, &lt0)) return cudaErrorInvalidValue;
         // a programmatic dependent of the kernel before (a previous decode
-        // call's tail overlaps its set-up), unless the per-kernel brackets are on
-        e = launch_adapter(lt0, st, launches, /*pdl=*/!prof_on());
+        // call's tail overlaps its start), unless the per-kernel brackets are on
+        e = launch_decode_t(a, T, st, launches, /*pdl=*/!prof_on());
         if (e != cudaSuccess) return e;
       }
       return launch_decode_fwd(a, sms, st, launches, t_first ? T : nullptr, false);
