@@ -864,13 +864,9 @@ __global__ void __launch_bounds__(kAdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
   // A kernel launched as this one's programmatic dependent (the forward GEMM
-  // or the decode GEMV after T) may start on the SMs this grid leaves free; it
-  // waits for this grid's completion before it reads the result.  When this
-  // grid is itself launched as a dependent (T before a decode GEMV), nothing
-  // is read or written before the kernel ahead of it has completed; otherwise
-  // the wait returns at once.
+  // after T) may start on the SMs this grid leaves free; it waits for this
+  // grid's completion before it reads the result.
   grid_dep_launch();
-  grid_dep_wait();
 
   // TMA copies: the A tile from warp 0 and the B tile from warp 2 (one warp
   // keeps only a few TMA copies going per microsecond); each arrives on the
@@ -1220,21 +1216,19 @@ bool prepare_adapter(const AdapterJob& j, uint32_t* status, AdapterLaunch* L) {
   return true;
 }
 
-cudaError_t launch_adapter(const AdapterLaunch& L, cudaStream_t st, int* launches, bool pdl = false) {
+cudaError_t launch_adapter(const AdapterLaunch& L, cudaStream_t st, int* launches) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = L.grid;
   cfg.blockDim = dim3(kAdThreads, 1, 1);
   cfg.dynamicSmemBytes = L.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = L.grid.y;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 2 : 1;
+  cfg.numAttrs = 1;
   NF4_PROF_BEGIN(st, L.prof_id);
   cudaError_t e = cudaLaunchKernelEx(&cfg, adapter_gemm, L.ma, L.mb, L.p);
   NF4_PROF_END(st, L.prof_id);
