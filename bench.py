@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the hash of the kernel source it was taken on; reported as null once the
 # source changes.
 NCU_TRAFFIC = {
-    # forward 126.1 MB, dx 177.2 MB per launch
-    "b6c61cf6b609ba98": {"fwd": 70_948_864 + 55_177_728, "dx": 157_914_880 + 19_273_728},
+    # forward 127.1 MB, dx 180.3 MB per launch
+    "0c1315b82a7b6fd3": {"fwd": 69_987_584 + 57_091_584, "dx": 162_196_224 + 18_145_536},
 }
 
 
