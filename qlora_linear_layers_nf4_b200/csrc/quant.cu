@@ -8,6 +8,7 @@
 // shuffle-xor reduction over the bs/8 lanes that hold it.
 #include <algorithm>
 #include <mutex>
+#include <utility>
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -180,6 +181,10 @@ __global__ void __launch_bounds__(256) quantize_vec_kernel(
   __shared__ EncodeTables tab;
   init_tables(tab);
   __syncthreads();
+  // Launched as a programmatic dependent: the tables above read no input;
+  // every read of w and every write comes after the previous kernel on the
+  // stream has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   uint32_t cta_max = 0;
   const Idx stride = Idx(gridDim.x) * blockDim.x;
   // Encode one word (8 elements) whose block max over the G lanes is known
@@ -324,6 +329,9 @@ __device__ __forceinline__ uint32_t dq_code(float a, float g, float s_g, bool fa
 __global__ void __launch_bounds__(256) double_quant_kernel(
     const float* __restrict__ absmax, int64_t n_blocks, const float* __restrict__ max_slots,
     int n_slots, uint8_t* __restrict__ absmax_q, float* __restrict__ absmax_scale) {
+  // a programmatic dependent of this kernel (the next quantize on the stream)
+  // may launch now: it waits for this grid before it touches memory
+  asm volatile("griddepcontrol.launch_dependents;");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t n4 = n_blocks / 4;
   const int64_t i4 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -430,6 +438,11 @@ __global__ void __launch_bounds__(256) dequant_vec_kernel(
   __shared__ float lut[16];   // 16 words in 16 banks: conflict-free for any codes
   if (threadIdx.x < 16) lut[threadIdx.x] = level(threadIdx.x);
   __syncthreads();
+  // Launched as a programmatic dependent, and lets the next one launch now:
+  // nothing above reads an input, and nothing below reads or writes memory
+  // before the previous kernel on the stream has completed.
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const float s_g = kDouble ? *absmax_scale : 0.0f;
   const Code* c = reinterpret_cast<const Code*>(codes);
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
@@ -492,6 +505,24 @@ __global__ void __launch_bounds__(256) dequant_bytes_kernel(
   }
 }
 
+// A one-dimensional launch with programmatic stream serialisation: the kernel
+// may start while the previous kernel on the stream finishes, and must touch
+// no input or output before its griddepcontrol.wait.
+template <typename... P, typename... A>
+cudaError_t launch_dependent(void (*kernel)(P...), int grid, int threads, cudaStream_t stream,
+                             A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid), 1, 1);
+  cfg.blockDim = dim3(unsigned(threads), 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 // CTAs of `kernel` (threads per CTA, no dynamic shared memory) resident on one
 // SM, from the occupancy calculator, cached per kernel and device.
 int resident_ctas(const void* kernel, int threads) {
@@ -542,11 +573,12 @@ void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes,
   if (n_full > 0 && vec) {
     const int64_t n_words = n_full * bs / 8;
     uint32_t* c32 = reinterpret_cast<uint32_t*>(codes);
+    cudaError_t launch_error = cudaSuccess;
     auto run = [&](auto kernel, auto n) {
       // one resident wave: every CTA stays for the whole pass
       const int grid = std::min(kMaxSlots - 1, grid_for(n_words, threads, sms,
                                                          resident_ctas(reinterpret_cast<const void*>(kernel), threads)));
-      kernel<<<grid, threads, 0, stream>>>(w, n, c32, absmax_out, status, max_slots);
+      launch_error = launch_dependent(kernel, grid, threads, stream, w, n, c32, absmax_out, status, max_slots);
       *n_slots = grid;
     };
     // 32-bit word indices while every index the loop forms (up to n_words plus
@@ -561,6 +593,7 @@ void launch_quantize_typed(const void* w, int64_t numel, int bs, uint8_t* codes,
       case 16: if (small) run(quantize_vec_kernel<16, IN, uint32_t>, n32); else run(quantize_vec_kernel<16, IN, int64_t>, n_words); break;
       default: if (small) run(quantize_vec_kernel<32, IN, uint32_t>, n32); else run(quantize_vec_kernel<32, IN, int64_t>, n_words); break;
     }
+    if (launch_error != cudaSuccess) return;   // the caller reads it back from cudaGetLastError
     ++*launches;
   } else if (n_full > 0) {
     const int grid = std::min(kMaxSlots - 1, grid_for(n_full, threads, sms, 8));
@@ -648,6 +681,7 @@ cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int
   const int64_t n_words = (bs % 8 == 0) ? (numel / bs) * bs / 8 : 0;
   const int64_t byte0 = n_words * 4, byte1 = (numel + 1) / 2;
   int n = 0;
+  cudaError_t launch_error = cudaSuccess;
   NF4_PROF_BEGIN(stream, kKDequantize);
   if (n_words > 0) {
     // units of E elements: 4 for fp32 output, 8 for bf16 / f16
@@ -658,8 +692,8 @@ cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int
     auto run = [&](auto kernel, auto* o) {
       const int grid = grid_for((n_units + kDqSteps - 1) / kDqSteps, threads, sms,
                                 resident_ctas(reinterpret_cast<const void*>(kernel), threads));
-      kernel<<<grid, threads, 0, stream>>>(w.codes, n_units, shift, units_per_block, w.absmax,
-                                           w.absmax_q, w.absmax_scale, o);
+      launch_error = launch_dependent(kernel, grid, threads, stream, w.codes, n_units, shift, units_per_block,
+                                      w.absmax, w.absmax_q, w.absmax_scale, o);
     };
     if (out_dtype == NF4_F32) {
       float* o = reinterpret_cast<float*>(out);
@@ -673,7 +707,7 @@ cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int
     }
     ++n;
   }
-  if (byte1 > byte0) {
+  if (byte1 > byte0 && launch_error == cudaSuccess) {
     const int grid = grid_for(byte1 - byte0, threads, sms, 8);
 #define NF4_DQB_LAUNCH(T, D)                                                               \
   dequant_bytes_kernel<T, D><<<grid, threads, 0, stream>>>(w.codes, byte0, byte1, numel, bs, \
@@ -692,6 +726,7 @@ cudaError_t launch_dequantize(const nf4_weight& w, int out_dtype, void* out, int
   }
   NF4_PROF_END(stream, kKDequantize);
   cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = launch_error;
   if (e == cudaSuccess) *launches += n;
   return e;
 }
