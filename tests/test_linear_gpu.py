@@ -249,11 +249,24 @@ def test_decode_shapes(cuda_device, case):
 @pytest.mark.parametrize("m,rank,dq", [
     (17, 16, True), (24, 16, True), (32, 16, True), (32, 16, False),
     (5, 8, True), (32, 8, True), (9, 64, True), (32, 64, False),
-    (4, 32, True), (8, 24, False), (3, 48, True), (1, 64, True),
+    (4, 32, True), (8, 24, False), (3, 48, True), (1, 64, True), (12, 32, True),
 ])
 def test_decode_wide_and_rank_edges(cuda_device, m, rank, dq):
     case = WL.LinearCase(f"decode 4096x4096 M={m} r={rank}", n=4096, k=4096, m=m, r=rank,
                          alpha=2.0 * rank, seed=2, double_quant=dq)
+    for zero_w in (False, True):
+        r = Run(case, cuda_device, zero_w=zero_w, bias=not zero_w)
+        r.check_forward()
+        r.check_backward()
+
+
+# Decode with K = 64 (one K block: one slice, so the final sum has a single
+# lane per output) and with K = 192 (three blocks: two slices, the second with
+# one block).
+@pytest.mark.parametrize("m,n,k", [(3, 256, 64), (16, 384, 64), (2, 256, 192)])
+def test_decode_few_k_blocks(cuda_device, m, n, k):
+    case = WL.LinearCase(f"decode {n}x{k} M={m}", n=n, k=k, m=m, r=16, alpha=32.0,
+                         seed=7000 + m + n + k, double_quant=True)
     for zero_w in (False, True):
         r = Run(case, cuda_device, zero_w=zero_w, bias=not zero_w)
         r.check_forward()
