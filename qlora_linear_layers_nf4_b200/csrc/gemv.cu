@@ -719,11 +719,13 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
   const int phases = kGvWWarps / (8 / rg);
   const int np = 8 * nt8;
   const int r_pad = (a.r + 15) / 16 * 16;
-  // With at most 8 tokens and one or two adapter row groups, the x A^T of a
-  // slice is split over the four adapter warps by K block as well, so it
-  // finishes with the weight rows (more tokens keep the W warps busier).
+  // With one or two adapter row groups, the x A^T of a slice is split over the
+  // four adapter warps by K block as well, so it finishes with the weight rows
+  // (with 17..32 tokens into two parts only: four would not leave room for the
+  // weight tiles).
   const int t_groups = r_pad / 16;
-  const int t_parts = t_given != nullptr ? 0 : ((nt8 == 1 && t_groups <= 2) ? 4 / t_groups : 1);
+  const int t_parts = t_given != nullptr ? 0
+                      : (t_groups > 2 ? 1 : (nt8 <= 2 ? 4 / t_groups : (t_groups == 1 ? 2 : 1)));
   const int lay_r = t_given != nullptr ? 0 : r_pad;   // A tile rows held in shared memory
   // K slices: one wave of one CTA per SM where possible, and everything a CTA
   // reads fits in its shared memory at once.
@@ -798,21 +800,25 @@ cudaError_t launch_decode_fwd(const LinearArgs& a, int sms, cudaStream_t st, int
       if (n8 == 1)
         return tp == 4 ? nf4_gemv<1, 2, true, 4>
                        : (tp == 2 ? nf4_gemv<1, 2, true, 2> : (tp == 1 ? nf4_gemv<1, 2, true, 1> : nf4_gemv<1, 2, true, 0>));
-      if (n8 == 2) return tp == 1 ? nf4_gemv<2, 2, true, 1> : nf4_gemv<2, 2, true, 0>;
-      return tp == 1 ? nf4_gemv<4, 1, true, 1> : nf4_gemv<4, 1, true, 0>;
+      if (n8 == 2)
+        return tp == 4 ? nf4_gemv<2, 2, true, 4>
+                       : (tp == 2 ? nf4_gemv<2, 2, true, 2> : (tp == 1 ? nf4_gemv<2, 2, true, 1> : nf4_gemv<2, 2, true, 0>));
+      return tp == 2 ? nf4_gemv<4, 1, true, 2> : (tp == 1 ? nf4_gemv<4, 1, true, 1> : nf4_gemv<4, 1, true, 0>);
     }
     if (n8 == 1)
       return tp == 4 ? nf4_gemv<1, 2, false, 4>
                      : (tp == 2 ? nf4_gemv<1, 2, false, 2> : (tp == 1 ? nf4_gemv<1, 2, false, 1> : nf4_gemv<1, 2, false, 0>));
-    if (n8 == 2) return tp == 1 ? nf4_gemv<2, 2, false, 1> : nf4_gemv<2, 2, false, 0>;
-    return tp == 1 ? nf4_gemv<4, 1, false, 1> : nf4_gemv<4, 1, false, 0>;
+    if (n8 == 2)
+      return tp == 4 ? nf4_gemv<2, 2, false, 4>
+                     : (tp == 2 ? nf4_gemv<2, 2, false, 2> : (tp == 1 ? nf4_gemv<2, 2, false, 1> : nf4_gemv<2, 2, false, 0>));
+    return tp == 2 ? nf4_gemv<4, 1, false, 2> : (tp == 1 ? nf4_gemv<4, 1, false, 1> : nf4_gemv<4, 1, false, 0>);
   };
-  // one slot per instantiation: (tokens, parts) in {(8, 4), (8, 2), (8, 1), (8, T given),
-  // (16, 1), (16, T given), (32, 1), (32, T given)} x dtype
-  static PerDeviceOnce attr_done[16];
-  const int kind = nt8 == 1 ? (t_parts == 4 ? 0 : (t_parts == 2 ? 1 : (t_parts == 1 ? 2 : 3)))
-                            : (nt8 == 2 ? (t_parts == 1 ? 4 : 5) : (t_parts == 1 ? 6 : 7));
-  const int slot = kind + (a.f16 ? 8 : 0);
+  // one slot per instantiation: (tokens, parts) in {8, 16, 32} x {4, 2, 1, T given}
+  // (32 tokens: 4 parts unused), times the dtype
+  static PerDeviceOnce attr_done[24];
+  const int part_kind = t_parts == 4 ? 0 : (t_parts == 2 ? 1 : (t_parts == 1 ? 2 : 3));
+  const int kind = (nt8 == 1 ? 0 : (nt8 == 2 ? 4 : 8)) + part_kind;
+  const int slot = kind + (a.f16 ? 12 : 0);
   auto* kernel = kernel_for(nt8, a.f16 != 0, t_parts);
   if (dry_run) return cudaSuccess;
   cudaError_t e = cudaSuccess;
