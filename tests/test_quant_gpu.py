@@ -171,3 +171,36 @@ def test_empty_input(cuda_device):
     q = Q.quantize(torch.zeros((0, 64), dtype=torch.float32, device=cuda_device), 64, True)
     torch.cuda.synchronize()
     assert q.absmax_scale.item() == 0.0
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_chained_calls_without_sync(cuda_device, dq):
+    """Quantize and dequantize back to back on one stream, each call reading the
+    previous call's output and the quantize calls sharing one workspace, with no
+    synchronisation in between (the kernels are launched as programmatic
+    dependents of one another): every round is bit-exact against the oracle's
+    own chain of the same rounds."""
+    import torch
+    Q = _q()
+    w = WL.draw_weight((1024, 1024), seed=31)
+    rounds = 4
+    qs, outs = [], []
+    cur = _to_dev(w, cuda_device)
+    for _ in range(rounds):
+        q = Q.quantize(cur, block_size=64, double_quant=dq, keep_absmax=True)
+        cur = Q.dequantize(q, "f32")
+        qs.append(q)
+        outs.append(cur)
+    torch.cuda.synchronize()
+    ref_w = w
+    for k in range(rounds):
+        ref = O.quantize(ref_w, 64, double=dq)
+        q = qs[k]
+        assert np.array_equal(q.codes.cpu().numpy()[: ref["codes"].size], ref["codes"]), f"round {k}: codes"
+        assert np.array_equal(q.absmax.cpu().numpy()[: ref["absmax"].size].view(np.uint32),
+                              ref["absmax"].view(np.uint32)), f"round {k}: absmax"
+        if dq:
+            assert np.array_equal(q.absmax_q.cpu().numpy()[: ref["absmax_q"].size], ref["absmax_q"])
+            assert q.absmax_scale.cpu().numpy()[0].view(np.uint32) == np.float32(ref["absmax_scale"]).view(np.uint32)
+        ref_w = O.dequantize(ref, "f32").reshape(w.shape)
+        assert np.array_equal(outs[k].cpu().numpy().view(np.uint32), ref_w.view(np.uint32)), f"round {k}: dequant"
