@@ -24,7 +24,14 @@
  *   Streams    `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *              default stream).  All work is enqueued on it; buffers must stay
  *              alive until it completes.  Nothing synchronizes except
- *              nf4_read_status.
+ *              nf4_read_status.  Several kernels (quantize, double quant,
+ *              dequantize, decode, the forward GEMM) are launched with
+ *              programmatic stream serialisation: each touches no input or
+ *              output before the previous kernel on the stream has completed,
+ *              and some let the kernel after them launch early.  A kernel the
+ *              caller launches after a call with that attribute must wait
+ *              (griddepcontrol.wait / cudaGridDependencySynchronize) before it
+ *              reads the call's outputs, as any such kernel must.
  *   Layouts    Row-major, densely packed.  W is [rows = N out, cols = K in].
  *              x is [M, K], A is [r, K], B is [N, r], y and dy are [M, N].
  *   Alignment  Device pointers must be 16-byte aligned unless the entry
