@@ -26,9 +26,10 @@
  *              alive until it completes.  Nothing synchronizes except
  *              nf4_read_status.  Several kernels (quantize, double quant,
  *              dequantize, decode, the forward GEMM) are launched with
- *              programmatic stream serialisation: each touches no input or
- *              output before the previous kernel on the stream has completed,
- *              and some let the kernel after them launch early.  A kernel the
+ *              programmatic stream serialisation: each reads nothing that
+ *              earlier work on the stream may still be writing (and writes
+ *              nothing it may still be reading) before that work has
+ *              completed, and some let the kernel after them launch early.  A kernel the
  *              caller launches after a call with that attribute must wait
  *              (griddepcontrol.wait / cudaGridDependencySynchronize) before it
  *              reads the call's outputs, as any such kernel must.
