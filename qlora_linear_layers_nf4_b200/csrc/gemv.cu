@@ -81,7 +81,8 @@ struct GemvParams {
 //   xs     [4 G blocks][NP token rows][128 B], 128-byte swizzle
 //   as     [4 G blocks][r_pad adapter rows][128 B], 128-byte swizzle
 //   bs     [128 W rows][r] bf16 (this tile's rows of B)
-//   scales [128 rows][kGvMaxBlocks] fp32                 8 KB
+//   scales [kGvMaxBlocks][128 rows] fp32                 8 KB (block-major:
+//          the eight rows a warp's lanes read at once sit in eight banks)
 //   recv   [slice][128 / S rows][NP] fp32: partials pushed by the cluster
 //   tpart  [t_parts][r_pad][NP] fp32: this slice's x A^T, in t_parts partial
 //          sums over interleaved K blocks
@@ -356,22 +357,28 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   }
 
   {
-    float* srow_dst = scales + srow * kGvMaxBlocks;
+    float* srow_dst = scales + srow;   // block b of this row at srow_dst[b * kGvRows]
     if (svec && dq) {
       if (threadIdx.x < kGvRows) {
         const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
-        for (int b = 0; b < 16; ++b) srow_dst[b] = __fmul_rn(float((w[b >> 2] >> (8 * (b & 3))) & 0xffu), s_g);
+        for (int b = 0; b < 16; ++b)
+          srow_dst[b * kGvRows] = __fmul_rn(float((w[b >> 2] >> (8 * (b & 3))) & 0xffu), s_g);
       }
     } else if (svec) {
-      if (threadIdx.x < 4 * kGvRows)
-        *reinterpret_cast<uint4*>(srow_dst + 4 * (threadIdx.x >> 7)) = sv;
+      if (threadIdx.x < 4 * kGvRows) {
+        const int b0 = 4 * (threadIdx.x >> 7);
+        srow_dst[(b0 + 0) * kGvRows] = __uint_as_float(sv.x);
+        srow_dst[(b0 + 1) * kGvRows] = __uint_as_float(sv.y);
+        srow_dst[(b0 + 2) * kGvRows] = __uint_as_float(sv.z);
+        srow_dst[(b0 + 3) * kGvRows] = __uint_as_float(sv.w);
+      }
     } else {
 #pragma unroll
       for (int j = 0; j < kScaleRegs; ++j) {
         const int b = (threadIdx.x >> 7) + kScaleSteps * j;
         const float v = dq ? __fmul_rn(float(sc_raw[j]), s_g) : __uint_as_float(sc_raw[j]);
-        if (b < kGvMaxBlocks) srow_dst[b] = v;
+        if (b < kGvMaxBlocks) srow_dst[b * kGvRows] = v;
       }
     }
   }
@@ -412,8 +419,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
           afr[k][2] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wa, j + 1, lane_off));
           afr[k][3] = *reinterpret_cast<const uint32_t*>(lut_bytes + lut_off(wb, j + 1, lane_off));
         }
-        const float s0 = scales[wr0 * kGvMaxBlocks + b];
-        const float s1 = scales[(wr0 + 1) * kGvMaxBlocks + b];
+        const float s0 = scales[b * kGvRows + wr0];
+        const float s1 = scales[b * kGvRows + wr0 + 1];
 #pragma unroll
         for (int t = 0; t < NT8; ++t) {
           float blk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
