@@ -947,8 +947,11 @@ __global__ void __launch_bounds__(kAdThreads, 1)
     tc_fence_after();
     const int quad = warp & 3;
     const int row = mo0 + quad * 32 + lane;
-    // partial tile [128][NP] fp32 over the (now idle) stage buffers
-    float* dst = reinterpret_cast<float*>(smem) + (quad * 32 + lane) * p.NP;
+    // partial tile [128][NP] fp32 over the (now idle) stage buffers; the
+    // 16-byte chunk v of row R sits at chunk v ^ (R & 7), so the eight rows a
+    // quarter-warp writes at once land in eight different bank groups
+    const int prow = quad * 32 + lane;
+    float* dst = reinterpret_cast<float*>(smem) + prow * p.NP;
     for (int c = 0; c < p.NP / 32; ++c) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + (uint32_t(quad * 32) << 16) + c * 32, v);
@@ -964,13 +967,13 @@ __global__ void __launch_bounds__(kAdThreads, 1)
           if (p.slices == 1) {
             if (col < p.r) adapter_store4(p, row, col, f);
           } else {
-            reinterpret_cast<float4*>(dst + col)[0] = f;
+            reinterpret_cast<float4*>(dst + 4 * ((col >> 2) ^ (prow & 7)))[0] = f;
           }
         }
       } else if (p.slices > 1) {
 #pragma unroll
         for (int g = 0; g < 8; ++g)
-          reinterpret_cast<float4*>(dst + c * 32 + 4 * g)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+          reinterpret_cast<float4*>(dst + 4 * ((c * 8 + g) ^ (prow & 7)))[0] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
   }
@@ -998,7 +1001,7 @@ __global__ void __launch_bounds__(kAdThreads, 1)
         cv = i % vec_per_row;
       }
       const int trow = int(q) * rows_per + rr;
-      const uint32_t off = uint32_t((trow * p.NP + 4 * cv) * 4);
+      const uint32_t off = uint32_t((trow * p.NP + 4 * (cv ^ (trow & 7))) * 4);   // the parking swizzle
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int sl = 0; sl < p.slices; ++sl) {
         const float4 v = ld_shared_cluster_f4(mapa_shared(base + off, uint32_t(sl)));
