@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the hash of the kernel source it was taken on; reported as null once the
 # source changes.
 NCU_TRAFFIC = {
-    # forward 127.1 MB, dx 180.3 MB per launch
-    "0c1315b82a7b6fd3": {"fwd": 69_987_584 + 57_091_584, "dx": 162_196_224 + 18_145_536},
+    # forward 127.4 MB, dx 181.0 MB per launch
+    "0afa7f14ba671346": {"fwd": 72_147_712 + 55_230_976, "dx": 162_442_240 + 18_569_984},
 }
 
 
