@@ -10,19 +10,22 @@
 //   - a CTA owns 128 W rows and one K slice.  Its block scales are requested
 //     first (plain loads, so they are not queued behind the weight bytes),
 //     then every code tile, x tile and A tile of the slice by TMA, one
-//     mbarrier per 64-wide K block, so compute starts on the first block to
-//     land;
+//     mbarrier per group of four 64-wide K blocks (one 128-byte code box), so
+//     compute starts on the first group to land.  The scales sit in shared
+//     memory block-major, so the eight rows a warp reads at once use eight
+//     banks;
 //   - a 4-bit pair becomes two bf16 levels with one shared-memory lookup in a
 //     256-entry table replicated per lane (conflict-free); the block scale is
 //     applied to each 64-wide block's fp32 partial, not to every element;
 //   - the dequantized values never leave registers: they are the A fragments
 //     of mma.sync m16n8k16 with x as B (the K order inside each block is
 //     permuted identically for both so a thread's fragments are contiguous
-//     bytes).  A warp takes one K block at a time for two 16-row groups, so
-//     each x fragment it loads serves both;
+//     bytes).  With up to 16 tokens a warp takes one K block at a time for
+//     two 16-row groups, so each x fragment it loads serves both;
 //   - x A^T (the slice's share of the adapter activation) is computed by four
-//     more warps from the same x tiles; its product with the tile's B rows is
-//     one more short MMA chain on the W-row accumulators;
+//     more warps from the same x tiles, split by K block when r is small; its
+//     product with the tile's B rows is one more short MMA chain on the W-row
+//     accumulators (or T comes finished from a small kernel before, r > 32);
 //   - the S K-slices of a row tile are one thread-block cluster.  CTA q owns
 //     rows [q 128/S, (q+1) 128/S) of the tile: every CTA pushes its partial
 //     for those rows into CTA q's shared memory and arrives on CTA q's
